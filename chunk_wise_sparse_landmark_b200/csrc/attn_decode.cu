@@ -1,0 +1,309 @@
+// Hierarchical-softmax sparse attention for decode (one new token per
+// sequence), split across CTAs.
+//
+// hyper.ai summary of arXiv 2607.02980 (HiLS-Attention), section 方法
+// (Method): token weight w_{i,j} = exp(s_ij)/Z_{i,c(j)} * exp(s^_{i,c(j)})/Z^_i,
+// Z^_i = sum_c exp(s^_{i,c}) + Z_{i,swa}; section 实验 (Experiments) reports
+// sublinear decode latency — the token touches only its K chunks and its
+// window.
+//
+// Work unit = one 64-key (S-key) tile: either a selected chunk or one chunk of
+// the window.  Per (sequence, KV group) the K + n_w units are dealt to
+// `nsplit` CTAs; each CTA serves all G query heads of the group, so every key
+// and value tile is read from HBM exactly once.  A unit contributes
+// e^{a} * o to the numerator and e^{a} * z to the denominator, where for a
+// selected chunk a = s^ - log l, z = l, and for a window tile a = m, z = l
+// (m = tile max, l = sum e^{s-m}, o = sum e^{s-m} v).  Each CTA folds its units
+// with a running maximum and writes one (M, den, num[d]) record per head to the
+// workspace; a second kernel folds the records of a head and divides.
+// Tiles arrive through 1-D bulk copies (TMA) into a two-stage shared-memory
+// ring; every wait is bounded.
+#include "launch.h"
+
+namespace hils {
+namespace {
+
+constexpr int kThreads = 256;
+
+template <typename T, int D, int S, int G>
+struct DecSmem {
+  alignas(128) T kt[2][S * D];
+  alignas(128) T vt[2][S * D];
+  float qs[G][D];
+  float p[G][S];
+  float a[G], z[G];
+  uint64_t full[2];
+};
+
+// shared-memory position of element e of key row j, rotated so that the 16-byte
+// vectors of consecutive rows start in different banks
+template <typename T, int D>
+HILS_DI const T* row_ptr(const T* tile, int j) { return tile + j * D; }
+
+template <typename T, int D, int S, int G>
+__global__ void __launch_bounds__(kThreads) attn_decode_partial(Shape s, const T* __restrict__ q,
+                                                                const T* __restrict__ k, const T* __restrict__ v,
+                                                                const int32_t* __restrict__ idx,
+                                                                const float* __restrict__ s_sel,
+                                                                float* __restrict__ ws, int nsplit, DevCtx ctx) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  auto& sm = *reinterpret_cast<DecSmem<T, D, S, G>*>(smem_raw);
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int L = s.N, pos = L - 1, cur = pos / S;
+  const int ncand = max(0, cur - s.nw + 1);
+  const int wc0 = max(0, cur - s.nw + 1);        // first window chunk
+  const int nwin = cur - wc0 + 1;                 // window tiles
+  const int nunits = s.K + nwin;
+  const int32_t* ir = idx + ((long long)b * s.Hkv + g) * s.K;
+  const long long kvbase = ((long long)b * s.Hkv + g) * (long long)L * D;
+
+  for (int e = tid; e < G * D; e += kThreads)
+    sm.qs[e / D][e % D] = to_f32(q[((long long)b * s.Hq + g * G + e / D) * D + e % D]);
+  if (tid == 0) {
+    mbar_init(&sm.full[0], 1);
+    mbar_init(&sm.full[1], 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  // this CTA's units: u = split, split + nsplit, ... ; resolve each to a key range
+  auto unit_keys = [&](int u, int& j0, int& nk, bool& sel, int& slot) -> bool {
+    if (u < s.K) {
+      const int c = ir[u];
+      sel = true;
+      slot = u;
+      if (c < 0) return false;
+      if (c >= ncand) {
+        if (tid == 0) raise_status(ctx, kStatusBadIndex);
+        return false;
+      }
+      j0 = c * S;
+      nk = S;
+      return true;
+    }
+    const int wc = wc0 + (u - s.K);
+    sel = false;
+    slot = -1;
+    j0 = wc * S;
+    nk = min(S, L - j0);
+    return true;
+  };
+  bool inflight[2] = {false, false};  // meaningful in thread 0
+  auto issue = [&](int stage, int j0, int nk) {
+    if (ctx.inject == 1) return;  // test hook: no copy, the wait below must run out
+    inflight[stage] = true;
+    fence_proxy_async_shared();
+    const uint32_t bytes = (uint32_t)(nk * D * sizeof(T));
+    mbar_arrive_expect_tx(&sm.full[stage], 2 * bytes);
+    tma_load_1d(sm.kt[stage], k + kvbase + (long long)j0 * D, bytes, &sm.full[stage]);
+    tma_load_1d(sm.vt[stage], v + kvbase + (long long)j0 * D, bytes, &sm.full[stage]);
+  };
+
+  // running fold per head, thread (h, e) owns num for dims e, e + 128 ... via loop
+  float Mh[G], den[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    Mh[h] = -INFINITY;
+    den[h] = 0.f;
+  }
+  constexpr int OUTS = (G * D + kThreads - 1) / kThreads;  // outputs per thread
+  float num[OUTS];
+#pragma unroll
+  for (int r = 0; r < OUTS; ++r) num[r] = 0.f;
+
+  // collect the list of live units first (uniform across the CTA)
+  int ulist[16];
+  int nu = 0;
+  for (int u = split; u < nunits && nu < 16; u += nsplit) {
+    int j0, nk, slot;
+    bool sel;
+    if (unit_keys(u, j0, nk, sel, slot)) ulist[nu++] = u;
+  }
+  uint32_t phase[2] = {0u, 0u};
+  if (tid == 0 && nu > 0) {
+    int j0, nk, slot;
+    bool sel;
+    unit_keys(ulist[0], j0, nk, sel, slot);
+    issue(0, j0, nk);
+  }
+  bool alive = true;  // CTA-wide: every thread sees the same value
+  for (int x = 0; x < nu; ++x) {
+    const int stage = x & 1;
+    int j0, nk, slot;
+    bool sel;
+    unit_keys(ulist[x], j0, nk, sel, slot);
+    if (tid == 0 && x + 1 < nu) {
+      int j0n, nkn, sln;
+      bool seln;
+      unit_keys(ulist[x + 1], j0n, nkn, seln, sln);
+      issue(stage ^ 1, j0n, nkn);
+    }
+    const bool landed = mbar_wait(&sm.full[stage], phase[stage], ctx);
+    if (landed) inflight[stage] = false;
+    phase[stage] ^= 1u;
+    if (!__syncthreads_and(landed)) {
+      alive = false;
+      break;
+    }
+    // logits: thread per (h, j)
+    for (int p = tid; p < G * S; p += kThreads) {
+      const int h = p / S, j = p % S;
+      float acc = -INFINITY;
+      if (j < nk) {
+        const T* kr = sm.kt[stage] + j * D;
+        acc = 0.f;
+        // rotated start so that lanes of a warp hit different banks
+#pragma unroll 4
+        for (int t = 0; t < D; ++t) {
+          const int e = (t + j * 8) & (D - 1);
+          acc = fmaf(sm.qs[h][e], to_f32(kr[e]), acc);
+        }
+        acc *= s.scale;
+      }
+      sm.p[h][j] = acc;
+    }
+    __syncthreads();
+    for (int h = warp; h < G; h += kThreads / 32) {
+      float m = -INFINITY;
+      for (int j = lane; j < S; j += 32) m = fmaxf(m, sm.p[h][j]);
+      m = warp_max(m);
+      float l = 0.f;
+      for (int j = lane; j < S; j += 32) {
+        const float e = j < nk ? expf(sm.p[h][j] - m) : 0.f;
+        sm.p[h][j] = e;
+        l += e;
+      }
+      l = warp_sum(l);
+      if (lane == 0) {
+        sm.a[h] = sel ? s_sel[((long long)b * s.Hq + g * G + h) * s.K + slot] - logf(l) : m;
+        sm.z[h] = l;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < OUTS; ++r) {
+      const int o = tid + r * kThreads;
+      if (o < G * D) {
+        const int h = o / D, e = o % D;
+        float acc = 0.f;
+        for (int j = 0; j < nk; ++j) acc = fmaf(sm.p[h][j], to_f32(sm.vt[stage][j * D + e]), acc);
+        const float a = sm.a[h];
+        const float Mn = fmaxf(Mh[h], a);
+        const float cf = expf(Mh[h] - Mn), cu = expf(a - Mn);
+        num[r] = num[r] * cf + cu * acc;
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float a = sm.a[h];
+      const float Mn = fmaxf(Mh[h], a);
+      den[h] = den[h] * expf(Mh[h] - Mn) + expf(a - Mn) * sm.z[h];
+      Mh[h] = Mn;
+    }
+    __syncthreads();  // stage may now be refilled
+  }
+  if (!alive) {
+    // a wait ran out: let copies this CTA issued land before its shared memory
+    // is released (bounded as well), then leave the record undefined
+    if (tid == 0)
+      for (int st2 = 0; st2 < 2; ++st2)
+        if (inflight[st2]) mbar_wait(&sm.full[st2], phase[st2], ctx);
+    return;
+  }
+  // record: [B, Hq, nsplit, D + 2] = (M, den, num[D])
+#pragma unroll
+  for (int r = 0; r < OUTS; ++r) {
+    const int o = tid + r * kThreads;
+    if (o < G * D) {
+      const int h = o / D, e = o % D;
+      float* rec = ws + (((long long)b * s.Hq + g * G + h) * nsplit + split) * (D + 2);
+      rec[2 + e] = num[r];
+      if (e == 0) {
+        rec[0] = Mh[h];
+        rec[1] = den[h];
+      }
+    }
+  }
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(D) attn_decode_merge(Shape s, const float* __restrict__ ws, T* __restrict__ out,
+                                                       int nsplit) {
+  const long long bh = blockIdx.x;
+  const int e = threadIdx.x;
+  const float* rec = ws + bh * nsplit * (D + 2);
+  float M = -INFINITY;
+  for (int x = 0; x < nsplit; ++x) M = fmaxf(M, rec[x * (D + 2)]);
+  float num = 0.f, den = 0.f;
+  for (int x = 0; x < nsplit; ++x) {
+    const float m = rec[x * (D + 2)];
+    if (m == -INFINITY) continue;
+    const float w = expf(m - M);
+    den += w * rec[x * (D + 2) + 1];
+    num += w * rec[x * (D + 2) + 2 + e];
+  }
+  out[bh * D + e] = from_f32<T>(num / den);
+}
+
+int pick_nsplit(const Shape& s) {
+  const int cur = (s.N - 1) / s.S;
+  const int nwin = cur - max(0, cur - s.nw + 1) + 1;
+  const int nunits = s.K + nwin;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int groups = s.B * s.Hkv;
+  int nsplit = (sms * 4 + groups - 1) / groups;
+  // at most 16 units per CTA, at least one unit per CTA
+  nsplit = max(nsplit, (nunits + 15) / 16);
+  nsplit = min(nsplit, nunits);
+  return max(nsplit, 1);
+}
+
+template <typename T, int D, int S, int G>
+cudaError_t go(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx, const float* s_sel,
+               void* out, void* ws, cudaStream_t st, const DevCtx& ctx) {
+  const int nsplit = pick_nsplit(s);
+  const size_t smem = sizeof(DecSmem<T, D, S, G>);
+  auto kern = attn_decode_partial<T, D, S, G>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  kern<<<dim3(nsplit, s.Hkv, s.B), kThreads, smem, st>>>(s, (const T*)q, (const T*)k, (const T*)v, idx, s_sel,
+                                                         (float*)ws, nsplit, ctx);
+  attn_decode_merge<T, D><<<s.B * s.Hq, D, 0, st>>>(s, (const float*)ws, (T*)out, nsplit);
+  return cudaGetLastError();
+}
+
+template <typename T, int D, int S>
+cudaError_t go_g(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx, const float* s_sel,
+                 void* out, void* ws, cudaStream_t st, const DevCtx& ctx) {
+  switch (s.G) {
+    case 1: return go<T, D, S, 1>(s, q, k, v, idx, s_sel, out, ws, st, ctx);
+    case 2: return go<T, D, S, 2>(s, q, k, v, idx, s_sel, out, ws, st, ctx);
+    case 4: return go<T, D, S, 4>(s, q, k, v, idx, s_sel, out, ws, st, ctx);
+    case 8: return go<T, D, S, 8>(s, q, k, v, idx, s_sel, out, ws, st, ctx);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+size_t decode_attn_workspace(const Shape& s) {
+  const int nsplit = pick_nsplit(s);
+  return (size_t)s.B * s.Hq * nsplit * (s.d + 2) * sizeof(float);
+}
+
+cudaError_t launch_attn_decode(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
+                               const float* s_sel, void* out, void* ws, cudaStream_t st, const DevCtx& ctx) {
+  if (s.dtype == 0) {
+    if (s.d == 64 && s.S == 32) return go_g<float, 64, 32>(s, q, k, v, idx, s_sel, out, ws, st, ctx);
+    if (s.d == 64 && s.S == 64) return go_g<float, 64, 64>(s, q, k, v, idx, s_sel, out, ws, st, ctx);
+    if (s.d == 128 && s.S == 64) return go_g<float, 128, 64>(s, q, k, v, idx, s_sel, out, ws, st, ctx);
+    if (s.d == 128 && s.S == 32) return go_g<float, 128, 32>(s, q, k, v, idx, s_sel, out, ws, st, ctx);
+  } else {
+    if (s.d == 128 && s.S == 64) return go_g<__nv_bfloat16, 128, 64>(s, q, k, v, idx, s_sel, out, ws, st, ctx);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace hils

@@ -1,0 +1,255 @@
+// C ABI of libhils.so (declared in include/hils.h): argument validation,
+// dispatch to the kernels, the per-device status word and error strings.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "hils.h"
+#include "launch.h"
+
+namespace hils {
+namespace {
+
+__device__ unsigned g_status_word;  // per device: bits of kStatus*
+
+thread_local char g_err[512] = "";
+long long g_wait_budget = 0;  // 0 = default
+int g_inject = 0;
+std::mutex g_mu;
+unsigned* g_status_ptr[64] = {nullptr};
+
+hils_status_t fail(hils_status_t st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+hils_status_t cuda_fail(cudaError_t e, const char* where) {
+  return fail(HILS_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+// Resolve the device address of this device's status word once per device.
+hils_status_t dev_ctx(DevCtx* ctx) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(HILS_ERR_CUDA, "device ordinal %d out of range", dev);
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_status_ptr[dev]) {
+      void* p = nullptr;
+      e = cudaGetSymbolAddress(&p, g_status_word);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status)");
+      g_status_ptr[dev] = (unsigned*)p;
+    }
+    ctx->status = g_status_ptr[dev];
+  }
+  // ~2 s at 2 GHz unless overridden by the test hook
+  ctx->wait_budget = g_wait_budget > 0 ? g_wait_budget : 4000000000LL;
+  ctx->inject = g_inject;
+  return HILS_OK;
+}
+
+bool aligned16(const void* p) { return p && ((uintptr_t)p & 15u) == 0; }
+
+hils_status_t make_shape(const hils_config_t* cfg, Shape* s, bool decode) {
+  if (!cfg) return fail(HILS_ERR_INVALID_ARG, "cfg is NULL");
+  const hils_config_t& c = *cfg;
+  if (c.batch < 1 || c.seq_len < 1 || c.n_q_heads < 1 || c.n_kv_heads < 1 || c.head_dim < 1 || c.chunk < 1 ||
+      c.window < 1 || c.top_k < 1)
+    return fail(HILS_ERR_INVALID_ARG, "sizes must be positive (B=%d N=%d Hq=%d Hkv=%d d=%d S=%d W=%d K=%d)",
+                c.batch, c.seq_len, c.n_q_heads, c.n_kv_heads, c.head_dim, c.chunk, c.window, c.top_k);
+  if (c.n_q_heads % c.n_kv_heads) return fail(HILS_ERR_INVALID_ARG, "Hq %% Hkv != 0");
+  if (c.window % c.chunk || c.window < c.chunk) return fail(HILS_ERR_INVALID_ARG, "W must be a positive multiple of S");
+  if (c.dtype != HILS_F32 && c.dtype != HILS_BF16) return fail(HILS_ERR_INVALID_ARG, "unknown dtype %d", c.dtype);
+  if (c.query_block < 0) return fail(HILS_ERR_INVALID_ARG, "query_block < 0");
+  if (!(c.scale >= 0.f) || isinf(c.scale)) return fail(HILS_ERR_INVALID_ARG, "scale must be finite and >= 0");
+  s->B = c.batch;
+  s->N = c.seq_len;
+  s->Hq = c.n_q_heads;
+  s->Hkv = c.n_kv_heads;
+  s->G = c.n_q_heads / c.n_kv_heads;
+  s->d = c.head_dim;
+  s->S = c.chunk;
+  s->W = c.window;
+  s->nw = c.window / c.chunk;
+  s->K = c.top_k;
+  s->C = c.seq_len / c.chunk;
+  s->M = c.query_block;
+  s->scale = c.scale > 0.f ? c.scale : 1.0f / sqrtf((float)c.head_dim);
+  s->dtype = c.dtype;
+  // kernel coverage
+  const bool g_ok = s->G == 1 || s->G == 2 || s->G == 4 || s->G == 8;
+  if (!g_ok) return fail(HILS_ERR_UNSUPPORTED, "G = Hq/Hkv = %d not in {1,2,4,8}", s->G);
+  if (s->K > 64) return fail(HILS_ERR_UNSUPPORTED, "K = %d > 64", s->K);
+  if (s->nw > 32) return fail(HILS_ERR_UNSUPPORTED, "W/S = %d > 32", s->nw);
+  if (c.dtype == HILS_F32) {
+    if (!(s->d == 32 || s->d == 64 || s->d == 128)) return fail(HILS_ERR_UNSUPPORTED, "f32: d=%d", s->d);
+    if (!(s->S == 16 || s->S == 32 || s->S == 64)) return fail(HILS_ERR_UNSUPPORTED, "f32: S=%d", s->S);
+  } else {
+    if (s->d != 128 || s->S != 64) return fail(HILS_ERR_UNSUPPORTED, "bf16 needs d=128, S=64 (got d=%d S=%d)", s->d, s->S);
+  }
+  (void)decode;
+  return HILS_OK;
+}
+
+#define HILS_TRY(x)                      \
+  do {                                   \
+    hils_status_t _st = (x);             \
+    if (_st != HILS_OK) return _st;      \
+  } while (0)
+
+#define HILS_LAUNCH(expr, where)                       \
+  do {                                                 \
+    cudaError_t _e = (expr);                           \
+    if (_e != cudaSuccess) return cuda_fail(_e, where); \
+  } while (0)
+
+size_t esize(const Shape& s) { return s.dtype == HILS_F32 ? 4 : 2; }
+
+}  // namespace
+}  // namespace hils
+
+using namespace hils;
+
+extern "C" {
+
+const char* hils_version(void) { return "hils-b200 1.0"; }
+
+const char* hils_last_error(void) { return g_err; }
+
+void hils_set_wait_budget(int64_t cycles) { g_wait_budget = cycles > 0 ? cycles : 0; }
+
+void hils_set_fault_injection(int32_t mode) { g_inject = mode == 1 ? 1 : 0; }
+
+hils_status_t hils_build_summaries(const hils_config_t* cfg, const void* k, const void* q_lmk, void* k_sum,
+                                   float* b_sum, void* stream) {
+  Shape s;
+  HILS_TRY(make_shape(cfg, &s, false));
+  if (!aligned16(k) || !aligned16(q_lmk) || !aligned16(k_sum) || !aligned16(b_sum))
+    return fail(HILS_ERR_INVALID_ARG, "hils_build_summaries: NULL or unaligned pointer");
+  DevCtx ctx;
+  HILS_TRY(dev_ctx(&ctx));
+  HILS_LAUNCH(launch_summaries(s, k, q_lmk, k_sum, b_sum, (cudaStream_t)stream, ctx), "summaries");
+  return HILS_OK;
+}
+
+size_t hils_workspace_bytes(const hils_config_t* cfg, int32_t which, int32_t qcal_rank) {
+  Shape s;
+  if (make_shape(cfg, &s, which != HILS_WS_SCORE_PREFILL) != HILS_OK) return (size_t)-1;
+  switch (which) {
+    case HILS_WS_SCORE_PREFILL: {
+      size_t b = 0;
+      if (s.dtype == HILS_BF16) b += score_tc_workspace(s);
+      if (qcal_rank > 0) b += (size_t)s.B * s.Hq * s.N * s.d * esize(s);  // q~
+      return b;
+    }
+    case HILS_WS_SCORE_DECODE:
+      return decode_score_workspace(s);
+    case HILS_WS_ATTN_DECODE:
+      return decode_attn_workspace(s);
+  }
+  return (size_t)-1;
+}
+
+hils_status_t hils_score_topk(const hils_config_t* cfg, const void* q, const hils_qcal_t* qcal, const void* k_sum,
+                              const float* b_sum, int32_t* idx, float* s_sel, void* workspace, size_t ws_bytes,
+                              int32_t decode, void* stream) {
+  Shape s;
+  HILS_TRY(make_shape(cfg, &s, decode != 0));
+  if (decode != 0 && decode != 1) return fail(HILS_ERR_INVALID_ARG, "decode must be 0 or 1");
+  if (!aligned16(q) || !aligned16(k_sum) || !aligned16(b_sum) || !aligned16(idx) || !aligned16(s_sel))
+    return fail(HILS_ERR_INVALID_ARG, "hils_score_topk: NULL or unaligned pointer");
+  const size_t need = hils_workspace_bytes(cfg, decode ? HILS_WS_SCORE_DECODE : HILS_WS_SCORE_PREFILL,
+                                           qcal ? qcal->rank : 0);
+  if (need > 0 && (ws_bytes < need || !aligned16(workspace)))
+    return fail(HILS_ERR_INVALID_ARG, "hils_score_topk: workspace needs %zu bytes (got %zu)", need, ws_bytes);
+  DevCtx ctx;
+  HILS_TRY(dev_ctx(&ctx));
+  cudaStream_t st = (cudaStream_t)stream;
+  if (decode) {
+    if (qcal) return fail(HILS_ERR_UNSUPPORTED, "Q-Cal is a prefill-only option");
+    HILS_LAUNCH(launch_score_topk_decode(s, q, k_sum, b_sum, idx, s_sel, workspace, st, ctx), "score_topk_decode");
+    return HILS_OK;
+  }
+  const void* q_score = q;
+  unsigned char* ws = (unsigned char*)workspace;
+  if (qcal) {
+    if (!aligned16(qcal->h) || !aligned16(qcal->w_down) || !aligned16(qcal->w_up))
+      return fail(HILS_ERR_INVALID_ARG, "Q-Cal: NULL or unaligned pointer");
+    if (qcal->rank < 16 || qcal->rank > 128 || qcal->rank % 16 || qcal->d_model < 64 || qcal->d_model % 64)
+      return fail(HILS_ERR_UNSUPPORTED, "Q-Cal: rank %d / d_model %d not supported", qcal->rank, qcal->d_model);
+    if (s.dtype != HILS_BF16) return fail(HILS_ERR_UNSUPPORTED, "Q-Cal needs bf16");
+    void* q_tilde = ws;
+    ws += (size_t)s.B * s.Hq * s.N * s.d * esize(s);
+    HILS_LAUNCH(launch_qcal_tc(s, q, qcal->h, qcal->w_down, qcal->w_up, qcal->rank, qcal->d_model, q_tilde, st, ctx),
+                "qcal");
+    q_score = q_tilde;
+  }
+  if (s.dtype == HILS_F32) {
+    HILS_LAUNCH(launch_score_topk_simt(s, q_score, k_sum, b_sum, idx, s_sel, st, ctx), "score_topk_simt");
+  } else {
+    HILS_LAUNCH(launch_score_topk_tc(s, q_score, k_sum, b_sum, idx, s_sel, st, ctx), "score_topk_tc");
+  }
+  return HILS_OK;
+}
+
+hils_status_t hils_attn_prefill(const hils_config_t* cfg, const void* q, const void* k, const void* v,
+                                const int32_t* idx, const float* s_sel, void* out, void* stream) {
+  Shape s;
+  HILS_TRY(make_shape(cfg, &s, false));
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(s_sel) || !aligned16(out))
+    return fail(HILS_ERR_INVALID_ARG, "hils_attn_prefill: NULL or unaligned pointer");
+  DevCtx ctx;
+  HILS_TRY(dev_ctx(&ctx));
+  cudaStream_t st = (cudaStream_t)stream;
+  if (s.dtype == HILS_F32) {
+    HILS_LAUNCH(launch_attn_prefill_simt(s, q, k, v, idx, s_sel, out, st, ctx), "attn_prefill_simt");
+  } else {
+    HILS_LAUNCH(launch_attn_prefill_tc(s, q, k, v, idx, s_sel, out, st, ctx), "attn_prefill_tc");
+  }
+  return HILS_OK;
+}
+
+hils_status_t hils_attn_decode(const hils_config_t* cfg, const void* q, const void* k_cache, const void* v_cache,
+                               const int32_t* idx, const float* s_sel, void* out, void* workspace, size_t ws_bytes,
+                               void* stream) {
+  Shape s;
+  HILS_TRY(make_shape(cfg, &s, true));
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(idx) || !aligned16(s_sel) ||
+      !aligned16(out))
+    return fail(HILS_ERR_INVALID_ARG, "hils_attn_decode: NULL or unaligned pointer");
+  const size_t need = decode_attn_workspace(s);
+  if (ws_bytes < need || !aligned16(workspace))
+    return fail(HILS_ERR_INVALID_ARG, "hils_attn_decode: workspace needs %zu bytes (got %zu)", need, ws_bytes);
+  DevCtx ctx;
+  HILS_TRY(dev_ctx(&ctx));
+  HILS_LAUNCH(launch_attn_decode(s, q, k_cache, v_cache, idx, s_sel, out, workspace, (cudaStream_t)stream, ctx),
+              "attn_decode");
+  return HILS_OK;
+}
+
+hils_status_t hils_sync_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  DevCtx ctx;
+  HILS_TRY(dev_ctx(&ctx));
+  unsigned word = 0;
+  e = cudaMemcpy(&word, ctx.status, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "read status");
+  if (word) {
+    const unsigned zero = 0;
+    e = cudaMemcpy(ctx.status, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "clear status");
+  }
+  if (word & kStatusTimeout) return fail(HILS_ERR_TIMEOUT, "a device wait exceeded its budget (status 0x%x)", word);
+  if (word & kStatusBadIndex) return fail(HILS_ERR_INVALID_ARG, "a kernel skipped an out-of-range chunk index");
+  return HILS_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,55 @@
+// Internal launchers (C++ linkage, not part of the public ABI).  Shapes have
+// been validated by the caller (hils_api.cu); these only enqueue kernels and
+// return the launch error.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace hils {
+
+struct Shape {
+  int B, Hq, Hkv, G, N, d, S, W, nw, K, C, M;
+  float scale;
+  int dtype;  // 0 f32, 1 bf16
+};
+
+// K1: landmark summaries (all dtypes)
+cudaError_t launch_summaries(const Shape& s, const void* k, const void* q_lmk, void* k_sum, float* b_sum,
+                             cudaStream_t st, const DevCtx& ctx);
+
+// fp32 SIMT prefill score + group max + top-K
+cudaError_t launch_score_topk_simt(const Shape& s, const void* q, const void* k_sum, const float* b_sum, int32_t* idx,
+                                   float* s_sel, cudaStream_t st, const DevCtx& ctx);
+
+// bf16 tensor-core prefill score + group max + top-K (d=128, S=64)
+cudaError_t launch_score_topk_tc(const Shape& s, const void* q, const void* k_sum, const float* b_sum, int32_t* idx,
+                                 float* s_sel, cudaStream_t st, const DevCtx& ctx);
+size_t score_tc_workspace(const Shape& s);
+
+// Q-Cal: q~ = q + W_up W_down h written to q_tilde [B,Hq,N,d] (bf16, d=128)
+cudaError_t launch_qcal_tc(const Shape& s, const void* q, const void* h, const void* w_down, const void* w_up,
+                           int rank, int d_model, void* q_tilde, cudaStream_t st, const DevCtx& ctx);
+
+// decode score + group max + top-K (all dtypes); workspace: scores
+size_t decode_score_workspace(const Shape& s);
+cudaError_t launch_score_topk_decode(const Shape& s, const void* q, const void* k_sum, const float* b_sum,
+                                     int32_t* idx, float* s_sel, void* ws, cudaStream_t st, const DevCtx& ctx);
+
+// fp32 SIMT prefill attention
+cudaError_t launch_attn_prefill_simt(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
+                                     const float* s_sel, void* out, cudaStream_t st, const DevCtx& ctx);
+
+// bf16 tensor-core prefill attention (d=128, S=64)
+cudaError_t launch_attn_prefill_tc(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
+                                   const float* s_sel, void* out, cudaStream_t st, const DevCtx& ctx);
+
+// decode attention (all dtypes): split-KV partials + merge
+size_t decode_attn_workspace(const Shape& s);
+cudaError_t launch_attn_decode(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
+                               const float* s_sel, void* out, void* ws, cudaStream_t st, const DevCtx& ctx);
+
+}  // namespace hils

@@ -1,0 +1,129 @@
+// K1 — landmark chunk summaries.
+//
+// hyper.ai summary of arXiv 2607.02980 (HiLS-Attention), section 方法
+// (Method), the paragraph after the surrogate-score equation: the landmark
+// query q'_c of a chunk induces an attention distribution p over the chunk's
+// keys; k'_c is the p-weighted sum of those keys and b'_c the entropy of p.
+//
+// One CTA (256 threads) handles one (batch, KV head, chunk) at a time and
+// serves all G query heads of the group, so each key tile is read from HBM
+// once.  The tile is staged in shared memory as fp32 with a padded row pitch
+// (conflict-free column and row walks); logits, the softmax and the entropy
+// are fp32.  The entropy is evaluated as (m + log Z) - sum p*l, which avoids
+// 0*log 0.  The kernel is HBM-bound: it reads K once and writes G summaries.
+#include "launch.h"
+
+namespace hils {
+namespace {
+
+constexpr int kThreads = 256;
+
+template <typename T, int D, int S, int G>
+__global__ void __launch_bounds__(kThreads) summaries_kernel(Shape s, const T* __restrict__ k,
+                                                             const T* __restrict__ q_lmk, T* __restrict__ k_sum,
+                                                             float* __restrict__ b_sum) {
+  __shared__ float ks[S][D + 1];
+  __shared__ float qs[G][D];
+  __shared__ float lg[G][S];
+  const int tid = threadIdx.x;
+  const long long units = (long long)s.B * s.Hkv * s.C;
+  for (long long u = blockIdx.x; u < units; u += gridDim.x) {
+    const int c = (int)(u % s.C);
+    const int g = (int)((u / s.C) % s.Hkv);
+    const int b = (int)(u / ((long long)s.C * s.Hkv));
+    const T* kc = k + (((long long)b * s.Hkv + g) * s.N + (long long)c * S) * D;
+    for (int e = tid; e < S * D; e += kThreads) ks[e / D][e % D] = to_f32(kc[e]);
+    for (int e = tid; e < G * D; e += kThreads) {
+      const int hg = e / D;
+      qs[hg][e % D] = to_f32(q_lmk[(((long long)b * s.Hq + g * G + hg) * s.C + c) * D + e % D]);
+    }
+    __syncthreads();
+    // logits l[h][j] = q'_h . k_j * scale
+    for (int p = tid; p < G * S; p += kThreads) {
+      const int hg = p / S, j = p % S;
+      float acc = 0.f;
+#pragma unroll 8
+      for (int e = 0; e < D; ++e) acc = fmaf(qs[hg][e], ks[j][e], acc);
+      lg[hg][j] = acc * s.scale;
+    }
+    __syncthreads();
+    // per head: softmax over the S keys, entropy
+    const int warp = tid >> 5, lane = tid & 31;
+    for (int hg = warp; hg < G; hg += kThreads / 32) {
+      float m = -INFINITY;
+      for (int j = lane; j < S; j += 32) m = fmaxf(m, lg[hg][j]);
+      m = warp_max(m);
+      float z = 0.f, zl = 0.f;
+      for (int j = lane; j < S; j += 32) {
+        const float e = expf(lg[hg][j] - m);
+        z += e;
+        zl += e * lg[hg][j];
+      }
+      z = warp_sum(z);
+      zl = warp_sum(zl);
+      __syncwarp();
+      for (int j = lane; j < S; j += 32) lg[hg][j] = expf(lg[hg][j] - m) / z;
+      if (lane == 0) b_sum[((long long)b * s.Hq + g * G + hg) * s.C + c] = (m + logf(z)) - zl / z;
+    }
+    __syncthreads();
+    // k'_h = sum_j p_hj k_j
+    for (int o = tid; o < G * D; o += kThreads) {
+      const int hg = o / D, e = o % D;
+      float acc = 0.f;
+#pragma unroll 8
+      for (int j = 0; j < S; ++j) acc = fmaf(lg[hg][j], ks[j][e], acc);
+      k_sum[(((long long)b * s.Hq + g * G + hg) * s.C + c) * D + e] = from_f32<T>(acc);
+    }
+    __syncthreads();
+  }
+}
+
+template <typename T, int D, int S, int G>
+cudaError_t go(const Shape& s, const void* k, const void* q_lmk, void* k_sum, float* b_sum, cudaStream_t st) {
+  const long long units = (long long)s.B * s.Hkv * s.C;
+  if (units == 0) return cudaSuccess;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long grid = units < (long long)sms * 8 ? units : (long long)sms * 8;
+  summaries_kernel<T, D, S, G><<<(unsigned)grid, kThreads, 0, st>>>(s, (const T*)k, (const T*)q_lmk, (T*)k_sum,
+                                                                     b_sum);
+  return cudaGetLastError();
+}
+
+template <typename T, int D, int S>
+cudaError_t go_g(const Shape& s, const void* k, const void* q_lmk, void* k_sum, float* b_sum, cudaStream_t st) {
+  switch (s.G) {
+    case 1: return go<T, D, S, 1>(s, k, q_lmk, k_sum, b_sum, st);
+    case 2: return go<T, D, S, 2>(s, k, q_lmk, k_sum, b_sum, st);
+    case 4: return go<T, D, S, 4>(s, k, q_lmk, k_sum, b_sum, st);
+    case 8: return go<T, D, S, 8>(s, k, q_lmk, k_sum, b_sum, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <typename T>
+cudaError_t go_t(const Shape& s, const void* k, const void* q_lmk, void* k_sum, float* b_sum, cudaStream_t st) {
+#define HILS_CASE(DD, SS) \
+  if (s.d == DD && s.S == SS) return go_g<T, DD, SS>(s, k, q_lmk, k_sum, b_sum, st);
+  HILS_CASE(64, 32)
+  HILS_CASE(64, 64)
+  HILS_CASE(128, 32)
+  HILS_CASE(128, 64)
+  HILS_CASE(32, 16)
+  HILS_CASE(64, 16)
+  HILS_CASE(128, 16)
+  HILS_CASE(32, 32)
+#undef HILS_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_summaries(const Shape& s, const void* k, const void* q_lmk, void* k_sum, float* b_sum,
+                             cudaStream_t st, const DevCtx&) {
+  if (s.dtype == 0) return go_t<float>(s, k, q_lmk, k_sum, b_sum, st);
+  return go_t<__nv_bfloat16>(s, k, q_lmk, k_sum, b_sum, st);
+}
+
+}  // namespace hils

@@ -1,0 +1,225 @@
+"""Thin Python binding of libhils.so (C ABI in include/hils.h).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  torch tensors supply device memory and the current CUDA stream.
+The library is loaded from this package's directory; if it is missing the
+first call raises (there is no fallback of any kind).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libhils.so")
+
+HILS_OK, HILS_ERR_INVALID_ARG, HILS_ERR_UNSUPPORTED, HILS_ERR_CUDA, HILS_ERR_TIMEOUT = range(5)
+HILS_F32, HILS_BF16 = 0, 1
+HILS_WS_SCORE_PREFILL, HILS_WS_SCORE_DECODE, HILS_WS_ATTN_DECODE = 0, 1, 2
+
+EXPORTS = (
+    "hils_build_summaries",
+    "hils_score_topk",
+    "hils_attn_prefill",
+    "hils_attn_decode",
+    "hils_workspace_bytes",
+    "hils_sync_status",
+    "hils_last_error",
+    "hils_set_wait_budget",
+    "hils_set_fault_injection",
+    "hils_version",
+)
+
+
+class HilsError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"hils status {status}: {msg}")
+        self.status = status
+
+
+class Config(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32),
+        ("seq_len", ctypes.c_int32),
+        ("n_q_heads", ctypes.c_int32),
+        ("n_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("chunk", ctypes.c_int32),
+        ("window", ctypes.c_int32),
+        ("top_k", ctypes.c_int32),
+        ("query_block", ctypes.c_int32),
+        ("scale", ctypes.c_float),
+        ("dtype", ctypes.c_int32),
+    ]
+
+
+class QCal(ctypes.Structure):
+    _fields_ = [
+        ("h", ctypes.c_void_p),
+        ("w_down", ctypes.c_void_p),
+        ("w_up", ctypes.c_void_p),
+        ("rank", ctypes.c_int32),
+        ("d_model", ctypes.c_int32),
+    ]
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libhils.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m chunk_wise_sparse_landmark_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        P, C = ctypes.c_void_p, ctypes.POINTER(Config)
+        lib.hils_build_summaries.argtypes = [C, P, P, P, P, P]
+        lib.hils_score_topk.argtypes = [C, P, ctypes.POINTER(QCal), P, P, P, P, P, ctypes.c_size_t, ctypes.c_int32, P]
+        lib.hils_attn_prefill.argtypes = [C, P, P, P, P, P, P, P]
+        lib.hils_attn_decode.argtypes = [C, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+        lib.hils_workspace_bytes.argtypes = [C, ctypes.c_int32, ctypes.c_int32]
+        lib.hils_workspace_bytes.restype = ctypes.c_size_t
+        lib.hils_sync_status.argtypes = [P]
+        lib.hils_last_error.restype = ctypes.c_char_p
+        lib.hils_set_wait_budget.argtypes = [ctypes.c_int64]
+        lib.hils_set_wait_budget.restype = None
+        lib.hils_set_fault_injection.argtypes = [ctypes.c_int32]
+        lib.hils_set_fault_injection.restype = None
+        lib.hils_version.restype = ctypes.c_char_p
+        for n in ("hils_build_summaries", "hils_score_topk", "hils_attn_prefill", "hils_attn_decode",
+                  "hils_sync_status"):
+            getattr(lib, n).restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def make_config(B, N, Hq, Hkv, d, S, W, K, dtype, M=0, scale=0.0) -> Config:
+    dt = HILS_F32 if dtype in ("f32", torch.float32, HILS_F32) else HILS_BF16
+    return Config(B, N, Hq, Hkv, d, S, W, K, M, scale, dt)
+
+
+def config_of(w) -> Config:
+    """Config for an :class:`inputs.Workload`."""
+    return make_config(w.B, w.N, w.Hq, w.Hkv, w.d, w.S, w.W, w.K, w.dtype, M=w.M)
+
+
+def _p(t: torch.Tensor | None):
+    if t is None:
+        return None
+    assert t.is_cuda and t.is_contiguous(), "tensors must be contiguous CUDA tensors"
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(st: int):
+    if st != HILS_OK:
+        raise HilsError(st, load().hils_last_error().decode())
+
+
+def workspace_bytes(cfg: Config, which: int, qcal_rank: int = 0) -> int:
+    n = load().hils_workspace_bytes(ctypes.byref(cfg), which, qcal_rank)
+    if n == ctypes.c_size_t(-1).value:
+        raise HilsError(HILS_ERR_INVALID_ARG, load().hils_last_error().decode())
+    return n
+
+
+def hils_build_summaries(cfg: Config, k, q_lmk, k_sum, b_sum, stream=None):
+    _check(load().hils_build_summaries(ctypes.byref(cfg), _p(k), _p(q_lmk), _p(k_sum), _p(b_sum), _stream(stream)))
+
+
+def hils_score_topk(cfg: Config, q, k_sum, b_sum, idx, s_sel, workspace=None, decode=False, qcal=None, stream=None):
+    """qcal: None or (h, w_down, w_up) tensors."""
+    qc = None
+    if qcal is not None:
+        h, wd, wu = qcal
+        qc = ctypes.byref(QCal(_p(h), _p(wd), _p(wu), wd.shape[0], wd.shape[1]))
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().hils_score_topk(ctypes.byref(cfg), _p(q), qc, _p(k_sum), _p(b_sum), _p(idx), _p(s_sel),
+                                  _p(workspace), ws_bytes, 1 if decode else 0, _stream(stream)))
+
+
+def hils_attn_prefill(cfg: Config, q, k, v, idx, s_sel, out, stream=None):
+    _check(load().hils_attn_prefill(ctypes.byref(cfg), _p(q), _p(k), _p(v), _p(idx), _p(s_sel), _p(out),
+                                    _stream(stream)))
+
+
+def hils_attn_decode(cfg: Config, q, k_cache, v_cache, idx, s_sel, out, workspace, stream=None):
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(load().hils_attn_decode(ctypes.byref(cfg), _p(q), _p(k_cache), _p(v_cache), _p(idx), _p(s_sel), _p(out),
+                                   _p(workspace), ws_bytes, _stream(stream)))
+
+
+def hils_sync_status(stream=None):
+    _check(load().hils_sync_status(_stream(stream)))
+
+
+def hils_set_wait_budget(cycles: int):
+    load().hils_set_wait_budget(int(cycles))
+
+
+def hils_set_fault_injection(mode: int):
+    load().hils_set_fault_injection(int(mode))
+
+
+# ------------------------------------------------------------- pipelines ---
+
+def alloc_workspace(nbytes: int, device) -> torch.Tensor | None:
+    if nbytes == 0:
+        return None
+    return torch.empty((nbytes + 15) // 16 * 16, dtype=torch.uint8, device=device)
+
+
+class Prefill:
+    """Buffers and calls for one prefill configuration (all device-resident)."""
+
+    def __init__(self, cfg: Config, device, qcal_rank: int = 0):
+        self.cfg = cfg
+        B, N, Hq, Hkv, d, S, K = cfg.batch, cfg.seq_len, cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.chunk, cfg.top_k
+        dt = torch.float32 if cfg.dtype == HILS_F32 else torch.bfloat16
+        C = N // S
+        self.k_sum = torch.empty((B, Hq, C, d), dtype=dt, device=device)
+        self.b_sum = torch.empty((B, Hq, C), dtype=torch.float32, device=device)
+        self.idx = torch.empty((B, Hkv, N, K), dtype=torch.int32, device=device)
+        self.s_sel = torch.empty((B, Hq, N, K), dtype=torch.float32, device=device)
+        self.out = torch.empty((B, Hq, N, d), dtype=dt, device=device)
+        self.ws = alloc_workspace(workspace_bytes(cfg, HILS_WS_SCORE_PREFILL, qcal_rank), device)
+
+    def run(self, q, k, v, q_lmk, qcal=None, stream=None):
+        hils_build_summaries(self.cfg, k, q_lmk, self.k_sum, self.b_sum, stream)
+        hils_score_topk(self.cfg, q, self.k_sum, self.b_sum, self.idx, self.s_sel, self.ws, False, qcal, stream)
+        hils_attn_prefill(self.cfg, q, k, v, self.idx, self.s_sel, self.out, stream)
+        return self.out
+
+
+class Decode:
+    """Buffers and calls for one decode configuration; summaries are built by
+    :meth:`summarize` (once per cache state) and reused by :meth:`step`."""
+
+    def __init__(self, cfg: Config, device):
+        self.cfg = cfg
+        B, L, Hq, Hkv, d, S, K = cfg.batch, cfg.seq_len, cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.chunk, cfg.top_k
+        dt = torch.float32 if cfg.dtype == HILS_F32 else torch.bfloat16
+        C = L // S
+        self.k_sum = torch.empty((B, Hq, C, d), dtype=dt, device=device)
+        self.b_sum = torch.empty((B, Hq, C), dtype=torch.float32, device=device)
+        self.idx = torch.empty((B, Hkv, K), dtype=torch.int32, device=device)
+        self.s_sel = torch.empty((B, Hq, K), dtype=torch.float32, device=device)
+        self.out = torch.empty((B, Hq, d), dtype=dt, device=device)
+        self.ws_score = alloc_workspace(workspace_bytes(cfg, HILS_WS_SCORE_DECODE), device)
+        self.ws_attn = alloc_workspace(workspace_bytes(cfg, HILS_WS_ATTN_DECODE), device)
+
+    def summarize(self, k_cache, q_lmk, stream=None):
+        hils_build_summaries(self.cfg, k_cache, q_lmk, self.k_sum, self.b_sum, stream)
+
+    def step(self, q, k_cache, v_cache, stream=None):
+        hils_score_topk(self.cfg, q, self.k_sum, self.b_sum, self.idx, self.s_sel, self.ws_score, True, None, stream)
+        hils_attn_decode(self.cfg, q, k_cache, v_cache, self.idx, self.s_sel, self.out, self.ws_attn, stream)
+        return self.out

@@ -1,0 +1,187 @@
+/*
+ * hils.h — C ABI of libhils.so: the forward hot path of Hierarchical Landmark
+ * Sparse (HiLS) attention on NVIDIA B200 (sm_100a).
+ *
+ * Source of the method: the hyper.ai summary of arXiv 2607.02980
+ * (HiLS-Attention), section "方法" (Method); cited below as [Method].
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor arguments are DEVICE pointers to dense, row-major
+ *    ("contiguous") buffers owned by the caller.  Element pointers must be
+ *    16-byte aligned.  The library never allocates, frees or retains them.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Every call is asynchronous on that stream: it validates its
+ *    arguments on the host, enqueues kernels and returns.
+ *  - Notation: B batch, Hq query heads, Hkv key/value heads (G = Hq/Hkv
+ *    query heads share one KV head, "a GQA group"), N sequence length,
+ *    d head dim, S chunk size, C = floor(N/S) complete chunks, W window,
+ *    n_w = W/S, K selected chunks, cur(i) = floor(i/S).
+ *  - Window of position i: keys [max(0, (cur(i)-n_w+1)*S), i] (the current
+ *    partial chunk plus the n_w-1 chunks before it).  Candidates of i: the
+ *    complete chunks c <= cur(i)-n_w.  ([Method], uniform chunking and the
+ *    chunk-aligned sliding window.)
+ *  - dtype (hils_config_t.dtype) is the type of q, k, v, q_lmk, k_sum, out
+ *    and of the Q-Cal tensors; scores (b_sum, s_sel) are always float32,
+ *    chunk indices int32.
+ *  - Errors: argument problems are caught on the host before any launch and
+ *    return HILS_ERR_INVALID_ARG; shapes/dtypes without a kernel return
+ *    HILS_ERR_UNSUPPORTED (there is no fallback of any kind); a failed launch
+ *    returns HILS_ERR_CUDA.  A device-side wait that exceeds its budget sets
+ *    a per-device status word and the kernel returns early; the caller sees it
+ *    as HILS_ERR_TIMEOUT from hils_sync_status().  hils_last_error() gives a
+ *    thread-local message for the last non-OK status.  No C++ exception
+ *    crosses this boundary.
+ *
+ * Supported kernels: dtype F32 (SIMT kernels, any d in {32,64,96,128},
+ * S in {16,32,64}); dtype BF16 with d = 128 and S = 64 (tensor-core prefill
+ * path; SIMT decode path).  K <= 64, n_w <= 32.
+ */
+#ifndef HILS_H
+#define HILS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HILS_OK = 0,
+  HILS_ERR_INVALID_ARG = 1,
+  HILS_ERR_UNSUPPORTED = 2,
+  HILS_ERR_CUDA = 3,
+  HILS_ERR_TIMEOUT = 4
+} hils_status_t;
+
+typedef enum { HILS_F32 = 0, HILS_BF16 = 1 } hils_dtype_t;
+
+typedef struct {
+  int32_t batch;       /* B */
+  int32_t seq_len;     /* N (prefill) or L, the decode cache length */
+  int32_t n_q_heads;   /* Hq */
+  int32_t n_kv_heads;  /* Hkv; Hq % Hkv == 0 */
+  int32_t head_dim;    /* d */
+  int32_t chunk;       /* S */
+  int32_t window;      /* W; W % S == 0, W >= S */
+  int32_t top_k;       /* K >= 1 */
+  int32_t query_block; /* prefill tuning hint (0 = library default); never changes results */
+  float scale;         /* logit scale; 0 means 1/sqrt(d) */
+  int32_t dtype;       /* hils_dtype_t */
+} hils_config_t;
+
+/* Optional low-rank query calibration (Q-Cal), [Method] second practical
+ * design choice: the scoring query is q~_i = q_i + W_up (W_down h_i), rank r.
+ * It changes only the chunk scores, never the attention logits. */
+typedef struct {
+  const void* h;       /* [B, N, d_model] hidden states (dtype); decode: [B, d_model] */
+  const void* w_down;  /* [r, d_model] (dtype) */
+  const void* w_up;    /* [Hq*d, r] (dtype); row hq*d+e feeds head hq, dim e */
+  int32_t rank;        /* r, a multiple of 16, <= 128 */
+  int32_t d_model;     /* a multiple of 64 */
+} hils_qcal_t;
+
+/*
+ * Landmark chunk summaries, [Method] (paragraph after the surrogate-score
+ * equation): for each (b, query head h, complete chunk c) the landmark query
+ * q'_{h,c} induces p = softmax_j(q'_{h,c}.k_j * scale) over the S keys of
+ * chunk c (KV head h/G); k'_{h,c} = sum_j p_j k_j and b'_{h,c} = the entropy
+ * of p in nats.
+ *   k      [B, Hkv, N, d]  (dtype)        q_lmk [B, Hq, C, d] (dtype)
+ *   k_sum  [B, Hq, C, d]   (dtype, out)   b_sum [B, Hq, C]    (float32, out)
+ * Decode uses the same call with N = L.
+ */
+hils_status_t hils_build_summaries(const hils_config_t* cfg, const void* k, const void* q_lmk, void* k_sum,
+                                   float* b_sum, void* stream);
+
+/*
+ * Chunk scoring and top-K selection, [Method] surrogate-score equation and
+ * third practical design choice (GQA):
+ *   s^_{h,i,c} = q~_{h,i}.k'_{h,c} * scale + b'_{h,c}   for candidates c of i,
+ *   g_{i,c}    = max over the G heads h of the group of s^_{h,i,c},
+ *   I_i        = the K candidates with the largest g (ties: smaller c; all of
+ *                them when there are fewer than K).
+ * Outputs, per (b, KV group, position): idx = I_i in ascending chunk order,
+ * padded with -1; per (b, query head, position): s_sel = that head's own s^ of
+ * the chosen chunks, slot-aligned with idx, padded with -inf.
+ *   prefill (decode = 0): q [B, Hq, N, d]; idx [B, Hkv, N, K]; s_sel [B, Hq, N, K]
+ *   decode  (decode = 1): q [B, Hq, d] is the token at position L-1 (its key and
+ *                         value are already in the cache); idx [B, Hkv, K];
+ *                         s_sel [B, Hq, K]
+ *   k_sum, b_sum: as produced by hils_build_summaries.
+ *   qcal: NULL, or the Q-Cal tensors (prefill only).
+ *   workspace: device scratch of at least
+ *              hils_workspace_bytes(cfg, HILS_WS_SCORE_PREFILL or _DECODE, rank)
+ *              bytes (may be NULL when that size is 0).  Contents on entry are
+ *              ignored; the call owns it until the stream passes the call.
+ */
+hils_status_t hils_score_topk(const hils_config_t* cfg, const void* q, const hils_qcal_t* qcal, const void* k_sum,
+                              const float* b_sum, int32_t* idx, float* s_sel, void* workspace, size_t ws_bytes,
+                              int32_t decode, void* stream);
+
+/*
+ * Hierarchical-softmax sparse attention, prefill ([Method], the factorised
+ * token weight w_{i,j} and the partition estimate Z^_i; the chatpaper abstract
+ * of HiLS: each query attends every retrieved chunk on its own and the chunk
+ * outputs are fused by the retrieval scores).  For query head h at position i:
+ *   O_{i,c} = sum_{j in c} softmax_{j in c}(s_ij) v_j   (s_ij = q.k_j * scale)
+ *   Z^_i    = sum_{c in I_i} exp(s^_c) + Z_swa,  Z_swa = sum_{j in window} exp(s_ij)
+ *   out_i   = [sum_c exp(s^_c) O_{i,c} + sum_{j in window} exp(s_ij) v_j] / Z^_i
+ * with s^_c taken from s_sel (each head its own).  Attention logits use the
+ * raw q.
+ *   q [B, Hq, N, d]; k, v [B, Hkv, N, d]; idx [B, Hkv, N, K]; s_sel [B, Hq, N, K];
+ *   out [B, Hq, N, d] (dtype, out).
+ * idx entries must be -1 or candidates of their position (checked on device:
+ * an out-of-range entry is skipped and recorded in the status word).
+ */
+hils_status_t hils_attn_prefill(const hils_config_t* cfg, const void* q, const void* k, const void* v,
+                                const int32_t* idx, const float* s_sel, void* out, void* stream);
+
+/*
+ * The same attention for one new token per sequence (decode), at position
+ * L-1 of a cache of length L = cfg->seq_len.  The K chunks and the window are
+ * split across CTAs and merged by a second kernel.
+ *   q [B, Hq, d]; k_cache, v_cache [B, Hkv, L, d]; idx [B, Hkv, K];
+ *   s_sel [B, Hq, K]; out [B, Hq, d] (dtype, out).
+ *   workspace: at least hils_workspace_bytes(cfg, HILS_WS_ATTN_DECODE, 0)
+ *              bytes of device scratch for the per-split partial results.
+ */
+hils_status_t hils_attn_decode(const hils_config_t* cfg, const void* q, const void* k_cache, const void* v_cache,
+                               const int32_t* idx, const float* s_sel, void* out, void* workspace, size_t ws_bytes,
+                               void* stream);
+
+enum { HILS_WS_SCORE_PREFILL = 0, HILS_WS_SCORE_DECODE = 1, HILS_WS_ATTN_DECODE = 2 };
+
+/* Bytes of workspace the call `which` needs for this configuration (0 if none);
+ * qcal_rank is the Q-Cal rank for HILS_WS_SCORE_PREFILL (0 = no Q-Cal).
+ * Returns (size_t)-1 for an invalid configuration. */
+size_t hils_workspace_bytes(const hils_config_t* cfg, int32_t which, int32_t qcal_rank);
+
+/* Synchronises `stream`, then reads and clears the calling device's status
+ * word: HILS_OK, HILS_ERR_TIMEOUT (a bounded device wait ran out), or
+ * HILS_ERR_INVALID_ARG (a kernel skipped an out-of-range index). */
+hils_status_t hils_sync_status(void* stream);
+
+/* Thread-local text for the last non-OK status returned on this thread. */
+const char* hils_last_error(void);
+
+/* Test hook: budget, in clock64 cycles, of every bounded device wait launched
+ * after this call (0 restores the default of about 2 s at 2 GHz). */
+void hils_set_wait_budget(int64_t cycles);
+
+/* Test hook: mode 1 makes every kernel launched afterwards that waits on
+ * tile copies (decode attention, tensor-core prefill) skip issuing those
+ * copies, so that its bounded waits run out with no copy left in flight; the
+ * kernels then return early and hils_sync_status() reports HILS_ERR_TIMEOUT.
+ * Outputs of such launches are undefined.  mode 0 turns the hook off. */
+void hils_set_fault_injection(int32_t mode);
+
+/* Library version, e.g. "hils-b200 1.0". */
+const char* hils_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HILS_H */

@@ -1,0 +1,73 @@
+"""The C ABI without a GPU: the library loads, exports every entry point that
+include/hils.h declares, and rejects bad arguments on the host before any
+device work."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from chunk_wise_sparse_landmark_b200 import hils as H
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "hils.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(hils_[a-z_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = H.load()
+    names = _declared()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(H.EXPORTS)
+
+
+def test_version():
+    assert H.load().hils_version().startswith(b"hils-b200")
+
+
+@pytest.mark.parametrize(
+    "kw,status",
+    [
+        (dict(Hkv=3), H.HILS_ERR_INVALID_ARG),        # Hq % Hkv
+        (dict(W=48), H.HILS_ERR_INVALID_ARG),         # W % S
+        (dict(W=16), H.HILS_ERR_INVALID_ARG),         # W < S
+        (dict(K=0), H.HILS_ERR_INVALID_ARG),
+        (dict(K=65), H.HILS_ERR_UNSUPPORTED),
+        (dict(d=48), H.HILS_ERR_UNSUPPORTED),
+        (dict(dtype="bf16"), H.HILS_ERR_UNSUPPORTED),  # bf16 needs d=128, S=64
+    ],
+)
+def test_bad_config_rejected_on_host(kw, status):
+    base = dict(B=1, N=512, Hq=4, Hkv=1, d=64, S=32, W=64, K=4, dtype="f32")
+    base.update(kw)
+    cfg = H.make_config(**base)
+    lib = H.load()
+    st = lib.hils_build_summaries(ctypes.byref(cfg), None, None, None, None, None)
+    assert st == status, lib.hils_last_error()
+    assert lib.hils_workspace_bytes(ctypes.byref(cfg), 0, 0) == ctypes.c_size_t(-1).value
+
+
+def test_null_and_unaligned_pointers_rejected():
+    lib = H.load()
+    cfg = H.make_config(1, 512, 4, 1, 64, 32, 64, 4, "f32")
+    assert lib.hils_build_summaries(ctypes.byref(cfg), None, None, None, None, None) == H.HILS_ERR_INVALID_ARG
+    p = ctypes.c_void_p(0x1000)
+    bad = ctypes.c_void_p(0x1004)
+    assert lib.hils_attn_prefill(ctypes.byref(cfg), p, p, p, p, p, bad, None) == H.HILS_ERR_INVALID_ARG
+    assert b"unaligned" in lib.hils_last_error()
+    # workspace too small for decode attention
+    assert lib.hils_attn_decode(ctypes.byref(cfg), p, p, p, p, p, p, p, 0, None) == H.HILS_ERR_INVALID_ARG
+    assert b"workspace" in lib.hils_last_error()
+
+
+def test_workspace_sizes():
+    cfg = H.make_config(16, 524288, 32, 8, 128, 64, 512, 32, "bf16")
+    ws = H.workspace_bytes(cfg, H.HILS_WS_SCORE_DECODE)
+    assert ws == (16 * 32 * 8192 + 16 * 8 * 8192) * 4
+    assert H.workspace_bytes(cfg, H.HILS_WS_ATTN_DECODE) > 0
