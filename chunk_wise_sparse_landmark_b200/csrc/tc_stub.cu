@@ -6,6 +6,4 @@ cudaError_t launch_score_topk_tc(const Shape&, const void*, const void*, const f
                                  const DevCtx&) { return cudaErrorNotSupported; }
 cudaError_t launch_qcal_tc(const Shape&, const void*, const void*, const void*, const void*, int, int, void*,
                            cudaStream_t, const DevCtx&) { return cudaErrorNotSupported; }
-cudaError_t launch_attn_prefill_tc(const Shape&, const void*, const void*, const void*, const int32_t*, const float*,
-                                   void*, cudaStream_t, const DevCtx&) { return cudaErrorNotSupported; }
 }  // namespace hils
