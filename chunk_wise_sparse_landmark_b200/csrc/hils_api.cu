@@ -104,10 +104,11 @@ hils_status_t make_shape(const hils_config_t* cfg, Shape* s, bool decode) {
     if (_st != HILS_OK) return _st;      \
   } while (0)
 
-#define HILS_LAUNCH(expr, where)                       \
-  do {                                                 \
-    cudaError_t _e = (expr);                           \
-    if (_e != cudaSuccess) return cuda_fail(_e, where); \
+#define HILS_LAUNCH(expr, where)                                                                  \
+  do {                                                                                            \
+    cudaError_t _e = (expr);                                                                      \
+    if (_e == cudaErrorNotSupported) return fail(HILS_ERR_UNSUPPORTED, "%s: no kernel for this shape", where); \
+    if (_e != cudaSuccess) return cuda_fail(_e, where);                                           \
   } while (0)
 
 size_t esize(const Shape& s) { return s.dtype == HILS_F32 ? 4 : 2; }
