@@ -98,8 +98,9 @@ def _e2e(w, x, all_rows_select=True):
     """Run the whole bf16 prefill through the C ABI and check every stage."""
     dm = _dims(w)
     d = {n: x[n].to(DEV) for n in ("q", "k", "v", "q_lmk")}
-    pre = H.Prefill(H.config_of(w), DEV)
-    pre.run(d["q"], d["k"], d["v"], d["q_lmk"])
+    qc = (x["h"].to(DEV), x["w_down"].to(DEV), x["w_up"].to(DEV)) if w.d_model else None
+    pre = H.Prefill(H.config_of(w), DEV, qcal_rank=w.qcal_rank)
+    pre.run(d["q"], d["k"], d["v"], d["q_lmk"], qcal=qc)
     H.hils_sync_status()
     q, k, v, ql = (to_np(x[n]) for n in ("q", "k", "v", "q_lmk"))
     ks, bs = oracle.summaries(dm, k, ql)
@@ -107,7 +108,14 @@ def _e2e(w, x, all_rows_select=True):
     np.testing.assert_allclose(to_np(pre.b_sum), bs, rtol=0, atol=2e-5)
     rows = oracle.all_rows(w.B, w.N) if all_rows_select else sample_rows(w, x["needles"], n_random=2048)
     ridx = np.array([b * w.N + p for b, p in rows])
-    idx_or, ssel_or, s_all, g_all = oracle.select(dm, rows, q, k_sum=ks, b_sum=bs, want_all=True)
+    qs = None
+    if w.d_model:
+        qs = oracle.qcal(dm, rows, q, to_np(x["h"]), to_np(x["w_down"]), to_np(x["w_up"]))
+        # the scoring query sits at the start of the workspace, in the layout of q (bf16)
+        qt = pre.ws[: w.B * w.Hq * w.N * w.d * 2].view(torch.bfloat16).view(w.B, w.Hq, w.N, w.d)
+        qt = to_np(qt).transpose(0, 2, 1, 3).reshape(-1, w.Hq, w.d)[ridx]
+        assert (np.abs(qt - qs) <= np.abs(qs) * 2.0 ** -8 + 2e-3).all(), np.abs(qt - qs).max()
+    idx_or, ssel_or, s_all, g_all = oracle.select(dm, rows, q, k_sum=ks, b_sum=bs, qs=qs, want_all=True)
     idx_g = to_np(pre.idx).astype(np.int64).transpose(0, 2, 1, 3).reshape(-1, w.Hkv, w.K)[ridx]
     n_strict, n = check_selection(idx_g, g_all, w.K)
     ssel_g = to_np(pre.s_sel).transpose(0, 2, 1, 3).reshape(-1, w.Hq, w.K)[ridx]
@@ -179,3 +187,22 @@ def test_prefill_wait_timeout_reports_status(stage):
     pre.run(x["q"], x["k"], x["v"], x["q_lmk"])
     H.hils_sync_status()
     assert torch.isfinite(pre.out.float()).all()
+
+
+def test_end_to_end_qcal_reduced():
+    # the 512K Q-Cal workload's K, window, rank and d_model on a shorter sequence
+    w = WORKLOADS["prefill_512k_qcal"].scaled(name="qcal_r", N=8192, Hq=8, Hkv=2, needles_per_head=8)
+    _e2e(w, prefill_inputs(w))
+
+
+def test_qcal_zero_up_projection_changes_nothing():
+    w = WORKLOADS["prefill_512k_qcal"].scaled(name="qcal0", N=4096, Hq=8, Hkv=2, needles_per_head=0)
+    x = {n: t.to(DEV) for n, t in prefill_inputs(w).items() if isinstance(t, torch.Tensor)}
+    base = H.Prefill(H.config_of(w), DEV)
+    base.run(x["q"], x["k"], x["v"], x["q_lmk"])
+    qc = H.Prefill(H.config_of(w), DEV, qcal_rank=w.qcal_rank)
+    qc.run(x["q"], x["k"], x["v"], x["q_lmk"], qcal=(x["h"], x["w_down"], torch.zeros_like(x["w_up"])))
+    H.hils_sync_status()
+    assert torch.equal(base.idx, qc.idx)
+    assert torch.equal(base.s_sel, qc.s_sel)
+    assert torch.equal(base.out, qc.out)
