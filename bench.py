@@ -1,0 +1,420 @@
+"""Benchmark of the HiLS forward hot path on B200 (one JSON line on rank 0).
+
+Step (prefill workloads): landmark summaries -> [Q-Cal ->] scoring + GQA
+group max + top-K -> hierarchical-softmax attention, all through the C ABI on
+device-resident synthetic inputs.  Metric: prefill tokens/s.  The decode
+workload (one token per sequence, score + top-K + split-KV attention over a
+pre-summarised cache) is measured in the same run and reported in "decode".
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                  [--impl reference] [--no-decode] [--no-e2e] [--no-cpu]
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own replica of
+the workload (independent sequences: the path has no exchange step), the time
+is the max over ranks, and the value is all ranks' tokens / that time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from chunk_wise_sparse_landmark_b200 import hils as H  # noqa: E402
+from chunk_wise_sparse_landmark_b200.inputs import WORKLOADS, decode_inputs, prefill_inputs  # noqa: E402
+
+METRIC = "HiLS prefill tokens/s & decode seqs/s at 128K-512K ctx; % of roofline"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------- utilities ---
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+class Clocks:
+    """nvidia-smi sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.gpu = gpu_index
+        self.p = None
+
+    def __enter__(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                                      stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+        return self
+
+    def __exit__(self, *a):
+        if self.p is not None:
+            self.p.terminate()
+            try:
+                self.p.wait(timeout=5)
+            except Exception:
+                self.p.kill()
+
+    def summary(self):
+        try:
+            lines = [ln.split(",") for ln in open(self.f.name).read().strip().splitlines() if ln.strip()]
+        except Exception:
+            lines = []
+        os.unlink(self.f.name)
+        if not lines:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(x[1]) for x in lines if x[1].strip().replace(".", "").isdigit()]
+        mx = [float(x[2]) for x in lines if x[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for x in lines for k in range(4) if len(x) > 5 + k and "Active" in x[5 + k]})
+        loaded = [v for v in sm if mx and v > 0.5 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(lines)}
+
+
+def prefill_flops(w):
+    """Algorithmic FLOP of one prefill pass (per token and query head:
+    2d|Cand(i)| scoring + 4d(|I_i| S + |Win(i)|) attention), and of the
+    attention kernel alone."""
+    nw = w.W // w.S
+    score = attn = 0
+    for i in range(w.N):
+        cur = i // w.S
+        cand = max(0, cur - nw + 1)
+        win = i - max(0, (cur - nw + 1) * w.S) + 1
+        score += 2 * w.d * cand
+        attn += 4 * w.d * (min(w.K, cand) * w.S + win)
+    return score * w.B * w.Hq, attn * w.B * w.Hq
+
+
+def decode_bytes(w):
+    """Algorithmic bytes of one decode step: k'/b' of every candidate for every
+    head, plus the K chunks and the window of K and V per KV head."""
+    cur = (w.N - 1) // w.S
+    nw = w.W // w.S
+    cand = max(0, cur - nw + 1)
+    win = w.N - max(0, (cur - nw + 1) * w.S)
+    esz = 2 if w.dtype == "bf16" else 4
+    score = w.B * w.Hq * cand * (w.d * esz + 4)
+    gather = w.B * w.Hkv * (min(w.K, cand) * w.S + win) * w.d * esz * 2
+    q_out = w.B * w.Hq * w.d * esz * 2
+    return score, gather, q_out
+
+
+def traffic_for(kernel_file: str, kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu capture (profiles/traffic.json),
+    or None if absent or if the kernel's source changed since the capture."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+        e = d[kernel][workload]
+        src = os.path.join(ROOT, "chunk_wise_sparse_landmark_b200", "csrc", kernel_file)
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        return e["bytes_per_launch"] if e.get("source_sha") == h else None
+    except Exception:
+        return None
+
+
+def timed(fn, stream):
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    fn()
+    b.record(stream)
+    return a, b
+
+
+# ----------------------------------------------------------------- arms -----
+
+def run_prefill(w, dev, steps, warmup, stream):
+    x = prefill_inputs(w, device=dev)
+    cfg = H.config_of(w)
+    qc = (x["h"], x["w_down"], x["w_up"]) if w.d_model else None
+    pre = H.Prefill(cfg, dev, qcal_rank=w.qcal_rank)
+    ev = {"summaries": [], "score_topk": [], "attn_prefill": []}
+
+    def step(record):
+        if record:
+            ev["summaries"].append(timed(lambda: H.hils_build_summaries(cfg, x["k"], x["q_lmk"], pre.k_sum,
+                                                                        pre.b_sum, stream), stream))
+            ev["score_topk"].append(timed(lambda: H.hils_score_topk(cfg, x["q"], pre.k_sum, pre.b_sum, pre.idx,
+                                                                    pre.s_sel, pre.ws, False, qc, stream), stream))
+            ev["attn_prefill"].append(timed(lambda: H.hils_attn_prefill(cfg, x["q"], x["k"], x["v"], pre.idx,
+                                                                        pre.s_sel, pre.out, stream), stream))
+        else:
+            pre.run(x["q"], x["k"], x["v"], x["q_lmk"], qcal=qc, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            step(False)
+        H.hils_sync_status(stream)
+    return x, pre, step, ev
+
+
+def run_decode(w, dev, steps, warmup, stream):
+    x = decode_inputs(w, device=dev)
+    cfg = H.config_of(w)
+    dec = H.Decode(cfg, dev)
+    with torch.cuda.stream(stream):
+        a, b = timed(lambda: dec.summarize(x["k"], x["q_lmk"], stream), stream)
+        for _ in range(warmup):
+            dec.step(x["q"], x["k"], x["v"], stream)
+        H.hils_sync_status(stream)
+    summ_ms = a.elapsed_time(b)
+    ev = {"score_topk": [], "attn_decode": []}
+
+    def step():
+        ev["score_topk"].append(timed(lambda: H.hils_score_topk(cfg, x["q"], dec.k_sum, dec.b_sum, dec.idx,
+                                                                dec.s_sel, dec.ws_score, True, None, stream),
+                                      stream))
+        ev["attn_decode"].append(timed(lambda: H.hils_attn_decode(cfg, x["q"], x["k"], x["v"], dec.idx,
+                                                                  dec.s_sel, dec.out, dec.ws_attn, stream), stream))
+
+    return x, dec, step, ev, summ_ms
+
+
+def mean_ms(pairs):
+    return sum(a.elapsed_time(b) for a, b in pairs) / max(1, len(pairs))
+
+
+def device_time(stream, fn, steps, dist_on):
+    """Barrier + sync, K steps between CUDA events, sync; max over ranks (ms)."""
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(steps):
+            fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    if dist_on:
+        t = torch.tensor([ms], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms
+
+
+def e2e_prefill(w, x, pre, stream, steps, dist_on):
+    """Through the public API with host buffers: H2D of the step's inputs from
+    pinned memory, the prefill, D2H of the output, all inside the timed region."""
+    names = ["q", "k", "v", "q_lmk"] + (["h", "w_down", "w_up"] if w.d_model else [])
+    host = {n: x[n].to("cpu").pin_memory() for n in names}
+    devb = {n: torch.empty_like(x[n]) for n in names}
+    out_h = torch.empty(pre.out.shape, dtype=pre.out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+
+    def step():
+        for n in names:
+            devb[n].copy_(host[n], non_blocking=True)
+        qc = (devb["h"], devb["w_down"], devb["w_up"]) if w.d_model else None
+        pre.run(devb["q"], devb["k"], devb["v"], devb["q_lmk"], qcal=qc, stream=stream)
+        out_h.copy_(pre.out, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        step()
+    torch.cuda.synchronize()
+    ms = device_time(stream, step, steps, dist_on)
+    return ms / steps, h2d, d2h
+
+
+def cpu_baseline_prefill(w, x, budget_s=15.0, rows=None, seed=0):
+    """The oracle, as it stands, on the host cores, on a sample of positions:
+    summaries of the whole sequence amortised per position, plus scoring,
+    selection and attention of the sampled positions for every head."""
+    import numpy as np
+
+    import oracle
+
+    dm = oracle.Dims(B=1, Hq=w.Hq, Hkv=w.Hkv, N=w.N, d=w.d, S=w.S, W=w.W, K=w.K)
+    q = x["q"][:1].float().cpu().numpy()
+    k = x["k"][:1].float().cpu().numpy()
+    v = x["v"][:1].float().cpu().numpy()
+    ql = x["q_lmk"][:1].float().cpu().numpy()
+    t0 = time.perf_counter()
+    ks, bs = oracle.summaries(dm, k, ql)
+    t_summ = time.perf_counter() - t0
+    rng = np.random.default_rng(seed)
+    n = rows or 32
+    done = 0
+    t_rows = 0.0
+    while True:
+        sel = [(0, int(i)) for i in rng.integers(0, w.N, n)]
+        t0 = time.perf_counter()
+        qs = None
+        if w.d_model:
+            qs = oracle.qcal(dm, sel, q, x["h"][:1].float().cpu().numpy(), x["w_down"].float().cpu().numpy(),
+                             x["w_up"].float().cpu().numpy())
+        idx, ssel = oracle.select(dm, sel, q, k_sum=ks, b_sum=bs, qs=qs)
+        oracle.attend(dm, sel, q, k, v, idx, ssel)
+        t_rows += time.perf_counter() - t0
+        done += n
+        if rows is not None or t_rows > budget_s:
+            break
+    per_token = t_rows / done + t_summ / w.N
+    return 1.0 / per_token, done, t_summ, t_rows
+
+
+# ------------------------------------------------------------------ main -----
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="prefill_128k", choices=[k for k, v in WORKLOADS.items() if not v.decode])
+    ap.add_argument("--decode-workload", default="decode_512k")
+    ap.add_argument("--impl", default="hils", choices=["hils", "reference"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    ws, rank, local = dist_env()
+    dist_on = ws > 1
+    if args.impl == "reference":
+        return reference_arm(args, ws, rank)
+    if dist_on:
+        import datetime
+
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    torch.cuda.set_device(local)
+    dev = f"cuda:{local}"
+    H.load()
+    stream = torch.cuda.Stream()
+    pk, pk_kind = peaks()
+
+    w = WORKLOADS[args.workload]
+    x, pre, step, ev = run_prefill(w, dev, args.steps, args.warmup, stream)
+    with Clocks(local) as clk:
+        ms_total = device_time(stream, lambda: step(True), args.steps, dist_on)
+    H.hils_sync_status(stream)
+    clocks = clk.summary()
+    ms_step = ms_total / args.steps
+    tokens = w.B * w.N * ws
+    value = tokens / (ms_step / 1e3)
+    score_f, attn_f = prefill_flops(w)
+    t_attn = mean_ms(ev["attn_prefill"])
+    t_score = mean_ms(ev["score_topk"])
+    t_summ = mean_ms(ev["summaries"])
+    peak_tf = pk["bf16_tflops_sustained"]
+    ach = attn_f / (t_attn / 1e3) / 1e12
+    roofline = {"kernel": "attn_union_kernel (hils_attn_prefill)", "bound": "tensor", "achieved": round(ach, 2),
+                "peak": peak_tf, "unit": "TFLOP/s", "frac": round(ach / peak_tf, 4),
+                "traffic": traffic_for("attn_union.cu", "attn_union_kernel", w.name),
+                "peak_source": f"{pk_kind} bf16_tflops_sustained",
+                "algorithmic_flop_per_launch": attn_f}
+    per_kernel = {"summaries_ms": round(t_summ, 4), "score_topk_ms": round(t_score, 4),
+                  "attn_prefill_ms": round(t_attn, 4),
+                  "score_tflops_alg": round(score_f / (t_score / 1e3) / 1e12, 2)}
+    line = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.B, "seq_len": w.N, "n_q_heads": w.Hq, "n_kv_heads": w.Hkv,
+                       "head_dim": w.d, "chunk": w.S, "window": w.W, "top_k": w.K,
+                       "qcal_rank": w.qcal_rank, "parallelism": f"replica x{ws}",
+                       "l2": "inputs larger than L2 (q 1.07 GB, k/v 268 MB each)"},
+            "roofline": roofline, "kernels": per_kernel, "clocks": clocks,
+            "gpu_launches": (3 + (1 if w.d_model else 0)) * args.steps}
+    if not args.no_e2e:
+        e2e_ms, h2d, d2h = e2e_prefill(w, x, pre, stream, max(2, args.steps // 3), dist_on)
+        line["e2e"] = {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                       "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)}
+    del pre
+    if not args.no_decode:
+        wd = WORKLOADS[args.decode_workload]
+        xd, dec, dstep, dev_ev, summ_ms = run_decode(wd, dev, args.steps, args.warmup, stream)
+        d_ms = device_time(stream, dstep, args.steps * 5, dist_on) / (args.steps * 5)
+        H.hils_sync_status(stream)
+        sb, gb, qb = decode_bytes(wd)
+        t_att = mean_ms(dev_ev["attn_decode"])
+        t_sc = mean_ms(dev_ev["score_topk"])
+        hbm = pk["hbm_gbs"]
+        line["decode"] = {
+            "workload": wd.name, "value": round(wd.B * ws / (d_ms / 1e3), 1), "unit": "seqs/s",
+            "ms_per_step": round(d_ms, 4), "score_topk_ms": round(t_sc, 4), "attn_decode_ms": round(t_att, 4),
+            "roofline": {"kernel": "attn_decode_partial (hils_attn_decode, KV gather)", "bound": "hbm",
+                         "achieved": round(gb / (t_att / 1e3) / 1e9, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(gb / (t_att / 1e3) / 1e9 / hbm, 4), "traffic": None,
+                         "peak_source": f"{pk_kind} hbm_gbs", "algorithmic_bytes_per_launch": gb},
+            "score_roofline": {"bound": "hbm", "achieved": round(sb / (t_sc / 1e3) / 1e9, 1), "peak": hbm,
+                               "unit": "GB/s", "frac": round(sb / (t_sc / 1e3) / 1e9 / hbm, 4),
+                               "algorithmic_bytes_per_launch": sb},
+            "step_roofline_frac": round((sb + gb + qb) / (d_ms / 1e3) / 1e9 / hbm, 4),
+            "summaries_ms": round(summ_ms, 3),
+            "summaries_gbs": round((wd.B * wd.Hkv * wd.N * wd.d * 2 + 2 * wd.B * wd.Hq * wd.C * wd.d * 2)
+                                   / (summ_ms / 1e3) / 1e9, 1),
+            "gpu_launches": 4 * args.steps * 5}
+        del xd, dec
+    if rank == 0 and not args.no_cpu:
+        v, done, t_s, t_r = cpu_baseline_prefill(w, x)
+        line["cpu_baseline"] = {"value": round(v, 2), "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
+                                "sample": f"{done} random positions of {w.name} (all {w.Hq} heads; summaries of "
+                                          f"the whole sequence amortised per position; {t_s:.1f}s summaries + "
+                                          f"{t_r:.1f}s rows)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist_on:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+def reference_arm(args, ws, rank):
+    """The oracle as the reference implementation, on the host cores."""
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    x = prefill_inputs(w, device="cuda" if torch.cuda.is_available() else "cpu")
+    vals = []
+    for it in range(args.warmup + args.steps):
+        v, done, _, _ = cpu_baseline_prefill(w, x, rows=8, seed=it)
+        if it >= args.warmup:
+            vals.append(v)
+    v = statistics.mean(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": round(v, 2), "unit": "tokens/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * 8 / v, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.B, "seq_len": w.N, "parallelism": "host cores"},
+            "cpu_baseline": {"value": round(v, 2), "unit": "tokens/s", "kind": "oracle", "cores": os.cpu_count(),
+                             "sample": f"8 random positions of {w.name} per step, all heads"},
+            "e2e": {"value": round(v, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()
