@@ -95,7 +95,7 @@ class Clocks:
         sm = [float(x[1]) for x in lines if x[1].strip().replace(".", "").isdigit()]
         mx = [float(x[2]) for x in lines if x[2].strip().replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[k] for x in lines for k in range(4) if len(x) > 5 + k and "Active" in x[5 + k]})
+        reasons = sorted({names[k] for x in lines for k in range(4) if len(x) > 5 + k and x[5 + k].strip() == "Active"})
         loaded = [v for v in sm if mx and v > 0.5 * max(mx)] or sm
         return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": max(mx) if mx else None,
                 "reasons": reasons, "samples": len(lines)}
