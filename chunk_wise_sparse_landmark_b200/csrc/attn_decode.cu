@@ -18,6 +18,8 @@
 // workspace; a second kernel folds the records of a head and divides.
 // Tiles arrive through 1-D bulk copies (TMA) into a two-stage shared-memory
 // ring; every wait is bounded.
+#include <mutex>
+
 #include "launch.h"
 
 namespace hils {
@@ -288,6 +290,12 @@ cudaError_t go_g(const Shape& s, const void* q, const void* k, const void* v, co
 
 }  // namespace
 
+// Fixed scratch for hils_attn_decode_noalloc: the split-KV partial records
+// live here instead of in a caller-provided workspace.  Every GPU that loads
+// the library holds this array until the process exits.
+constexpr size_t kStaticScratchFloats = size_t(1) << 20;  // 4 MiB
+static __device__ __align__(256) float g_decode_scratch[kStaticScratchFloats];
+
 size_t decode_attn_workspace(const Shape& s) {
   const int nsplit = pick_nsplit(s);
   return (size_t)s.B * s.Hq * nsplit * (s.d + 2) * sizeof(float);
@@ -304,6 +312,34 @@ cudaError_t launch_attn_decode(const Shape& s, const void* q, const void* k, con
     if (s.d == 128 && s.S == 64) return go_g<__nv_bfloat16, 128, 64>(s, q, k, v, idx, s_sel, out, ws, st, ctx);
   }
   return cudaErrorInvalidValue;
+}
+
+size_t decode_static_scratch_bytes() { return kStaticScratchFloats * sizeof(float); }
+
+// Host code cannot pass g_decode_scratch itself (its host-side name is a
+// stand-in, not a device address).  The device address is looked up once per
+// device, with that device current, and cached.
+cudaError_t launch_attn_decode_static(const Shape& s, const void* q, const void* k, const void* v,
+                                      const int32_t* idx, const float* s_sel, void* out, cudaStream_t st,
+                                      const DevCtx& ctx) {
+  static std::mutex mu;
+  static void* addr[64] = {nullptr};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  void* ws = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (!addr[dev]) {
+      void* p = nullptr;
+      e = cudaGetSymbolAddress(&p, g_decode_scratch);
+      if (e != cudaSuccess) return e;
+      addr[dev] = p;
+    }
+    ws = addr[dev];
+  }
+  return launch_attn_decode(s, q, k, v, idx, s_sel, out, ws, st, ctx);
 }
 
 }  // namespace hils

@@ -235,6 +235,27 @@ hils_status_t hils_attn_decode(const hils_config_t* cfg, const void* q, const vo
   return HILS_OK;
 }
 
+hils_status_t hils_attn_decode_noalloc(const hils_config_t* cfg, const void* q, const void* k_cache,
+                                       const void* v_cache, const int32_t* idx, const float* s_sel, void* out,
+                                       void* stream) {
+  Shape s;
+  HILS_TRY(make_shape(cfg, &s, true));
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(idx) || !aligned16(s_sel) ||
+      !aligned16(out))
+    return fail(HILS_ERR_INVALID_ARG, "hils_attn_decode_noalloc: NULL or unaligned pointer");
+  const size_t need = decode_attn_workspace(s), have = decode_static_scratch_bytes();
+  if (need > have)
+    return fail(HILS_ERR_UNSUPPORTED,
+                "hils_attn_decode_noalloc: this configuration needs %zu bytes of scratch, the library's fixed "
+                "scratch holds %zu; use hils_attn_decode with a workspace",
+                need, have);
+  DevCtx ctx;
+  HILS_TRY(dev_ctx(&ctx));
+  HILS_LAUNCH(launch_attn_decode_static(s, q, k_cache, v_cache, idx, s_sel, out, (cudaStream_t)stream, ctx),
+              "attn_decode_noalloc");
+  return HILS_OK;
+}
+
 hils_status_t hils_sync_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");

@@ -52,4 +52,10 @@ size_t decode_attn_workspace(const Shape& s);
 cudaError_t launch_attn_decode(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
                                const float* s_sel, void* out, void* ws, cudaStream_t st, const DevCtx& ctx);
 
+// decode attention with its partial records in a fixed device array (no allocation)
+size_t decode_static_scratch_bytes();
+cudaError_t launch_attn_decode_static(const Shape& s, const void* q, const void* k, const void* v,
+                                      const int32_t* idx, const float* s_sel, void* out, cudaStream_t st,
+                                      const DevCtx& ctx);
+
 }  // namespace hils

@@ -24,6 +24,7 @@ EXPORTS = (
     "hils_score_topk",
     "hils_attn_prefill",
     "hils_attn_decode",
+    "hils_attn_decode_noalloc",
     "hils_workspace_bytes",
     "hils_sync_status",
     "hils_last_error",
@@ -80,6 +81,7 @@ def load() -> ctypes.CDLL:
         lib.hils_score_topk.argtypes = [C, P, ctypes.POINTER(QCal), P, P, P, P, P, ctypes.c_size_t, ctypes.c_int32, P]
         lib.hils_attn_prefill.argtypes = [C, P, P, P, P, P, P, P]
         lib.hils_attn_decode.argtypes = [C, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+        lib.hils_attn_decode_noalloc.argtypes = [C, P, P, P, P, P, P, P]
         lib.hils_workspace_bytes.argtypes = [C, ctypes.c_int32, ctypes.c_int32]
         lib.hils_workspace_bytes.restype = ctypes.c_size_t
         lib.hils_sync_status.argtypes = [P]
@@ -90,7 +92,7 @@ def load() -> ctypes.CDLL:
         lib.hils_set_fault_injection.restype = None
         lib.hils_version.restype = ctypes.c_char_p
         for n in ("hils_build_summaries", "hils_score_topk", "hils_attn_prefill", "hils_attn_decode",
-                  "hils_sync_status"):
+                  "hils_attn_decode_noalloc", "hils_sync_status"):
             getattr(lib, n).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -155,6 +157,13 @@ def hils_attn_decode(cfg: Config, q, k_cache, v_cache, idx, s_sel, out, workspac
     ws_bytes = workspace.numel() * workspace.element_size()
     _check(load().hils_attn_decode(ctypes.byref(cfg), _p(q), _p(k_cache), _p(v_cache), _p(idx), _p(s_sel), _p(out),
                                    _p(workspace), ws_bytes, _stream(stream)))
+
+
+def hils_attn_decode_noalloc(cfg: Config, q, k_cache, v_cache, idx, s_sel, out, stream=None):
+    """hils_attn_decode for callers that cannot allocate device memory: the
+    partial records go to the library's fixed device scratch (see hils.h)."""
+    _check(load().hils_attn_decode_noalloc(ctypes.byref(cfg), _p(q), _p(k_cache), _p(v_cache), _p(idx), _p(s_sel),
+                                           _p(out), _stream(stream)))
 
 
 def hils_sync_status(stream=None):

@@ -151,6 +151,33 @@ hils_status_t hils_attn_decode(const hils_config_t* cfg, const void* q, const vo
                                const int32_t* idx, const float* s_sel, void* out, void* workspace, size_t ws_bytes,
                                void* stream);
 
+/*
+ * hils_attn_decode without a workspace argument.  The paper has no
+ * counterpart of this call: it exists for callers that cannot allocate
+ * device memory for the call, e.g. a serving engine that has given all free
+ * HBM to its own KV-cache pool, or a plug-in interface that hands over only
+ * input and output buffers and has no allocator to offer.  Same arguments,
+ * result and errors as hils_attn_decode, minus the workspace.
+ *
+ * The split-KV partial records go to one fixed device array inside the
+ * library (4 MiB, i.e. B * Hq * nsplit * (d + 2) floats at most; nsplit is
+ * the per-(sequence, group) split count, about 4 * SMs / (B * Hkv)).  Every
+ * GPU that loads the library holds that array until the process exits.  A
+ * configuration that needs more returns HILS_ERR_UNSUPPORTED with a message
+ * naming both sizes; hils_workspace_bytes(cfg, HILS_WS_ATTN_DECODE, 0) gives
+ * the need.  The call never allocates or frees memory.
+ *
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  All calls share the one array and it keeps the last call's
+ * contents: every record a call reads is written by the same call, so nothing
+ * needs clearing, but two calls that overlap on the GPU (different streams,
+ * or other threads) race on the array and must be serialised by the caller.
+ */
+hils_status_t hils_attn_decode_noalloc(const hils_config_t* cfg, const void* q, const void* k_cache,
+                                       const void* v_cache, const int32_t* idx, const float* s_sel, void* out,
+                                       void* stream);
+
 enum { HILS_WS_SCORE_PREFILL = 0, HILS_WS_SCORE_DECODE = 1, HILS_WS_ATTN_DECODE = 2 };
 
 /* Bytes of workspace the call `which` needs for this configuration (0 if none);
