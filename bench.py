@@ -191,15 +191,23 @@ def run_decode(w, dev, steps, warmup, stream):
             dec.step(x["q"], x["k"], x["v"], stream)
         H.hils_sync_status(stream)
     summ_ms = a.elapsed_time(b)
+    # The decode step is a few microsecond-scale launches: capture each call in a
+    # CUDA graph (after the warm-up above has done every once-per-device set-up)
+    # so that host-side argument handling cannot show up as device time.
+    g_score, g_attn = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_score, stream=stream):
+        H.hils_score_topk(cfg, x["q"], dec.k_sum, dec.b_sum, dec.idx, dec.s_sel, dec.ws_score, True, None,
+                          torch.cuda.current_stream())
+    with torch.cuda.graph(g_attn, stream=stream):
+        H.hils_attn_decode(cfg, x["q"], x["k"], x["v"], dec.idx, dec.s_sel, dec.out, dec.ws_attn,
+                           torch.cuda.current_stream())
     ev = {"score_topk": [], "attn_decode": []}
 
     def step():
-        ev["score_topk"].append(timed(lambda: H.hils_score_topk(cfg, x["q"], dec.k_sum, dec.b_sum, dec.idx,
-                                                                dec.s_sel, dec.ws_score, True, None, stream),
-                                      stream))
-        ev["attn_decode"].append(timed(lambda: H.hils_attn_decode(cfg, x["q"], x["k"], x["v"], dec.idx,
-                                                                  dec.s_sel, dec.out, dec.ws_attn, stream), stream))
+        ev["score_topk"].append(timed(g_score.replay, stream))
+        ev["attn_decode"].append(timed(g_attn.replay, stream))
 
+    dec._graphs = (g_score, g_attn)
     return x, dec, step, ev, summ_ms
 
 
@@ -301,6 +309,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--seq-len", type=int, default=0, help="override N of the prefill workload (profiling)")
+    ap.add_argument("--decode-seq-len", type=int, default=0, help="override L of the decode workload (profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -320,6 +330,8 @@ def main():
     pk, pk_kind = peaks()
 
     w = WORKLOADS[args.workload]
+    if args.seq_len:
+        w = w.scaled(N=args.seq_len, needles_per_head=min(w.needles_per_head, max(1, args.seq_len // 2048)))
     x, pre, step, ev = run_prefill(w, dev, args.steps, args.warmup, stream)
     with Clocks(local) as clk:
         ms_total = device_time(stream, lambda: step(True), args.steps, dist_on)
@@ -358,6 +370,8 @@ def main():
     del pre
     if not args.no_decode:
         wd = WORKLOADS[args.decode_workload]
+        if args.decode_seq_len:
+            wd = wd.scaled(N=args.decode_seq_len)
         xd, dec, dstep, dev_ev, summ_ms = run_decode(wd, dev, args.steps, args.warmup, stream)
         d_ms = device_time(stream, dstep, args.steps * 5, dist_on) / (args.steps * 5)
         H.hils_sync_status(stream)

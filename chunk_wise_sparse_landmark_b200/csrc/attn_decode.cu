@@ -21,6 +21,7 @@
 #include <mutex>
 
 #include "launch.h"
+#include "tmap.h"
 
 namespace hils {
 namespace {
@@ -252,9 +253,7 @@ int pick_nsplit(const Shape& s) {
   const int cur = (s.N - 1) / s.S;
   const int nwin = cur - max(0, cur - s.nw + 1) + 1;
   const int nunits = s.K + nwin;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = device_sm_count();
   const int groups = s.B * s.Hkv;
   int nsplit = (sms * 4 + groups - 1) / groups;
   // at most 16 units per CTA, at least one unit per CTA
@@ -269,7 +268,8 @@ cudaError_t go(const Shape& s, const void* q, const void* k, const void* v, cons
   const int nsplit = pick_nsplit(s);
   const size_t smem = sizeof(DecSmem<T, D, S, G>);
   auto kern = attn_decode_partial<T, D, S, G>;
-  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = ensure_dynamic_smem((const void*)kern, (int)smem);
+  if (e != cudaSuccess) return e;
   kern<<<dim3(nsplit, s.Hkv, s.B), kThreads, smem, st>>>(s, (const T*)q, (const T*)k, (const T*)v, idx, s_sel,
                                                          (float*)ws, nsplit, ctx);
   attn_decode_merge<T, D><<<s.B * s.Hq, D, 0, st>>>(s, (const float*)ws, (T*)out, nsplit);

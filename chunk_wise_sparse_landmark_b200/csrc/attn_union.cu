@@ -360,7 +360,7 @@ cudaError_t launch_attn_prefill_tc(const Shape& s, const void* q, const void* k,
   e = make_tmap_bf16(&tmv, v, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
   const size_t smem = sizeof(Smem) + 1024;
-  e = cudaFuncSetAttribute(attn_union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  e = ensure_dynamic_smem((const void*)attn_union_kernel, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((s.N + QB - 1) / QB, s.Hkv, s.B);
   attn_union_kernel<<<grid, THREADS, smem, st>>>(s, tmk, tmv, (const __nv_bfloat16*)q, idx, s_sel,

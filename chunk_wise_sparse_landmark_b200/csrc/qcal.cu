@@ -239,7 +239,7 @@ cudaError_t launch_qcal_tc(const Shape& s, const void* q, const void* h, const v
     if (e != cudaSuccess) return e;
   }
   const size_t smem = sizeof(SmemQ) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(qcal_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = ensure_dynamic_smem((const void*)qcal_kernel, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((s.N + MQ - 1) / MQ, s.B);
   qcal_kernel<<<grid, THREADS, smem, st>>>(s, d_model, tmh, tmwd, tmwu, (const __nv_bfloat16*)q,

@@ -16,6 +16,7 @@
 //    workspace, then a per-(sequence, group) radix select that picks the K
 //    best chunks deterministically (ties: smaller chunk index).
 #include "launch.h"
+#include "tmap.h"
 
 namespace hils {
 namespace {
@@ -289,9 +290,7 @@ cudaError_t go_decode(const Shape& s, const void* q, const void* k_sum, const fl
     constexpr int LPR = D / 8 >= 32 ? 32 : D / 8;
     const int rows_per_block = 8 * (32 / LPR);
     int gx = (ncand + rows_per_block - 1) / rows_per_block;
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int sms = device_sm_count();
     const int want = (sms * 8 + s.B * s.Hkv - 1) / (s.B * s.Hkv);
     if (gx > want) gx = want;
     decode_scores<T, D, G><<<dim3(gx, s.Hkv, s.B), 256, 0, st>>>(s, (const T*)q, (const T*)k_sum, b_sum, s_all,

@@ -308,7 +308,7 @@ cudaError_t launch_score_topk_tc(const Shape& s, const void* q, const void* k_su
   cudaError_t e = make_tmap_bf16(&tmk, k_sum, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
   const size_t smem = sizeof(SmemS) + 1024;
-  e = cudaFuncSetAttribute(score_topk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  e = ensure_dynamic_smem((const void*)score_topk_tc_kernel, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((s.N + MQ - 1) / MQ, s.Hkv, s.B);
   score_topk_tc_kernel<<<grid, THREADS, smem, st>>>(s, tmk, (const __nv_bfloat16*)q, b_sum, idx, s_sel, ctx);

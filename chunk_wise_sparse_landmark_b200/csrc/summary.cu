@@ -12,6 +12,7 @@
 // are fp32.  The entropy is evaluated as (m + log Z) - sum p*l, which avoids
 // 0*log 0.  The kernel is HBM-bound: it reads K once and writes G summaries.
 #include "launch.h"
+#include "tmap.h"
 
 namespace hils {
 namespace {
@@ -82,9 +83,7 @@ template <typename T, int D, int S, int G>
 cudaError_t go(const Shape& s, const void* k, const void* q_lmk, void* k_sum, float* b_sum, cudaStream_t st) {
   const long long units = (long long)s.B * s.Hkv * s.C;
   if (units == 0) return cudaSuccess;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = device_sm_count();
   const long long grid = units < (long long)sms * 8 ? units : (long long)sms * 8;
   summaries_kernel<T, D, S, G><<<(unsigned)grid, kThreads, 0, st>>>(s, (const T*)k, (const T*)q_lmk, (T*)k_sum,
                                                                      b_sum);

@@ -14,4 +14,11 @@ namespace hils {
 cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                            const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swizzle);
 
+// Multiprocessor count of the current device (queried once per device).
+int device_sm_count();
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (device, kernel);
+// later calls for the same pair return immediately.
+cudaError_t ensure_dynamic_smem(const void* func, int bytes);
+
 }  // namespace hils
