@@ -1,0 +1,299 @@
+// Hierarchical-softmax sparse attention, bf16 prefill (d = 128, S = 64, G = 4).
+//
+// hyper.ai summary of arXiv 2607.02980 (HiLS-Attention), section 方法
+// (Method): each selected chunk is attended with its own softmax, the chunk
+// outputs are weighted by exp(s^_{i,c}) / Z^_i and the chunk-aligned window by
+// Z_swa / Z^_i, Z^_i = sum_c exp(s^_{i,c}) + Z_swa.  The section's hardware
+// paragraph groups adjacent queries and attends the union of their chunks;
+// here a warp groups 2 adjacent positions (8 query-head rows of one GQA group)
+// and walks the union of their two chunk lists.
+//
+// Why this shape.  On inputs whose adjacent positions pick unrelated chunks,
+// a loaded 64-key chunk is used by about one position (4 rows).  Staging
+// chunks in shared memory for a block of positions then buys almost no reuse
+// but costs a shared-memory write and read per chunk and ties each ring slot
+// up while one warp computes.  Instead every warp gathers its own chunks
+// straight from L2 into tensor-core fragments with coalesced 16-byte loads:
+//
+//   S^T (64 keys x 8 rows)   = K_c (keys x d)  . Q^T (d x rows)
+//   O^T (128 d x 8 rows)    += V_c^T (d x keys) . P^T (keys x rows)
+//
+// bf16 mma.sync m16n8k16, fp32 accumulation.  Keys are the MMA's M, so the
+// 8 rows fill N = 8 with no padding when both positions chose the chunk.  The
+// contraction index d of S^T is permuted (consistently for K and Q) so that a
+// thread's eight elements of two k-steps are one 16-byte vector; the M index
+// of O^T is permuted so that a thread owns 16 consecutive output dims; P^T
+// reaches B-fragment layout by an in-register 8x8 transpose (movmatrix).
+//
+// Row state (per query-head row): m2 = reference exponent (log2 units, >= all
+// exponents used so far), den = sum of weights, acc = weighted values.
+// Selected chunk: P_j = e^{s_j - mu}/Z_c * e^{s^ - m}, den += e^{s^ - m}.
+// Window chunk: P_j = e^{s_j - m}, den += sum_j P_j; m is raised (acc and den
+// rescaled) when a window logit exceeds it.  out = acc / den.
+#include <climits>
+
+#include "launch.h"
+#include "tmap.h"
+
+namespace hils {
+namespace {
+
+constexpr int D = 128, S = 64, G = 4;
+constexpr int WARPS = 8;            // per CTA; 2 positions per warp
+constexpr int THREADS = WARPS * 32;
+constexpr int POS_PER_CTA = 2 * WARPS;
+
+HILS_DI uint4 ldg16(const __nv_bfloat16* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
+
+// element e (0..7) of a 16-byte vector of bf16, as the low half-word
+HILS_DI uint32_t half_of(const uint4& v, int e) {
+  const uint32_t w = e < 2 ? v.x : e < 4 ? v.y : e < 6 ? v.z : v.w;
+  return (e & 1) ? (w >> 16) : (w & 0xffffu);
+}
+
+HILS_DI uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+__global__ void __launch_bounds__(THREADS, 2)
+    attn_warp_kernel(Shape s, const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                     const __nv_bfloat16* __restrict__ v, const int32_t* __restrict__ idx,
+                     const float* __restrict__ s_sel, __nv_bfloat16* __restrict__ out, DevCtx ctx) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gq = lane >> 2, c4 = lane & 3;  // fragment coordinates
+  const int g = blockIdx.y, b = blockIdx.z;
+  const int p0 = blockIdx.x * POS_PER_CTA + warp * 2;  // the warp's two positions p0, p0 + 1
+  if (p0 >= s.N) return;
+  const int K = s.K;
+  const int cur = p0 / S;  // both positions share their chunk (p0 is even)
+  const int ncand = max(0, cur - s.nw + 1);
+  const bool valid1 = p0 + 1 < s.N;
+  const long long kvbase = ((long long)b * s.Hkv + g) * (long long)s.N * D;
+  const __nv_bfloat16* kb = k + kvbase;
+  const __nv_bfloat16* vb = v + kvbase;
+
+  // rows of the warp: n = 0..7 -> position p0 + n/4, head n%4.
+  // B operand of S^T: row gq; the thread's rows for S^T columns / O^T columns: 2*c4, 2*c4+1
+  uint32_t qf[4][4];  // [d block j][b0(2j), b1(2j), b0(2j+1), b1(2j+1)]
+  {
+    const int pos = p0 + (gq >> 2);
+    const bool ok = (gq >> 2) == 0 || valid1;
+    const __nv_bfloat16* qr = q + (((long long)b * s.Hq + g * G + (gq & 3)) * s.N + (ok ? pos : p0)) * D;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint4 u = ok ? ldg16(qr + 32 * j + 8 * c4) : make_uint4(0, 0, 0, 0);
+      qf[j][0] = u.x;
+      qf[j][1] = u.y;
+      qf[j][2] = u.z;
+      qf[j][3] = u.w;
+    }
+  }
+  // this thread's two rows (columns of S^T / O^T): position my_q, heads my_h, my_h + 1
+  const int my_q = c4 >> 1;  // 0 or 1
+  const int my_h = 2 * (c4 & 1);
+  const int my_pos = p0 + my_q;
+  const bool my_valid = my_q == 0 || valid1;
+
+  float acc[8][4];
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+  float m2[2], den[2] = {0.f, 0.f};
+  // chunk lists of the two positions (broadcast loads, every lane walks both)
+  const int32_t* L0 = idx + (((long long)b * s.Hkv + g) * s.N + p0) * K;
+  const int32_t* L1 = L0 + K;
+  const float* ss[2];
+#pragma unroll
+  for (int r = 0; r < 2; ++r) ss[r] = s_sel + (((long long)b * s.Hq + g * G + my_h + r) * s.N + my_pos) * K;
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    float mx = -INFINITY;
+    if (my_valid)
+      for (int x = 0; x < K; ++x) mx = fmaxf(mx, __ldg(ss[r] + x));
+    m2[r] = mx * kLog2e;
+  }
+  const float sl2 = s.scale * kLog2e;
+  const int wc0 = max(0, cur - s.nw + 1);
+  int cu0 = 0, cu1 = 0;  // cursors into L0, L1
+  const int len1 = valid1 ? K : 0;
+  auto head = [&](const int32_t* Lx, int& cu, int len) -> int {
+    while (cu < len) {
+      const int c = __ldg(Lx + cu);
+      if (c >= 0 && c < ncand) return c;
+      if (c >= ncand) raise_status(ctx, kStatusBadIndex);
+      ++cu;  // skip -1 padding and invalid entries
+    }
+    return INT_MAX;
+  };
+
+  for (int step = 0;; ++step) {
+    int c, slot_me = -1;
+    bool win, part0, part1;
+    if (step <= cur - wc0) {
+      c = wc0 + step;
+      win = true;
+      part0 = true;
+      part1 = valid1;
+    } else {
+      const int a0 = head(L0, cu0, K), a1 = head(L1, cu1, len1);
+      c = min(a0, a1);
+      if (c == INT_MAX) break;
+      win = false;
+      part0 = a0 == c;
+      part1 = a1 == c;
+      if (my_q == 0 && part0) slot_me = cu0;
+      if (my_q == 1 && part1) slot_me = cu1;
+      if (part0) ++cu0;
+      if (part1) ++cu1;
+    }
+    const bool my_part = my_valid && (my_q == 0 ? part0 : part1);
+    float a2[2] = {-INFINITY, -INFINITY};
+    if (!win && my_part) {
+      a2[0] = __ldg(ss[0] + slot_me) * kLog2e;
+      a2[1] = __ldg(ss[1] + slot_me) * kLog2e;
+    }
+    const __nv_bfloat16* kc = kb + (long long)c * S * D;
+    const __nv_bfloat16* vc = vb + (long long)c * S * D;
+    // the current chunk may end past the sequence: clamp key rows to the last
+    // valid one (those keys are causally masked, the load must stay in bounds)
+    const int kmax = min(S - 1, s.N - 1 - c * S);
+
+    // ---- S^T = K_c Q^T : 4 m-tiles (16 keys) x 8 k-steps (16 d)
+    float sc[4][4];
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt) sc[mt][0] = sc[mt][1] = sc[mt][2] = sc[mt][3] = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint4 ka[4], kb8[4];
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt) {
+        ka[mt] = ldg16(kc + min(16 * mt + gq, kmax) * D + 32 * j + 8 * c4);
+        kb8[mt] = ldg16(kc + min(16 * mt + gq + 8, kmax) * D + 32 * j + 8 * c4);
+      }
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt) {
+        const uint32_t A0[4] = {ka[mt].x, kb8[mt].x, ka[mt].y, kb8[mt].y};
+        const uint32_t A1[4] = {ka[mt].z, kb8[mt].z, ka[mt].w, kb8[mt].w};
+        mma_bf16_16816(sc[mt], A0, qf[j][0], qf[j][1]);
+        mma_bf16_16816(sc[mt], A1, qf[j][2], qf[j][3]);
+      }
+    }
+    // ---- per-row weights; this thread holds keys 16mt+gq (+8) of rows 2c4, 2c4+1
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      float mx = -INFINITY;
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+        for (int hi = 0; hi < 2; ++hi) {
+          const int key = 16 * mt + gq + 8 * hi;
+          float t = sc[mt][2 * hi + r] * sl2;
+          if (!my_part || (win && c * S + key > my_pos)) t = -INFINITY;
+          sc[mt][2 * hi + r] = t;
+          mx = fmaxf(mx, t);
+        }
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      float base = mx;
+      if (my_part && win && mx > m2[r]) {
+        const float f = exp2f(m2[r] - mx);
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          acc[mt][r] *= f;
+          acc[mt][2 + r] *= f;
+        }
+        den[r] *= f;
+        m2[r] = mx;
+      }
+      if (win) base = m2[r];
+      float z = 0.f;
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+        for (int hi = 0; hi < 2; ++hi) {
+          const float t = sc[mt][2 * hi + r];
+          const float p = (my_part && t != -INFINITY) ? exp2f(t - base) : 0.f;
+          sc[mt][2 * hi + r] = p;
+          z += p;
+        }
+      z += __shfl_xor_sync(0xffffffffu, z, 4);
+      z += __shfl_xor_sync(0xffffffffu, z, 8);
+      z += __shfl_xor_sync(0xffffffffu, z, 16);
+      if (my_part) {
+        if (win) {
+          den[r] += z;
+        } else {
+          const float wgt = exp2f(a2[r] - m2[r]);  // <= 1
+          den[r] += wgt;
+          const float f = wgt / z;
+#pragma unroll
+          for (int mt = 0; mt < 4; ++mt) {
+            sc[mt][r] *= f;
+            sc[mt][2 + r] *= f;
+          }
+        }
+      }
+    }
+    // ---- O^T += V_c^T P^T : 8 m-tiles (16 d) x 4 k-steps (16 keys)
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      // P^T B fragment for keys 16kk..16kk+15 via 8x8 transposes of the S^T C fragment
+      const uint32_t b0 = movmatrix_trans(pack_bf16x2(sc[kk][0], sc[kk][1]));
+      const uint32_t b1 = movmatrix_trans(pack_bf16x2(sc[kk][2], sc[kk][3]));
+      // V rows 16kk + {2c, 2c+1, 2c+8, 2c+9}, dims [16 gq, 16 gq + 16)
+      const int key0 = 16 * kk + 2 * c4;
+      uint4 va[4][2];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int key = min(key0 + (e & 1) + 8 * (e >> 1), kmax);
+        va[e][0] = ldg16(vc + key * D + 16 * gq);
+        va[e][1] = ldg16(vc + key * D + 16 * gq + 8);
+      }
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        uint32_t A[4];
+        A[0] = half_of(va[0][0], mt) | (half_of(va[1][0], mt) << 16);
+        A[1] = half_of(va[0][1], mt) | (half_of(va[1][1], mt) << 16);
+        A[2] = half_of(va[2][0], mt) | (half_of(va[3][0], mt) << 16);
+        A[3] = half_of(va[2][1], mt) | (half_of(va[3][1], mt) << 16);
+        mma_bf16_16816(acc[mt], A, b0, b1);
+      }
+    }
+  }
+
+  // epilogue: this thread's rows 2c4, 2c4+1 (position my_pos, heads my_h, my_h+1),
+  // output dims [16 gq, 16 gq + 16): d = 16 gq + mt <- acc[mt][r], 16 gq + 8 + mt <- acc[mt][2 + r]
+  if (my_valid) {
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const float inv = 1.f / den[r];
+      __nv_bfloat16* o = out + (((long long)b * s.Hq + g * G + my_h + r) * s.N + my_pos) * D + 16 * gq;
+      uint4 lo, hi;
+      lo.x = pack_bf16x2(acc[0][r] * inv, acc[1][r] * inv);
+      lo.y = pack_bf16x2(acc[2][r] * inv, acc[3][r] * inv);
+      lo.z = pack_bf16x2(acc[4][r] * inv, acc[5][r] * inv);
+      lo.w = pack_bf16x2(acc[6][r] * inv, acc[7][r] * inv);
+      hi.x = pack_bf16x2(acc[0][2 + r] * inv, acc[1][2 + r] * inv);
+      hi.y = pack_bf16x2(acc[2][2 + r] * inv, acc[3][2 + r] * inv);
+      hi.z = pack_bf16x2(acc[4][2 + r] * inv, acc[5][2 + r] * inv);
+      hi.w = pack_bf16x2(acc[6][2 + r] * inv, acc[7][2 + r] * inv);
+      reinterpret_cast<uint4*>(o)[0] = lo;
+      reinterpret_cast<uint4*>(o)[1] = hi;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_attn_prefill_tc(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
+                                   const float* s_sel, void* out, cudaStream_t st, const DevCtx& ctx) {
+  if (s.d != D || s.S != S || s.G != G || s.K > 64) return cudaErrorNotSupported;
+  dim3 grid((s.N + POS_PER_CTA - 1) / POS_PER_CTA, s.Hkv, s.B);
+  attn_warp_kernel<<<grid, THREADS, 0, st>>>(s, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
+                                             (const __nv_bfloat16*)v, idx, s_sel, (__nv_bfloat16*)out, ctx);
+  return cudaGetLastError();
+}
+
+}  // namespace hils

@@ -46,6 +46,7 @@ constexpr uint32_t DCOL = 256;                // D stage sd, head h at DCOL + 12
 struct __align__(1024) SmemS {
   unsigned char b[NSTB][G][2][BBOX];
   unsigned long long buf[CAP][MQ];  // column per row: conflict-free per-thread access
+  alignas(16) float bt[2][G][TCH];  // b' of the tile in each accumulator stage
   uint64_t bfull[NSTB], bempty[NSTB], dfull[2], dempty[2], afull, done;
   uint32_t tmem;
 };
@@ -225,27 +226,37 @@ __global__ void __launch_bounds__(THREADS, 1)
         break;
       }
       tc_fence_after();
+      // b' of this tile, 4 heads x 32 chunks: one coalesced element per epilogue
+      // thread into shared memory, then a barrier among the four epilogue warps
+      {
+        const int hh = r >> 5, jj = r & 31, cc = c0 + jj;
+        sm.bt[sd][hh][jj] = cc < s.C ? __ldg(b_sum + ((long long)b * s.Hq + g * G + hh) * s.C + cc) : 0.f;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      // group score g = max_h (acc * scale + b'); identical in both passes
       uint32_t v[G][32];
 #pragma unroll
       for (int h = 0; h < G; ++h) tmem_ld32(lane_addr + DCOL + sd * 128 + h * 32, v[h]);
       tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.dempty[sd]);
-      // group score g = max_h (acc * scale + b'), identical in both passes
       float gv[TCH];
 #pragma unroll
       for (int j = 0; j < TCH; ++j) gv[j] = -INFINITY;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const float* bp = b_sum + ((long long)b * s.Hq + g * G + h) * s.C + c0;
+        const float4* bt4 = reinterpret_cast<const float4*>(sm.bt[sd][h]);
 #pragma unroll
-        for (int j = 0; j < TCH; ++j) {
-          const float bb = c0 + j < s.C ? __ldg(bp + j) : 0.f;
-          gv[j] = fmaxf(gv[j], __fmaf_rn(__uint_as_float(v[h][j]), scale, bb));
+        for (int j4 = 0; j4 < TCH / 4; ++j4) {
+          const float4 bb = bt4[j4];
+          gv[4 * j4 + 0] = fmaxf(gv[4 * j4 + 0], __fmaf_rn(__uint_as_float(v[h][4 * j4 + 0]), scale, bb.x));
+          gv[4 * j4 + 1] = fmaxf(gv[4 * j4 + 1], __fmaf_rn(__uint_as_float(v[h][4 * j4 + 1]), scale, bb.y));
+          gv[4 * j4 + 2] = fmaxf(gv[4 * j4 + 2], __fmaf_rn(__uint_as_float(v[h][4 * j4 + 2]), scale, bb.z));
+          gv[4 * j4 + 3] = fmaxf(gv[4 * j4 + 3], __fmaf_rn(__uint_as_float(v[h][4 * j4 + 3]), scale, bb.w));
         }
       }
       if (pass == 0) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.dempty[sd]);
 #pragma unroll
         for (int j = 0; j < TCH; ++j) {
           const int c = c0 + j;
@@ -261,24 +272,37 @@ __global__ void __launch_bounds__(THREADS, 1)
           else tau = tau - 1ull;  // pass 2 takes keys >= the K-th key
         }
       } else {
+        uint32_t selmask = 0;
 #pragma unroll
         for (int j = 0; j < TCH; ++j) {
           const int c = c0 + j;
-          if (c < ncand && make_key(gv[j], c) > tau && nsel < K) {
-            idx[row_idx + nsel] = c;
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-              const float bb = __ldg(b_sum + ((long long)b * s.Hq + g * G + h) * s.C + c);
-              s_sel[(((long long)b * s.Hq + g * G + h) * s.N + i) * K + nsel] =
-                  __fmaf_rn(__uint_as_float(v[h][j]), scale, bb);
-            }
-            ++nsel;
-          }
+          if (c < ncand && make_key(gv[j], c) > tau) selmask |= 1u << j;
         }
+        if (selmask != 0) {
+          const int base = nsel;
+#pragma unroll
+          for (int j = 0; j < TCH; ++j) {
+            if ((selmask >> j) & 1u) {
+              const int slot = base + __popc(selmask & ((1u << j) - 1u));
+              if (slot < K) {
+                idx[row_idx + slot] = c0 + j;
+#pragma unroll
+                for (int h = 0; h < G; ++h)
+                  s_sel[(((long long)b * s.Hq + g * G + h) * s.N + i) * K + slot] =
+                      __fmaf_rn(__uint_as_float(v[h][j]), scale, sm.bt[sd][h][j]);
+              }
+            }
+          }
+          nsel = base + __popc(selmask);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.dempty[sd]);
       }
     }
     if (valid && ok) {
       if (nsel != min(ncand, K)) raise_status(ctx, kStatusBadIndex);
+      nsel = min(nsel, K);
       for (int x = nsel; x < K; ++x) {
         idx[row_idx + x] = -1;
 #pragma unroll
