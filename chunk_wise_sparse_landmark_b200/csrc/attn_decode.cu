@@ -249,6 +249,239 @@ __global__ void __launch_bounds__(D) attn_decode_merge(Shape s, const float* __r
   out[bh * D + e] = from_f32<T>(num / den);
 }
 
+// ---------------------------------------------------------------------------
+// bf16, d = 128, S = 64: every warp gathers its tiles straight from HBM into
+// tensor-core fragments (no shared-memory staging) and computes
+//   S^T (64 keys x 8 cols) = K_tile . Q^T,   O^T (128 x 8 cols) += V_tile^T . P^T
+// with the group's G <= 8 heads as the N = 8 columns (bf16 mma.sync, fp32
+// accumulation).  Same fragment layouts as the prefill attention kernel: the
+// contraction index d of S^T and the M index of O^T are permuted so that all
+// loads are 16-byte vectors, and P^T reaches B-fragment layout by an 8x8
+// in-register transpose.  Each warp folds its units with a running maximum
+// per head; the CTA folds its warps in shared memory and writes one record
+// per head, like the CUDA-core kernel above.
+constexpr int kMmaWarps = 4;
+
+HILS_DI uint4 ldg16_bf(const __nv_bfloat16* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
+HILS_DI uint32_t half_word(const uint4& v, int e) {
+  const uint32_t w = e < 2 ? v.x : e < 4 ? v.y : e < 6 ? v.z : v.w;
+  return (e & 1) ? (w >> 16) : (w & 0xffffu);
+}
+HILS_DI uint32_t mov_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+template <int G>
+__global__ void __launch_bounds__(kMmaWarps * 32) attn_decode_mma(Shape s, const __nv_bfloat16* __restrict__ q,
+                                                                  const __nv_bfloat16* __restrict__ k,
+                                                                  const __nv_bfloat16* __restrict__ v,
+                                                                  const int32_t* __restrict__ idx,
+                                                                  const float* __restrict__ s_sel,
+                                                                  float* __restrict__ ws, int nsplit, DevCtx ctx) {
+  constexpr int D = 128, S = 64;
+  __shared__ float red_acc[kMmaWarps][G][D];
+  __shared__ float red_m[kMmaWarps][G], red_d[kMmaWarps][G];
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gq = lane >> 2, c4 = lane & 3;
+  const int L = s.N, pos = L - 1, cur = pos / S;
+  const int ncand = max(0, cur - s.nw + 1);
+  const int wc0 = max(0, cur - s.nw + 1);
+  const int nunits = s.K + (cur - wc0 + 1);
+  const int32_t* ir = idx + ((long long)b * s.Hkv + g) * s.K;
+  const long long kvbase = ((long long)b * s.Hkv + g) * (long long)L * D;
+  // Q^T as the B operand of S^T: column gq = head gq (zero past G)
+  uint32_t qf[4][4];
+  {
+    const bool ok = gq < G;
+    const __nv_bfloat16* qr = q + ((long long)b * s.Hq + g * G + (ok ? gq : 0)) * D;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint4 u = ok ? ldg16_bf(qr + 32 * j + 8 * c4) : make_uint4(0, 0, 0, 0);
+      qf[j][0] = u.x;
+      qf[j][1] = u.y;
+      qf[j][2] = u.z;
+      qf[j][3] = u.w;
+    }
+  }
+  // this thread's columns 2c4, 2c4+1 (heads; >= G are padding)
+  float acc[8][4];
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+  float M[2] = {-INFINITY, -INFINITY}, den[2] = {0.f, 0.f};
+
+  // units of this CTA: u = split + nsplit * t; of this warp: every kMmaWarps-th of those
+  for (int u = split + nsplit * warp; u < nunits; u += nsplit * kMmaWarps) {
+    int j0, nk;
+    bool sel;
+    int slot = -1;
+    if (u < s.K) {
+      const int c = ir[u];
+      if (c < 0) continue;
+      if (c >= ncand) {
+        if (lane == 0) raise_status(ctx, kStatusBadIndex);
+        continue;
+      }
+      sel = true;
+      slot = u;
+      j0 = c * S;
+      nk = S;
+    } else {
+      sel = false;
+      j0 = (wc0 + (u - s.K)) * S;
+      nk = min(S, L - j0);
+    }
+    const __nv_bfloat16* kc = k + kvbase + (long long)j0 * D;
+    const __nv_bfloat16* vc = v + kvbase + (long long)j0 * D;
+    const int kmax = nk - 1;
+    float sc[4][4];
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt) sc[mt][0] = sc[mt][1] = sc[mt][2] = sc[mt][3] = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint4 ka[4], kb8[4];
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt) {
+        ka[mt] = ldg16_bf(kc + min(16 * mt + gq, kmax) * D + 32 * j + 8 * c4);
+        kb8[mt] = ldg16_bf(kc + min(16 * mt + gq + 8, kmax) * D + 32 * j + 8 * c4);
+      }
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt) {
+        const uint32_t A0[4] = {ka[mt].x, kb8[mt].x, ka[mt].y, kb8[mt].y};
+        const uint32_t A1[4] = {ka[mt].z, kb8[mt].z, ka[mt].w, kb8[mt].w};
+        mma_bf16_16816(sc[mt], A0, qf[j][0], qf[j][1]);
+        mma_bf16_16816(sc[mt], A1, qf[j][2], qf[j][3]);
+      }
+    }
+    // per column (head): m = max logit, l = sum e^{s-m}; log-weight lam
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int hcol = 2 * c4 + r;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+        for (int hi = 0; hi < 2; ++hi) {
+          float t = sc[mt][2 * hi + r] * s.scale;
+          if (16 * mt + gq + 8 * hi >= nk) t = -INFINITY;
+          sc[mt][2 * hi + r] = t;
+          mx = fmaxf(mx, t);
+        }
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      float l = 0.f;
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+        for (int hi = 0; hi < 2; ++hi) {
+          const float t = sc[mt][2 * hi + r];
+          const float p = t == -INFINITY ? 0.f : __expf(t - mx);
+          sc[mt][2 * hi + r] = p;
+          l += p;
+        }
+      l += __shfl_xor_sync(0xffffffffu, l, 4);
+      l += __shfl_xor_sync(0xffffffffu, l, 8);
+      l += __shfl_xor_sync(0xffffffffu, l, 16);
+      float lam = mx;
+      if (sel && hcol < G) lam = __ldg(s_sel + ((long long)b * s.Hq + g * G + hcol) * s.K + slot) - __logf(l);
+      if (hcol >= G) lam = -INFINITY;
+      const float Mn = fmaxf(M[r], lam);
+      if (Mn == -INFINITY) {
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt) sc[mt][r] = sc[mt][2 + r] = 0.f;
+        continue;
+      }
+      const float fo = __expf(M[r] - Mn), fu = __expf(lam - Mn);
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        acc[mt][r] *= fo;
+        acc[mt][2 + r] *= fo;
+      }
+      den[r] = den[r] * fo + fu * l;
+      M[r] = Mn;
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt) {
+        sc[mt][r] *= fu;
+        sc[mt][2 + r] *= fu;
+      }
+    }
+    // O^T += V^T P^T
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      const uint32_t b0 = mov_trans(pack_bf16x2(sc[kk][0], sc[kk][1]));
+      const uint32_t b1 = mov_trans(pack_bf16x2(sc[kk][2], sc[kk][3]));
+      const int key0 = 16 * kk + 2 * c4;
+      uint4 va[4][2];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int key = min(key0 + (e & 1) + 8 * (e >> 1), kmax);
+        va[e][0] = ldg16_bf(vc + key * D + 16 * gq);
+        va[e][1] = ldg16_bf(vc + key * D + 16 * gq + 8);
+      }
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        uint32_t A[4];
+        A[0] = half_word(va[0][0], mt) | (half_word(va[1][0], mt) << 16);
+        A[1] = half_word(va[0][1], mt) | (half_word(va[1][1], mt) << 16);
+        A[2] = half_word(va[2][0], mt) | (half_word(va[3][0], mt) << 16);
+        A[3] = half_word(va[2][1], mt) | (half_word(va[3][1], mt) << 16);
+        mma_bf16_16816(acc[mt], A, b0, b1);
+      }
+    }
+  }
+  // fold the warps: thread holds dims [16 gq, 16 gq + 16) of columns 2c4, 2c4+1
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int hcol = 2 * c4 + r;
+    if (hcol < G) {
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        red_acc[warp][hcol][16 * gq + mt] = acc[mt][r];
+        red_acc[warp][hcol][16 * gq + 8 + mt] = acc[mt][2 + r];
+      }
+      if (gq == 0) {
+        red_m[warp][hcol] = M[r];
+        red_d[warp][hcol] = den[r];
+      }
+    }
+  }
+  __syncthreads();
+  for (int o = threadIdx.x; o < G * D; o += kMmaWarps * 32) {
+    const int h = o / D, e = o % D;
+    float Mx = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kMmaWarps; ++w) Mx = fmaxf(Mx, red_m[w][h]);
+    float num = 0.f, dd = 0.f;
+#pragma unroll
+    for (int w = 0; w < kMmaWarps; ++w) {
+      if (red_m[w][h] == -INFINITY) continue;
+      const float f = __expf(red_m[w][h] - Mx);
+      num += f * red_acc[w][h][e];
+      dd += f * red_d[w][h];
+    }
+    float* rec = ws + (((long long)b * s.Hq + g * G + h) * nsplit + split) * (D + 2);
+    rec[2 + e] = num;
+    if (e == 0) {
+      rec[0] = Mx;
+      rec[1] = dd;
+    }
+  }
+}
+
+template <int G>
+cudaError_t go_mma(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
+                   const float* s_sel, void* out, void* ws, int nsplit, cudaStream_t st, const DevCtx& ctx) {
+  attn_decode_mma<G><<<dim3(nsplit, s.Hkv, s.B), kMmaWarps * 32, 0, st>>>(
+      s, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, idx, s_sel, (float*)ws, nsplit,
+      ctx);
+  attn_decode_merge<__nv_bfloat16, 128><<<s.B * s.Hq, 128, 0, st>>>(s, (const float*)ws, (__nv_bfloat16*)out,
+                                                                     nsplit);
+  return cudaGetLastError();
+}
+
 int pick_nsplit(const Shape& s) {
   const int cur = (s.N - 1) / s.S;
   const int nwin = cur - max(0, cur - s.nw + 1) + 1;
@@ -308,8 +541,14 @@ cudaError_t launch_attn_decode(const Shape& s, const void* q, const void* k, con
     if (s.d == 64 && s.S == 64) return go_g<float, 64, 64>(s, q, k, v, idx, s_sel, out, ws, st, ctx);
     if (s.d == 128 && s.S == 64) return go_g<float, 128, 64>(s, q, k, v, idx, s_sel, out, ws, st, ctx);
     if (s.d == 128 && s.S == 32) return go_g<float, 128, 32>(s, q, k, v, idx, s_sel, out, ws, st, ctx);
-  } else {
-    if (s.d == 128 && s.S == 64) return go_g<__nv_bfloat16, 128, 64>(s, q, k, v, idx, s_sel, out, ws, st, ctx);
+  } else if (s.d == 128 && s.S == 64) {
+    const int nsplit = pick_nsplit(s);
+    switch (s.G) {
+      case 1: return go_mma<1>(s, q, k, v, idx, s_sel, out, ws, nsplit, st, ctx);
+      case 2: return go_mma<2>(s, q, k, v, idx, s_sel, out, ws, nsplit, st, ctx);
+      case 4: return go_mma<4>(s, q, k, v, idx, s_sel, out, ws, nsplit, st, ctx);
+      case 8: return go_mma<8>(s, q, k, v, idx, s_sel, out, ws, nsplit, st, ctx);
+    }
   }
   return cudaErrorInvalidValue;
 }

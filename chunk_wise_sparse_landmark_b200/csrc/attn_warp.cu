@@ -21,8 +21,9 @@
 // bf16 mma.sync m16n8k16, fp32 accumulation.  Keys are the MMA's M, so the
 // 8 rows fill N = 8 with no padding when both positions chose the chunk.  The
 // contraction index d of S^T is permuted (consistently for K and Q) so that a
-// thread's eight elements of two k-steps are one 16-byte vector; the M index
-// of O^T is permuted so that a thread owns 16 consecutive output dims; P^T
+// thread's sixteen elements of four k-steps are one 32-byte vector and each
+// warp load covers whole 128-byte lines; the M index of O^T is permuted so
+// that the value loads of a key row are one contiguous line as well; P^T
 // reaches B-fragment layout by an in-register 8x8 transpose (movmatrix).
 //
 // Row state (per query-head row): m2 = reference exponent (log2 units, >= all
@@ -39,11 +40,18 @@ namespace hils {
 namespace {
 
 constexpr int D = 128, S = 64, G = 4;
-constexpr int WARPS = 8;            // per CTA; 2 positions per warp
+constexpr int WARPS = 4;            // per CTA; 2 positions per warp
 constexpr int THREADS = WARPS * 32;
 constexpr int POS_PER_CTA = 2 * WARPS;
 
 HILS_DI uint4 ldg16(const __nv_bfloat16* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
+
+// 32 consecutive bytes (16 bf16) of read-only global memory; p is 32-byte aligned
+HILS_DI void ldg32(const __nv_bfloat16* p, uint32_t (&w)[8]) {
+  asm volatile("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+               : "l"(p));
+}
 
 // element e (0..7) of a 16-byte vector of bf16, as the low half-word
 HILS_DI uint32_t half_of(const uint4& v, int e) {
@@ -57,7 +65,7 @@ HILS_DI uint32_t movmatrix_trans(uint32_t x) {
   return y;
 }
 
-__global__ void __launch_bounds__(THREADS, 2)
+__global__ void __launch_bounds__(THREADS, 3)
     attn_warp_kernel(Shape s, const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                      const __nv_bfloat16* __restrict__ v, const int32_t* __restrict__ idx,
                      const float* __restrict__ s_sel, __nv_bfloat16* __restrict__ out, DevCtx ctx) {
@@ -76,18 +84,20 @@ __global__ void __launch_bounds__(THREADS, 2)
 
   // rows of the warp: n = 0..7 -> position p0 + n/4, head n%4.
   // B operand of S^T: row gq; the thread's rows for S^T columns / O^T columns: 2*c4, 2*c4+1
-  uint32_t qf[4][4];  // [d block j][b0(2j), b1(2j), b0(2j+1), b1(2j+1)]
+  // d is permuted: for k-step ks = 4jj + t (jj = 0,1; t = 0..3) thread c holds
+  // logical k {2c, 2c+1} at physical d 64jj + 16c + 4t + {0,1} and {2c+8, 2c+9}
+  // at 64jj + 16c + 4t + {2,3}, so one 32-byte load feeds four k-steps
+  uint32_t qf[2][8];  // [jj][2t] = b0(ks), [2t+1] = b1(ks)
   {
     const int pos = p0 + (gq >> 2);
     const bool ok = (gq >> 2) == 0 || valid1;
     const __nv_bfloat16* qr = q + (((long long)b * s.Hq + g * G + (gq & 3)) * s.N + (ok ? pos : p0)) * D;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint4 u = ok ? ldg16(qr + 32 * j + 8 * c4) : make_uint4(0, 0, 0, 0);
-      qf[j][0] = u.x;
-      qf[j][1] = u.y;
-      qf[j][2] = u.z;
-      qf[j][3] = u.w;
+    for (int jj = 0; jj < 2; ++jj) {
+      ldg32(qr + 64 * jj + 16 * c4, qf[jj]);
+      if (!ok)
+#pragma unroll
+        for (int x = 0; x < 8; ++x) qf[jj][x] = 0u;
     }
   }
   // this thread's two rows (columns of S^T / O^T): position my_q, heads my_h, my_h + 1
@@ -164,19 +174,17 @@ __global__ void __launch_bounds__(THREADS, 2)
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt) sc[mt][0] = sc[mt][1] = sc[mt][2] = sc[mt][3] = 0.f;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      uint4 ka[4], kb8[4];
+    for (int jj = 0; jj < 2; ++jj) {
 #pragma unroll
       for (int mt = 0; mt < 4; ++mt) {
-        ka[mt] = ldg16(kc + min(16 * mt + gq, kmax) * D + 32 * j + 8 * c4);
-        kb8[mt] = ldg16(kc + min(16 * mt + gq + 8, kmax) * D + 32 * j + 8 * c4);
-      }
+        uint32_t ka[8], kb8[8];  // key rows 16mt+gq and 16mt+gq+8, d [64jj + 16c, +16)
+        ldg32(kc + min(16 * mt + gq, kmax) * D + 64 * jj + 16 * c4, ka);
+        ldg32(kc + min(16 * mt + gq + 8, kmax) * D + 64 * jj + 16 * c4, kb8);
 #pragma unroll
-      for (int mt = 0; mt < 4; ++mt) {
-        const uint32_t A0[4] = {ka[mt].x, kb8[mt].x, ka[mt].y, kb8[mt].y};
-        const uint32_t A1[4] = {ka[mt].z, kb8[mt].z, ka[mt].w, kb8[mt].w};
-        mma_bf16_16816(sc[mt], A0, qf[j][0], qf[j][1]);
-        mma_bf16_16816(sc[mt], A1, qf[j][2], qf[j][3]);
+        for (int t = 0; t < 4; ++t) {
+          const uint32_t A[4] = {ka[2 * t], kb8[2 * t], ka[2 * t + 1], kb8[2 * t + 1]};
+          mma_bf16_16816(sc[mt], A, qf[jj][2 * t], qf[jj][2 * t + 1]);
+        }
       }
     }
     // ---- per-row weights; this thread holds keys 16mt+gq (+8) of rows 2c4, 2c4+1
@@ -242,14 +250,15 @@ __global__ void __launch_bounds__(THREADS, 2)
       // P^T B fragment for keys 16kk..16kk+15 via 8x8 transposes of the S^T C fragment
       const uint32_t b0 = movmatrix_trans(pack_bf16x2(sc[kk][0], sc[kk][1]));
       const uint32_t b1 = movmatrix_trans(pack_bf16x2(sc[kk][2], sc[kk][3]));
-      // V rows 16kk + {2c, 2c+1, 2c+8, 2c+9}, dims [16 gq, 16 gq + 16)
+      // V rows 16kk + {2c, 2c+1, 2c+8, 2c+9}, dims [8 gq, 8 gq + 8) and [64 + 8 gq, 64 + 8 gq + 8):
+      // O^T row r of m-tile mt is output dim 8 gq + mt (r = gq) or 64 + 8 gq + mt (r = gq + 8)
       const int key0 = 16 * kk + 2 * c4;
       uint4 va[4][2];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int key = min(key0 + (e & 1) + 8 * (e >> 1), kmax);
-        va[e][0] = ldg16(vc + key * D + 16 * gq);
-        va[e][1] = ldg16(vc + key * D + 16 * gq + 8);
+        va[e][0] = ldg16(vc + key * D + 8 * gq);
+        va[e][1] = ldg16(vc + key * D + 64 + 8 * gq);
       }
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt) {
@@ -264,12 +273,12 @@ __global__ void __launch_bounds__(THREADS, 2)
   }
 
   // epilogue: this thread's rows 2c4, 2c4+1 (position my_pos, heads my_h, my_h+1),
-  // output dims [16 gq, 16 gq + 16): d = 16 gq + mt <- acc[mt][r], 16 gq + 8 + mt <- acc[mt][2 + r]
+  // output dims d = 8 gq + mt <- acc[mt][r] and 64 + 8 gq + mt <- acc[mt][2 + r]
   if (my_valid) {
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
       const float inv = 1.f / den[r];
-      __nv_bfloat16* o = out + (((long long)b * s.Hq + g * G + my_h + r) * s.N + my_pos) * D + 16 * gq;
+      __nv_bfloat16* o = out + (((long long)b * s.Hq + g * G + my_h + r) * s.N + my_pos) * D;
       uint4 lo, hi;
       lo.x = pack_bf16x2(acc[0][r] * inv, acc[1][r] * inv);
       lo.y = pack_bf16x2(acc[2][r] * inv, acc[3][r] * inv);
@@ -279,8 +288,8 @@ __global__ void __launch_bounds__(THREADS, 2)
       hi.y = pack_bf16x2(acc[2][2 + r] * inv, acc[3][2 + r] * inv);
       hi.z = pack_bf16x2(acc[4][2 + r] * inv, acc[5][2 + r] * inv);
       hi.w = pack_bf16x2(acc[6][2 + r] * inv, acc[7][2 + r] * inv);
-      reinterpret_cast<uint4*>(o)[0] = lo;
-      reinterpret_cast<uint4*>(o)[1] = hi;
+      *reinterpret_cast<uint4*>(o + 8 * gq) = lo;
+      *reinterpret_cast<uint4*>(o + 64 + 8 * gq) = hi;
     }
   }
 }

@@ -212,6 +212,8 @@ hils_status_t hils_attn_prefill(const hils_config_t* cfg, const void* q, const v
   if (s.dtype == HILS_F32) {
     HILS_LAUNCH(launch_attn_prefill_simt(s, q, k, v, idx, s_sel, out, st, ctx), "attn_prefill_simt");
   } else {
+    if (((uintptr_t)q | (uintptr_t)k | (uintptr_t)v) & 31u)
+      return fail(HILS_ERR_INVALID_ARG, "hils_attn_prefill: bf16 q, k, v must be 32-byte aligned");
     HILS_LAUNCH(launch_attn_prefill_tc(s, q, k, v, idx, s_sel, out, st, ctx), "attn_prefill_tc");
   }
   return HILS_OK;

@@ -164,8 +164,20 @@ __global__ void __launch_bounds__(256) decode_scores(Shape s, const T* __restric
       const int h = g * G + hg;
       const T* kp = k_sum + (((long long)b * s.Hq + h) * s.C + c) * D + l * EPL;
       float acc = 0.f;
+      if constexpr (sizeof(T) == 2 && EPL == 8) {
+        // one 16-byte vector of bf16 per lane
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(kp));
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) acc = fmaf(qs[hg][l * EPL + e], to_f32(kp[e]), acc);
+        for (int x = 0; x < 4; ++x) {
+          const float2 f = bf16x2_to_f32x2(w[x]);
+          acc = fmaf(qs[hg][l * EPL + 2 * x], f.x, acc);
+          acc = fmaf(qs[hg][l * EPL + 2 * x + 1], f.y, acc);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) acc = fmaf(qs[hg][l * EPL + e], to_f32(kp[e]), acc);
+      }
 #pragma unroll
       for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
       const float sv = acc * s.scale + b_sum[((long long)b * s.Hq + h) * s.C + c];

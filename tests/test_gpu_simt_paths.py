@@ -129,7 +129,9 @@ def test_summaries_bf16_prefill_8k():
 
 
 def test_decode_wait_timeout_reports_status():
-    w = WORKLOADS["decode_512k"].scaled(name="dec_to", B=1, N=4096)
+    # the fp32 decode kernel stages tiles with bounded waits (the bf16 one loads
+    # straight into registers and has none)
+    w = WORKLOADS["tiny_f32"].scaled(name="dec_to", B=1, N=4096, Hq=8, Hkv=2, decode=True)
     x = _to_dev(decode_inputs(w))
     dec = H.Decode(H.config_of(w), DEV)
     dec.summarize(x["k"], x["q_lmk"])
