@@ -134,6 +134,8 @@ hils_status_t hils_build_summaries(const hils_config_t* cfg, const void* k, cons
   HILS_TRY(make_shape(cfg, &s, false));
   if (!aligned16(k) || !aligned16(q_lmk) || !aligned16(k_sum) || !aligned16(b_sum))
     return fail(HILS_ERR_INVALID_ARG, "hils_build_summaries: NULL or unaligned pointer");
+  if (s.dtype == HILS_BF16 && (((uintptr_t)k | (uintptr_t)q_lmk) & 31u))
+    return fail(HILS_ERR_INVALID_ARG, "hils_build_summaries: bf16 k and q_lmk must be 32-byte aligned");
   DevCtx ctx;
   HILS_TRY(dev_ctx(&ctx));
   HILS_LAUNCH(launch_summaries(s, k, q_lmk, k_sum, b_sum, (cudaStream_t)stream, ctx), "summaries");
