@@ -8,7 +8,7 @@ import torch
 import oracle
 from chunk_wise_sparse_landmark_b200 import hils as H
 from chunk_wise_sparse_landmark_b200.inputs import WORKLOADS, decode_inputs, prefill_inputs
-from tests.parity import TOL_BF16, TOL_F32, check_selection, forced_s_sel, to_np
+from tests.parity import KSUM_ATOL, TOL_BF16, TOL_F32, check_selection, forced_s_sel, to_np
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -84,7 +84,7 @@ def _decode_check(w, tol):
     if w.dtype == "f32":
         np.testing.assert_allclose(to_np(dec.k_sum), ks, rtol=0, atol=1e-5)
     else:  # one bf16 rounding of k'
-        assert (np.abs(to_np(dec.k_sum) - ks) <= np.abs(ks) * 2.0 ** -8 + 1e-6).all()
+        assert (np.abs(to_np(dec.k_sum) - ks) <= np.abs(ks) * 2.0 ** -8 + KSUM_ATOL).all()
     np.testing.assert_allclose(to_np(dec.b_sum), bs, rtol=0, atol=2e-5 if w.dtype == "bf16" else 1e-5)
     rows = [(b, w.N - 1) for b in range(w.B)]
     idx_or, ssel_or, s_all, g_all = oracle.select(dm, rows, q, k_sum=ks, b_sum=bs, want_all=True)
@@ -124,7 +124,7 @@ def test_summaries_bf16_prefill_8k():
     ks, bs = oracle.summaries(_dims(w), to_np(x["k"]), to_np(x["q_lmk"]))
     # k' is stored in bf16: error bounded by one bf16 rounding of |k'| (< 2^-8 relative)
     err_k = np.abs(to_np(ks_g) - ks)
-    assert (err_k <= np.abs(ks) * 2.0 ** -8 + 1e-6).all(), err_k.max()
+    assert (err_k <= np.abs(ks) * 2.0 ** -8 + KSUM_ATOL).all(), err_k.max()
     np.testing.assert_allclose(to_np(bs_g), bs, rtol=0, atol=2e-5)
 
 
