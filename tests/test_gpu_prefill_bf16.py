@@ -207,4 +207,6 @@ def test_qcal_zero_up_projection_changes_nothing():
     H.hils_sync_status()
     assert torch.equal(base.idx, qc.idx)
     assert torch.equal(base.s_sel, qc.s_sel)
-    assert torch.equal(base.out, qc.out)
+    # the attention adds chunk contributions with shared-memory atomics, so two
+    # runs may round differently in the last bf16 bit
+    torch.testing.assert_close(base.out.float(), qc.out.float(), atol=1e-3, rtol=2.0 ** -7)
