@@ -20,6 +20,7 @@
 // ring; every wait is bounded.
 #include <mutex>
 
+#include "gather_mma.cuh"
 #include "launch.h"
 #include "tmap.h"
 
@@ -254,24 +255,10 @@ __global__ void __launch_bounds__(D) attn_decode_merge(Shape s, const float* __r
 // tensor-core fragments (no shared-memory staging) and computes
 //   S^T (64 keys x 8 cols) = K_tile . Q^T,   O^T (128 x 8 cols) += V_tile^T . P^T
 // with the group's G <= 8 heads as the N = 8 columns (bf16 mma.sync, fp32
-// accumulation).  Same fragment layouts as the prefill attention kernel: the
-// contraction index d of S^T and the M index of O^T are permuted so that all
-// loads are 16-byte vectors, and P^T reaches B-fragment layout by an 8x8
-// in-register transpose.  Each warp folds its units with a running maximum
+// accumulation); fragment layouts and line-wide loads: gather_mma.cuh.  Each warp folds its units with a running maximum
 // per head; the CTA folds its warps in shared memory and writes one record
 // per head, like the CUDA-core kernel above.
 constexpr int kMmaWarps = 4;
-
-HILS_DI uint4 ldg16_bf(const __nv_bfloat16* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
-HILS_DI uint32_t half_word(const uint4& v, int e) {
-  const uint32_t w = e < 2 ? v.x : e < 4 ? v.y : e < 6 ? v.z : v.w;
-  return (e & 1) ? (w >> 16) : (w & 0xffffu);
-}
-HILS_DI uint32_t mov_trans(uint32_t x) {
-  uint32_t y;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
-  return y;
-}
 
 template <int G>
 __global__ void __launch_bounds__(kMmaWarps * 32) attn_decode_mma(Shape s, const __nv_bfloat16* __restrict__ q,
@@ -293,19 +280,8 @@ __global__ void __launch_bounds__(kMmaWarps * 32) attn_decode_mma(Shape s, const
   const int32_t* ir = idx + ((long long)b * s.Hkv + g) * s.K;
   const long long kvbase = ((long long)b * s.Hkv + g) * (long long)L * D;
   // Q^T as the B operand of S^T: column gq = head gq (zero past G)
-  uint32_t qf[4][4];
-  {
-    const bool ok = gq < G;
-    const __nv_bfloat16* qr = q + ((long long)b * s.Hq + g * G + (ok ? gq : 0)) * D;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint4 u = ok ? ldg16_bf(qr + 32 * j + 8 * c4) : make_uint4(0, 0, 0, 0);
-      qf[j][0] = u.x;
-      qf[j][1] = u.y;
-      qf[j][2] = u.z;
-      qf[j][3] = u.w;
-    }
-  }
+  uint32_t qf[2][8];
+  load_qcol(gq < G ? q + ((long long)b * s.Hq + g * G + gq) * D : nullptr, c4, qf);
   // this thread's columns 2c4, 2c4+1 (heads; >= G are padding)
   float acc[8][4];
 #pragma unroll
@@ -339,22 +315,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32) attn_decode_mma(Shape s, const
     float sc[4][4];
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt) sc[mt][0] = sc[mt][1] = sc[mt][2] = sc[mt][3] = 0.f;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      uint4 ka[4], kb8[4];
-#pragma unroll
-      for (int mt = 0; mt < 4; ++mt) {
-        ka[mt] = ldg16_bf(kc + min(16 * mt + gq, kmax) * D + 32 * j + 8 * c4);
-        kb8[mt] = ldg16_bf(kc + min(16 * mt + gq + 8, kmax) * D + 32 * j + 8 * c4);
-      }
-#pragma unroll
-      for (int mt = 0; mt < 4; ++mt) {
-        const uint32_t A0[4] = {ka[mt].x, kb8[mt].x, ka[mt].y, kb8[mt].y};
-        const uint32_t A1[4] = {ka[mt].z, kb8[mt].z, ka[mt].w, kb8[mt].w};
-        mma_bf16_16816(sc[mt], A0, qf[j][0], qf[j][1]);
-        mma_bf16_16816(sc[mt], A1, qf[j][2], qf[j][3]);
-      }
-    }
+    mma_st_tile(kc, kmax, gq, c4, qf, sc);
     // per column (head): m = max logit, l = sum e^{s-m}; log-weight lam
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
@@ -369,9 +330,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32) attn_decode_mma(Shape s, const
           sc[mt][2 * hi + r] = t;
           mx = fmaxf(mx, t);
         }
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      mx = col_max(mx);
       float l = 0.f;
 #pragma unroll
       for (int mt = 0; mt < 4; ++mt)
@@ -382,9 +341,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32) attn_decode_mma(Shape s, const
           sc[mt][2 * hi + r] = p;
           l += p;
         }
-      l += __shfl_xor_sync(0xffffffffu, l, 4);
-      l += __shfl_xor_sync(0xffffffffu, l, 8);
-      l += __shfl_xor_sync(0xffffffffu, l, 16);
+      l = col_sum(l);
       float lam = mx;
       if (sel && hcol < G) lam = __ldg(s_sel + ((long long)b * s.Hq + g * G + hcol) * s.K + slot) - __logf(l);
       if (hcol >= G) lam = -INFINITY;
@@ -409,38 +366,17 @@ __global__ void __launch_bounds__(kMmaWarps * 32) attn_decode_mma(Shape s, const
       }
     }
     // O^T += V^T P^T
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      const uint32_t b0 = mov_trans(pack_bf16x2(sc[kk][0], sc[kk][1]));
-      const uint32_t b1 = mov_trans(pack_bf16x2(sc[kk][2], sc[kk][3]));
-      const int key0 = 16 * kk + 2 * c4;
-      uint4 va[4][2];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int key = min(key0 + (e & 1) + 8 * (e >> 1), kmax);
-        va[e][0] = ldg16_bf(vc + key * D + 16 * gq);
-        va[e][1] = ldg16_bf(vc + key * D + 16 * gq + 8);
-      }
-#pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        uint32_t A[4];
-        A[0] = half_word(va[0][0], mt) | (half_word(va[1][0], mt) << 16);
-        A[1] = half_word(va[0][1], mt) | (half_word(va[1][1], mt) << 16);
-        A[2] = half_word(va[2][0], mt) | (half_word(va[3][0], mt) << 16);
-        A[3] = half_word(va[2][1], mt) | (half_word(va[3][1], mt) << 16);
-        mma_bf16_16816(acc[mt], A, b0, b1);
-      }
-    }
+    mma_ot_tile(vc, kmax, gq, c4, sc, acc);
   }
-  // fold the warps: thread holds dims [16 gq, 16 gq + 16) of columns 2c4, 2c4+1
+  // fold the warps: thread holds dims 8 gq + mt and 64 + 8 gq + mt of columns 2c4, 2c4+1
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
     const int hcol = 2 * c4 + r;
     if (hcol < G) {
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt) {
-        red_acc[warp][hcol][16 * gq + mt] = acc[mt][r];
-        red_acc[warp][hcol][16 * gq + 8 + mt] = acc[mt][2 + r];
+        red_acc[warp][hcol][8 * gq + mt] = acc[mt][r];
+        red_acc[warp][hcol][64 + 8 * gq + mt] = acc[mt][2 + r];
       }
       if (gq == 0) {
         red_m[warp][hcol] = M[r];

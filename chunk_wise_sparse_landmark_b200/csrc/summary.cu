@@ -11,6 +11,7 @@
 // (conflict-free column and row walks); logits, the softmax and the entropy
 // are fp32.  The entropy is evaluated as (m + log Z) - sum p*l, which avoids
 // 0*log 0.  The kernel is HBM-bound: it reads K once and writes G summaries.
+#include "gather_mma.cuh"
 #include "launch.h"
 #include "tmap.h"
 
@@ -125,25 +126,8 @@ cudaError_t go_t(const Shape& s, const void* k, const void* q_lmk, void* k_sum, 
 // on the tensor cores (bf16 mma.sync, fp32 accumulation), with the group's
 // G <= 8 landmark queries as the N = 8 columns.  P is split into bf16 hi + lo
 // parts (two MMAs) so k' keeps close to fp32 accuracy before its final bf16
-// rounding; the entropy uses the fp32 logits.  Loads are 32-byte (S^T) and
-// 16-byte (k'^T) vectors covering whole 128-byte lines; the second read of
-// the tile hits L1.  Fragment layouts as in the attention kernels.
-HILS_DI void ldg32_words(const __nv_bfloat16* p, uint32_t (&w)[8]) {
-  asm volatile("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-               : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
-               : "l"(p));
-}
-HILS_DI uint4 ldg16_words(const __nv_bfloat16* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
-HILS_DI uint32_t half_w(const uint4& v, int e) {
-  const uint32_t w = e < 2 ? v.x : e < 4 ? v.y : e < 6 ? v.z : v.w;
-  return (e & 1) ? (w >> 16) : (w & 0xffffu);
-}
-HILS_DI uint32_t movm_trans(uint32_t x) {
-  uint32_t y;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
-  return y;
-}
-
+// rounding; the entropy uses the fp32 logits.  Fragment layouts and
+// line-wide loads: gather_mma.cuh; the second read of the tile hits L1.
 template <int G>
 __global__ void __launch_bounds__(256) summaries_mma(Shape s, const __nv_bfloat16* __restrict__ k,
                                                      const __nv_bfloat16* __restrict__ q_lmk,
@@ -160,34 +144,11 @@ __global__ void __launch_bounds__(256) summaries_mma(Shape s, const __nv_bfloat1
     const __nv_bfloat16* kc = k + (((long long)b * s.Hkv + g) * s.N + (long long)c * S) * D;
     // Q'^T as the B operand: column gq = landmark query of head g*G + gq
     uint32_t qf[2][8];
-    {
-      const bool ok = gq < G;
-      const __nv_bfloat16* qr = q_lmk + (((long long)b * s.Hq + g * G + (ok ? gq : 0)) * s.C + c) * D;
-#pragma unroll
-      for (int jj = 0; jj < 2; ++jj) {
-        ldg32_words(qr + 64 * jj + 16 * c4, qf[jj]);
-        if (!ok)
-#pragma unroll
-          for (int x = 0; x < 8; ++x) qf[jj][x] = 0u;
-      }
-    }
+    load_qcol(gq < G ? q_lmk + (((long long)b * s.Hq + g * G + gq) * s.C + c) * D : nullptr, c4, qf);
     float sc[4][4];
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt) sc[mt][0] = sc[mt][1] = sc[mt][2] = sc[mt][3] = 0.f;
-#pragma unroll
-    for (int jj = 0; jj < 2; ++jj) {
-#pragma unroll
-      for (int mt = 0; mt < 4; ++mt) {
-        uint32_t ka[8], kb8[8];
-        ldg32_words(kc + (16 * mt + gq) * D + 64 * jj + 16 * c4, ka);
-        ldg32_words(kc + (16 * mt + gq + 8) * D + 64 * jj + 16 * c4, kb8);
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const uint32_t A[4] = {ka[2 * t], kb8[2 * t], ka[2 * t + 1], kb8[2 * t + 1]};
-          mma_bf16_16816(sc[mt], A, qf[jj][2 * t], qf[jj][2 * t + 1]);
-        }
-      }
-    }
+    mma_st_tile(kc, S - 1, gq, c4, qf, sc);
     // softmax per column, entropy = (m + log Z) - sum p l
     float phi[4][4], plo[4][4];
 #pragma unroll
@@ -199,9 +160,7 @@ __global__ void __launch_bounds__(256) summaries_mma(Shape s, const __nv_bfloat1
         sc[mt][2 + r] *= s.scale;
         mx = fmaxf(mx, fmaxf(sc[mt][r], sc[mt][2 + r]));
       }
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      mx = col_max(mx);
       float z = 0.f, zl = 0.f;
 #pragma unroll
       for (int mt = 0; mt < 4; ++mt)
@@ -213,11 +172,8 @@ __global__ void __launch_bounds__(256) summaries_mma(Shape s, const __nv_bfloat1
           z += e;
           zl += e * l;
         }
-#pragma unroll
-      for (int o = 4; o <= 16; o <<= 1) {
-        z += __shfl_xor_sync(0xffffffffu, z, o);
-        zl += __shfl_xor_sync(0xffffffffu, zl, o);
-      }
+      z = col_sum(z);
+      zl = col_sum(zl);
       const float inv = 1.f / z;
       const int hcol = 2 * c4 + r;
       if (hcol < G && gq == 0) b_sum[((long long)b * s.Hq + g * G + hcol) * s.C + c] = (mx + logf(z)) - zl * inv;
@@ -235,31 +191,8 @@ __global__ void __launch_bounds__(256) summaries_mma(Shape s, const __nv_bfloat1
     float acc[8][4];
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      const uint32_t bh0 = movm_trans(pack_bf16x2(phi[kk][0], phi[kk][1]));
-      const uint32_t bh1 = movm_trans(pack_bf16x2(phi[kk][2], phi[kk][3]));
-      const uint32_t bl0 = movm_trans(pack_bf16x2(plo[kk][0], plo[kk][1]));
-      const uint32_t bl1 = movm_trans(pack_bf16x2(plo[kk][2], plo[kk][3]));
-      const int key0 = 16 * kk + 2 * c4;
-      uint4 va[4][2];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int key = key0 + (e & 1) + 8 * (e >> 1);
-        va[e][0] = ldg16_words(kc + key * D + 8 * gq);
-        va[e][1] = ldg16_words(kc + key * D + 64 + 8 * gq);
-      }
-#pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        uint32_t A[4];
-        A[0] = half_w(va[0][0], mt) | (half_w(va[1][0], mt) << 16);
-        A[1] = half_w(va[0][1], mt) | (half_w(va[1][1], mt) << 16);
-        A[2] = half_w(va[2][0], mt) | (half_w(va[3][0], mt) << 16);
-        A[3] = half_w(va[2][1], mt) | (half_w(va[3][1], mt) << 16);
-        mma_bf16_16816(acc[mt], A, bh0, bh1);
-        mma_bf16_16816(acc[mt], A, bl0, bl1);
-      }
-    }
+    mma_ot_tile(kc, S - 1, gq, c4, phi, acc);
+    mma_ot_tile(kc, S - 1, gq, c4, plo, acc);
     // thread holds dims 8 gq + mt (acc[mt][r]) and 64 + 8 gq + mt (acc[mt][2 + r]) of columns 2c4 + r
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
