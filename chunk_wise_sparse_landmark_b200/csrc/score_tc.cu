@@ -9,23 +9,26 @@
 // position (same section), i.e. a causal GEMM Q~ (N x d) . K'^T (d x N/S).
 //
 // One CTA = 128 positions (the MMA's M) of one (sequence, KV group).  The
-// four heads' query tiles are written once into tensor memory and used as the
-// A operand of every MMA (256 TMEM columns); k' tiles of 32 chunks x 128 for
-// the four heads (32 KB) stream through a 2-stage TMA ring (128-byte swizzle,
-// chunks past C read as zero); the 4 x 32 fp32 accumulators are
-// double-buffered in tensor memory (256 columns).  Warp roles: 0 = TMA
-// producer, 1 = MMA issuer (and TMEM owner), 2..9 = epilogue: two threads per
-// position (its TMEM lane), one per half of each 32-chunk tile.
+// four heads' query tiles are written once into tensor memory (256 columns)
+// and serve as the A operand of every MMA; k' tiles of 64 chunks x 128 for the
+// four heads (64 KB) stream through a 3-stage TMA ring (128-byte swizzle,
+// chunks past C read as zero) into one 4 x 64-column fp32 accumulator.  A
+// thread that issues tcgen05.mma gets one instruction through every ~130
+// cycles whatever its N, so each head has its own issuing warp (warps 0..3,
+// lane 0; warp 0 also drives the TMA ring): together they keep the tensor
+// pipe busy.  Warps 4..11 are the epilogue: two threads per position (its
+// TMEM lane), one per 32-chunk half of each tile.
 //
 // Selection is exact and deterministic.  Pass 1 streams every tile; each
-// epilogue thread keeps the K largest keys of its half, key = (ordered bits of
-// g) << 32 | (~c) (larger g first, ties to the smaller c): candidates above
-// the current threshold go to a per-thread buffer of K + 16 entries that is
-// folded into a min-heap of size K whenever it could overflow.  After the
-// last tile the two halves of a row are merged, giving the row's K-th key.
-// Pass 2 recomputes the same tiles (same instructions, bit-identical scores)
-// and emits every candidate whose key is >= the K-th key, in ascending chunk
-// order (the halves exchange their per-tile counts), with each head's own s^.
+// epilogue thread keeps the multiset of the KT >= K largest group scores of
+// its half, sorted in registers, updated by branch-free insertion of the few
+// candidates above its current KT-th value.  After the last tile the row's
+// threshold tau (its K-th largest score) is the minimum over j < K of
+// max(a_j, b_{K-1-j}) for the two halves' sorted lists a, b, and A = the
+// number of scores above tau.  Pass 2 recomputes the same tiles (same
+// instructions, bit-identical scores) and emits, in ascending chunk order,
+// every candidate scoring above tau plus the first K - A scoring exactly tau
+// (ties go to the smaller chunk), with each head's own s^.
 #include "launch.h"
 #include "tmap.h"
 
@@ -33,75 +36,31 @@ namespace hils {
 namespace {
 
 constexpr int D = 128, G = 4;
-constexpr int MQ = 128;   // positions per CTA
-constexpr int TCH = 32;   // chunks per tile (MMA N)
+constexpr int MQ = 128;   // positions per CTA (MMA M, TMEM lanes)
+constexpr int TCH = 64;   // chunks per tile (MMA N)
 constexpr int HALF = TCH / 2;
-constexpr int NSTB = 2;   // k' ring stages
+constexpr int NST = 3;    // k' ring stages
 constexpr int KMAX = 64;
-constexpr int THREADS = 320;
+constexpr int NMMA = G;   // MMA-issuing warps, one per head
 constexpr int EPI = 256;  // epilogue threads
-constexpr uint32_t BBOX = TCH * 128;          // one [32 chunks x 64 d] bf16 box
-constexpr uint32_t BSTAGE = G * 2 * BBOX;     // 32 KB
+constexpr int THREADS = 32 * NMMA + EPI;
+constexpr int STG = 16;   // survivors staged per thread and round
+constexpr uint32_t BBOX = TCH * 128;       // one [64 chunks x 64 d] bf16 box
+constexpr uint32_t BSTAGE = G * 2 * BBOX;  // 64 KB
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t ACOL = 0;                  // A: head h at ACOL + 64 h
-constexpr uint32_t DCOL = 256;                // D stage sd, head h at DCOL + 128 sd + 32 h
+constexpr uint32_t ACOL = 0;    // A: head h at ACOL + 64 h
+constexpr uint32_t DCOL = 256;  // D: head h at DCOL + 64 h
 
-// Fixed part of the shared memory; the per-thread key buffers follow it
-// (K + 16 entries per thread, one column per thread).
 struct __align__(1024) SmemS {
-  unsigned char b[NSTB][G][2][BBOX];
-  alignas(16) float bt[2][G][TCH];     // b' of the tile in each accumulator stage
-  uint8_t cnt[2][MQ];                  // per-tile selection counts of each half (pass 2)
-  uint64_t bfull[NSTB], bempty[NSTB], dfull[2], dempty[2], afull, done;
+  unsigned char b[NST][G][2][BBOX];
+  float stage[STG][EPI];          // staged survivors; [32][MQ] half-merge area after pass 1
+  alignas(16) float bt[2][G][TCH];  // b' of the tile, by tile parity
+  uint8_t cnt[2][2][2][MQ];       // pass 2, by tile parity: [half][above / equal][row]
+  float tau[MQ];
+  int nab[2][MQ];
+  uint64_t bfull[NST], bempty[NST], dfull, dempty, afull, done;
   uint32_t tmem;
 };
-
-HILS_DI unsigned long long make_key(float g, int c) {
-  return ((unsigned long long)float_key(g) << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)c);
-}
-// the float whose ordered image is the high word of `key` (-inf for key 0)
-HILS_DI float key_float(unsigned long long key) {
-  if (key == 0ull) return -INFINITY;
-  const uint32_t u = (uint32_t)(key >> 32);
-  return (u & 0x80000000u) ? __uint_as_float(u & 0x7FFFFFFFu) : __uint_as_float(~u);
-}
-
-// min-heap of K keys in column `col` of buf (pitch EPI)
-HILS_DI void sift_down(unsigned long long* buf, int col, int K, int i, unsigned long long key) {
-  while (true) {
-    const int l = 2 * i + 1;
-    if (l >= K) break;
-    int m = l;
-    if (l + 1 < K && buf[(l + 1) * EPI + col] < buf[l * EPI + col]) m = l + 1;
-    if (buf[m * EPI + col] >= key) break;
-    buf[i * EPI + col] = buf[m * EPI + col];
-    i = m;
-  }
-  buf[i * EPI + col] = key;
-}
-
-struct TopK {
-  int cnt = 0;
-  bool heap = false;
-  unsigned long long tau = 0ull;  // keys must exceed tau to enter
-  float tau_f = -INFINITY;        // cheap pre-filter: g >= tau_f
-};
-
-// fold buffered entries K..cnt-1 into the heap (building it once cnt >= K)
-HILS_DI void fold(unsigned long long* buf, int col, int K, TopK& t) {
-  if (!t.heap) {
-    if (t.cnt < K) return;
-    for (int x = K / 2 - 1; x >= 0; --x) sift_down(buf, col, K, x, buf[x * EPI + col]);
-    t.heap = true;
-  }
-  for (int e = K; e < t.cnt; ++e) {
-    const unsigned long long key = buf[e * EPI + col];
-    if (key > buf[col]) sift_down(buf, col, K, 0, key);
-  }
-  t.cnt = K;
-  t.tau = buf[col];
-  t.tau_f = key_float(t.tau);
-}
 
 HILS_DI void epi_barrier() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 // barrier among the epilogue warps that also ANDs a flag, so that all of them
@@ -116,42 +75,53 @@ HILS_DI bool epi_all(bool v) {
   return out != 0;
 }
 
-HILS_DI void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
-        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
+// insert x into the descending list a (x = -inf leaves it unchanged)
+template <int KT>
+HILS_DI void insert_desc(float (&a)[KT], float x) {
+#pragma unroll
+  for (int j = KT - 1; j > 0; --j) a[j] = fmaxf(fminf(a[j - 1], x), a[j]);
+  a[0] = fmaxf(a[0], x);
 }
 
+// v[j] for a runtime j in [0, 32), by a tree of selects (no local memory)
+HILS_DI uint32_t pick32(const uint32_t (&v)[32], int j) {
+  uint32_t a[16], c[8], d[4], e[2];
+#pragma unroll
+  for (int t = 0; t < 16; ++t) a[t] = (j & 16) ? v[t + 16] : v[t];
+#pragma unroll
+  for (int t = 0; t < 8; ++t) c[t] = (j & 8) ? a[t + 8] : a[t];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) d[t] = (j & 4) ? c[t + 4] : c[t];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) e[t] = (j & 2) ? d[t + 2] : d[t];
+  return (j & 1) ? e[1] : e[0];
+}
+
+template <int KT>
 __global__ void __launch_bounds__(THREADS, 1)
     score_topk_tc_kernel(Shape s, const __grid_constant__ CUtensorMap tmk, const __nv_bfloat16* __restrict__ q,
                          const float* __restrict__ b_sum, int32_t* __restrict__ idx, float* __restrict__ s_sel,
                          DevCtx ctx) {
   extern __shared__ unsigned char smem_raw[];
   SmemS& sm = *reinterpret_cast<SmemS*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned long long* buf = reinterpret_cast<unsigned long long*>(&sm + 1);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = blockIdx.y, b = blockIdx.z;
   const int i0 = blockIdx.x * MQ;
   const int K = s.K;
-  const int CAP = K + HALF;
   const int last = min(i0 + MQ, s.N) - 1;
   const int ncand_max = max(0, last / 64 - s.nw + 1);
   const int T = (ncand_max + TCH - 1) / TCH;  // tiles per pass
   const int NIT = 2 * T;
 
   if (tid == 0) {
-    for (int x = 0; x < NSTB; ++x) {
+    for (int x = 0; x < NST; ++x) {
       mbar_init(&sm.bfull[x], 1);
-      mbar_init(&sm.bempty[x], 1);
+      mbar_init(&sm.bempty[x], NMMA);
     }
-    for (int x = 0; x < 2; ++x) {
-      mbar_init(&sm.dfull[x], 1);
-      mbar_init(&sm.dempty[x], EPI / 32);
-    }
+    mbar_init(&sm.dfull, NMMA);
+    mbar_init(&sm.dempty, EPI / 32);
     mbar_init(&sm.afull, EPI / 32);
-    mbar_init(&sm.done, 1);
+    mbar_init(&sm.done, NMMA);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -163,41 +133,35 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem;
 
-  if (warp == 0) {
-    // ---------------------------------------------------------- producer ----
-    int last_round[NSTB];
-#pragma unroll
-    for (int x = 0; x < NSTB; ++x) last_round[x] = -1;
-    if (lane == 0 && NIT > 0) prefetch_tmap(&tmk);
-    bool ok = true;
-    for (int it = 0; it < NIT && ok; ++it) {
-      const int t = it % T, sb = it % NSTB, rnd = it / NSTB;
-      if (rnd > 0) ok = mbar_wait(&sm.bempty[sb], (rnd - 1) & 1, ctx);
-      if (!ok) break;
+  if (warp < NMMA) {
+    // ------------------------------------- MMA issue (+ TMA ring, warp 0) ---
+    const int h = warp;
+    int nprod = 0;  // items put into the ring (warp 0)
+    auto produce = [&](int it) {
+      const int t = it % T, sb = it % NST;
       if (lane == 0 && ctx.inject != 1) {
         mbar_arrive_expect_tx(&sm.bfull[sb], BSTAGE);
-        for (int h = 0; h < G; ++h) {
-          const int z = b * s.Hq + g * G + h;
-          tma_load_3d(sm.b[sb][h][0], &tmk, 0, t * TCH, z, &sm.bfull[sb]);
-          tma_load_3d(sm.b[sb][h][1], &tmk, 64, t * TCH, z, &sm.bfull[sb]);
+        for (int hh = 0; hh < G; ++hh) {
+          const int z = b * s.Hq + g * G + hh;
+          tma_load_3d(sm.b[sb][hh][0], &tmk, 0, t * TCH, z, &sm.bfull[sb]);
+          tma_load_3d(sm.b[sb][hh][1], &tmk, 64, t * TCH, z, &sm.bfull[sb]);
         }
-        last_round[sb] = rnd;
       }
+      nprod = it + 1;
+    };
+    if (warp == 0) {
+      if (lane == 0 && NIT > 0) prefetch_tmap(&tmk);
+      for (int it = 0; it < min(NST, NIT); ++it) produce(it);
       __syncwarp();
     }
-    if (lane == 0)
-      for (int x = 0; x < NSTB; ++x)
-        if (last_round[x] >= 0) mbar_wait(&sm.bfull[x], last_round[x] & 1, ctx);
-    __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------- MMA ------
     const uint32_t idesc = idesc_bf16_f32(MQ, TCH);
     bool ok = NIT == 0 || mbar_wait(&sm.afull, 0, ctx);
+    ok = __all_sync(0xffffffffu, ok);
     tc_fence_after();
     for (int it = 0; it < NIT && ok; ++it) {
-      const int sb = it % NSTB, sd = it % 2;
-      ok = mbar_wait(&sm.bfull[sb], (it / NSTB) & 1, ctx);
-      if (ok && it >= 2) ok = mbar_wait(&sm.dempty[sd], ((it / 2) - 1) & 1, ctx);
+      const int sb = it % NST;
+      ok = mbar_wait(&sm.bfull[sb], (it / NST) & 1, ctx);
+      if (ok && it > 0) ok = mbar_wait(&sm.dempty, (it - 1) & 1, ctx);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
@@ -205,18 +169,25 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_after();
       if (lane == 0) {
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t bdesc_addr = smem_u32(sm.b[sb][h][kk >> 2]) + (kk & 3) * 32;
-            mma_ts(tmem + DCOL + sd * 128 + h * 32, tmem + ACOL + h * 64 + kk * 8, sdesc_k_sw128(bdesc_addr),
-                   idesc, kk > 0 ? 1u : 0u);
-          }
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t bdesc_addr = smem_u32(sm.b[sb][h][kk >> 2]) + (kk & 3) * 32;
+          mma_ts(tmem + DCOL + h * 64, tmem + ACOL + h * 64 + kk * 8, sdesc_k_sw128(bdesc_addr), idesc,
+                 kk > 0 ? 1u : 0u);
         }
         tc_commit(&sm.bempty[sb]);
-        tc_commit(&sm.dfull[sd]);
+        tc_commit(&sm.dfull);
       }
       __syncwarp();
+      if (warp == 0 && it + NST < NIT) {
+        // the stage is free once every head's MMAs of this tile have completed
+        ok = __all_sync(0xffffffffu, mbar_wait(&sm.bempty[sb], (it / NST) & 1, ctx));
+        if (ok) produce(it + NST);
+        __syncwarp();
+      }
+    }
+    if (warp == 0 && lane == 0) {
+      // copies still in flight land before the CTA may exit
+      for (int x = 0; x < NST && x < nprod; ++x) mbar_wait(&sm.bfull[x], ((nprod - 1 - x) / NST) & 1, ctx);
     }
     // every MMA issued above has completed before the columns are released
     if (lane == 0) {
@@ -226,18 +197,19 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------------- epilogue ----
-    const int e = warp - 2;           // 0..7
-    const int hf = e >> 2;            // half of each tile: chunks [16 hf, 16 hf + 16)
+    const int e = warp - NMMA;        // 0..7
+    const int hf = e >> 2;            // half of each tile: chunks [32 hf, 32 hf + 32)
     const int qd = warp & 3;          // TMEM lane quadrant of this warp
     const int r = qd * 32 + lane;     // row = TMEM lane
-    const int col = hf * MQ + r;      // buffer column of this thread
+    const int et = e * 32 + lane;     // epilogue thread index
     const int i = i0 + r;
     const bool valid = i < s.N;
     const uint32_t lane_addr = tmem + ((uint32_t)(qd * 32) << 16);
+    float(*mrg)[MQ] = reinterpret_cast<float(*)[MQ]>(&sm.stage[0][0]);
     // A: this row's scoring query, heads 2 hf and 2 hf + 1 -> TMEM
-    for (int h = 2 * hf; h < 2 * hf + 2; ++h) {
+    for (int hh = 2 * hf; hh < 2 * hf + 2; ++hh) {
       const uint4* src =
-          reinterpret_cast<const uint4*>(q + (((long long)b * s.Hq + g * G + h) * s.N + (valid ? i : 0)) * D);
+          reinterpret_cast<const uint4*>(q + (((long long)b * s.Hq + g * G + hh) * s.N + (valid ? i : 0)) * D);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t w[32];
@@ -249,7 +221,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           w[4 * x + 2] = u.z;
           w[4 * x + 3] = u.w;
         }
-        tmem_st32(lane_addr + ACOL + h * 64 + half * 32, w);
+        tmem_st32(lane_addr + ACOL + hh * 64 + half * 32, w);
       }
     }
     tmem_wait_st();
@@ -259,111 +231,161 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     const int ncand = valid ? max(0, i / 64 - s.nw + 1) : 0;
     const float scale = s.scale;
-    TopK tk;
+    float top[KT];  // pass 1: this half's KT largest group scores, descending
+#pragma unroll
+    for (int j = 0; j < KT; ++j) top[j] = -INFINITY;
+    float tau = -INFINITY;  // pass 2: the row's K-th largest group score
+    int t_rem = 0;          // pass 2: scores equal to tau still to take
     int nsel = 0;
     const long long row_idx = (((long long)b * s.Hkv + g) * s.N + i) * K;
     bool ok = true;
 
     for (int it = 0; it < NIT; ++it) {
-      const int pass = it / T, t = it % T, sd = it % 2;
+      const int pass = it >= T ? 1 : 0, t = it - pass * T, par = it & 1;
       const int c0 = t * TCH + hf * HALF;  // first chunk of this thread's half
-      const bool landed = mbar_wait(&sm.dfull[sd], (it / 2) & 1, ctx);
+      // b' of the tile: thread et fetches head et / 64, chunk et % 64
+      const int bh = et >> 6, bj = et & 63, bc = t * TCH + bj;
+      const float bval = bc < s.C ? __ldg(b_sum + ((long long)b * s.Hq + g * G + bh) * s.C + bc) : 0.f;
+      const bool landed = mbar_wait(&sm.dfull, it & 1, ctx);
       if (!epi_all(landed)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      if (hf == 0) {
-        const int hh = r >> 5, jj = r & 31, cc = t * TCH + jj;
-        sm.bt[sd][hh][jj] = cc < s.C ? __ldg(b_sum + ((long long)b * s.Hq + g * G + hh) * s.C + cc) : 0.f;
-      }
+      sm.bt[par][bh][bj] = bval;
       epi_barrier();
-      uint32_t v[G][HALF];
-#pragma unroll
-      for (int h = 0; h < G; ++h) tmem_ld16(lane_addr + DCOL + sd * 128 + h * 32 + hf * HALF, v[h]);
-      tmem_wait_ld();
+      // group score of each chunk of this half: max over heads of v * scale + b'
       float gv[HALF];
+      constexpr int HW = KT <= 32 ? 2 : 1;  // heads loaded per TMEM wait
 #pragma unroll
-      for (int j = 0; j < HALF; ++j) gv[j] = -INFINITY;
+      for (int h0 = 0; h0 < G; h0 += HW) {
+        uint32_t v[HW][HALF];
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float4* bt4 = reinterpret_cast<const float4*>(&sm.bt[sd][h][hf * HALF]);
+        for (int u = 0; u < HW; ++u) tmem_ld32(lane_addr + DCOL + (h0 + u) * 64 + hf * HALF, v[u]);
+        tmem_wait_ld();
 #pragma unroll
-        for (int j4 = 0; j4 < HALF / 4; ++j4) {
-          const float4 bb = bt4[j4];
-          gv[4 * j4 + 0] = fmaxf(gv[4 * j4 + 0], __fmaf_rn(__uint_as_float(v[h][4 * j4 + 0]), scale, bb.x));
-          gv[4 * j4 + 1] = fmaxf(gv[4 * j4 + 1], __fmaf_rn(__uint_as_float(v[h][4 * j4 + 1]), scale, bb.y));
-          gv[4 * j4 + 2] = fmaxf(gv[4 * j4 + 2], __fmaf_rn(__uint_as_float(v[h][4 * j4 + 2]), scale, bb.z));
-          gv[4 * j4 + 3] = fmaxf(gv[4 * j4 + 3], __fmaf_rn(__uint_as_float(v[h][4 * j4 + 3]), scale, bb.w));
+        for (int u = 0; u < HW; ++u) {
+          const int hh = h0 + u;
+          const float4* bt4 = reinterpret_cast<const float4*>(&sm.bt[par][hh][hf * HALF]);
+#pragma unroll
+          for (int j4 = 0; j4 < HALF / 4; ++j4) {
+            const float4 bb = bt4[j4];
+            const float x0 = __fmaf_rn(__uint_as_float(v[u][4 * j4 + 0]), scale, bb.x);
+            const float x1 = __fmaf_rn(__uint_as_float(v[u][4 * j4 + 1]), scale, bb.y);
+            const float x2 = __fmaf_rn(__uint_as_float(v[u][4 * j4 + 2]), scale, bb.z);
+            const float x3 = __fmaf_rn(__uint_as_float(v[u][4 * j4 + 3]), scale, bb.w);
+            gv[4 * j4 + 0] = hh == 0 ? x0 : fmaxf(gv[4 * j4 + 0], x0);
+            gv[4 * j4 + 1] = hh == 0 ? x1 : fmaxf(gv[4 * j4 + 1], x1);
+            gv[4 * j4 + 2] = hh == 0 ? x2 : fmaxf(gv[4 * j4 + 2], x2);
+            gv[4 * j4 + 3] = hh == 0 ? x3 : fmaxf(gv[4 * j4 + 3], x3);
+          }
         }
       }
       if (pass == 0) {
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.dempty[sd]);
+        if (lane == 0) mbar_arrive(&sm.dempty);
+        // candidates above the current KT-th value, staged, then inserted
 #pragma unroll
-        for (int j = 0; j < HALF; ++j) {
-          const int c = c0 + j;
-          if (c < ncand && gv[j] >= tk.tau_f) {
-            const unsigned long long key = make_key(gv[j], c);
-            if (key > tk.tau) buf[(tk.cnt++) * EPI + col] = key;
+        for (int rd = 0; rd < HALF / STG; ++rd) {
+          const float thr = top[KT - 1];
+          int ns = 0;
+#pragma unroll
+          for (int j = 0; j < STG; ++j) {
+            const int jj = rd * STG + j;
+            if (c0 + jj < ncand && gv[jj] > thr) {
+              sm.stage[ns][et] = gv[jj];
+              ++ns;
+            }
           }
+          for (int k = 0; __any_sync(0xffffffffu, k < ns); ++k) insert_desc(top, k < ns ? sm.stage[k][et] : -INFINITY);
         }
-        if (__any_sync(0xffffffffu, tk.heap ? tk.cnt > K : tk.cnt >= K)) fold(buf, col, K, tk);
         if (t == T - 1) {
-          // merge the two halves of each row: half 1 hands its entries to half 0
-          fold(buf, col, K, tk);
-          if (hf == 1) sm.cnt[0][r] = (uint8_t)tk.cnt;
-          epi_barrier();
-          if (hf == 0) {
-            const int n1 = sm.cnt[0][r];
-            for (int x = 0; x < n1; ++x) {
-              const unsigned long long key = buf[x * EPI + MQ + r];
-              if (key > tk.tau) {
-                buf[(tk.cnt++) * EPI + col] = key;
-                if (tk.cnt == CAP || (!tk.heap && tk.cnt >= K)) fold(buf, col, K, tk);
+          // row threshold from the two halves' sorted lists a (half 0), b (half 1):
+          // tau = min_{j<K} max(a_j, b_{K-1-j})
+          epi_barrier();  // staging reads done before the area is reused
+          float tmin = INFINITY;
+#pragma unroll
+          for (int rd = 0; rd < (KT + 31) / 32; ++rd) {
+            if (hf == 1) {
+#pragma unroll
+              for (int x = 0; x < 32; ++x)
+                if (32 * rd + x < KT) mrg[x][r] = top[min(32 * rd + x, KT - 1)];
+            }
+            epi_barrier();
+            if (hf == 0) {
+#pragma unroll
+              for (int j = 0; j < KT; ++j) {
+                const int jb = K - 1 - j - 32 * rd;
+                if (j < K && jb >= 0 && jb < 32) tmin = fminf(tmin, fmaxf(top[j], mrg[jb][r]));
               }
             }
-            fold(buf, col, K, tk);
+            epi_barrier();
           }
-          epi_barrier();  // half 1's entries have been read; its column is free
-          if (hf == 0) buf[MQ + r] = tk.heap ? tk.tau - 1ull : 0ull;
+          if (hf == 0) sm.tau[r] = tmin;
           epi_barrier();
-          // pass 2 takes keys >= the row's K-th key (all candidates if fewer than K)
-          tk.tau = buf[MQ + r];
-          tk.tau_f = key_float(tk.tau);
+          tau = sm.tau[r];
+          int above = 0;
+#pragma unroll
+          for (int j = 0; j < KT; ++j) above += top[j] > tau ? 1 : 0;
+          sm.nab[hf][r] = above;
+          epi_barrier();
+          t_rem = max(0, K - (sm.nab[0][r] + sm.nab[1][r]));
         }
       } else {
-        uint32_t selmask = 0;
+        uint32_t gt = 0u, eq = 0u;
 #pragma unroll
         for (int j = 0; j < HALF; ++j) {
-          const int c = c0 + j;
-          if (c < ncand && gv[j] >= tk.tau_f && make_key(gv[j], c) > tk.tau) selmask |= 1u << j;
+          if (c0 + j < ncand) {
+            if (gv[j] > tau) gt |= 1u << j;
+            else if (gv[j] == tau) eq |= 1u << j;
+          }
         }
-        sm.cnt[hf][r] = (uint8_t)__popc(selmask);
+        sm.cnt[par][hf][0][r] = (uint8_t)__popc(gt);
+        sm.cnt[par][hf][1][r] = (uint8_t)__popc(eq);
         epi_barrier();
-        const int n0 = sm.cnt[0][r], n1 = sm.cnt[1][r];
-        epi_barrier();  // counts consumed before the next tile overwrites them
-        const int base = nsel + (hf ? n0 : 0);
-        if (selmask != 0) {
-#pragma unroll
-          for (int j = 0; j < HALF; ++j) {
-            if ((selmask >> j) & 1u) {
-              const int slot = base + __popc(selmask & ((1u << j) - 1u));
-              if (slot < K) {
-                idx[row_idx + slot] = c0 + j;
-#pragma unroll
-                for (int h = 0; h < G; ++h)
-                  s_sel[(((long long)b * s.Hq + g * G + h) * s.N + i) * K + slot] =
-                      __fmaf_rn(__uint_as_float(v[h][j]), scale, sm.bt[sd][h][hf * HALF + j]);
+        const int g0 = sm.cnt[par][0][0][r], e0 = sm.cnt[par][0][1][r];
+        const int g1 = sm.cnt[par][1][0][r], e1 = sm.cnt[par][1][1][r];
+        const int take0 = min(e0, t_rem), take1 = min(e1, t_rem - take0);
+        uint32_t sel = gt, em = eq;
+        for (int x = 0; x < (hf ? take1 : take0); ++x) {
+          sel |= em & (0u - em);
+          em &= em - 1u;
+        }
+        const int base = nsel + (hf ? g0 + take0 : 0);
+        nsel += g0 + take0 + g1 + take1;
+        t_rem -= take0 + take1;
+        if (__any_sync(0xffffffffu, sel != 0u)) {
+          // one pass per selected chunk of the busiest lane (usually one or two)
+          const int nmine = __popc(sel);
+          {
+            uint32_t rem = sel;
+            for (int k = 0; __any_sync(0xffffffffu, k < nmine); ++k) {
+              if (k < nmine) {
+                const int j = __ffs(rem) - 1;
+                rem &= rem - 1u;
+                if (base + k < K) idx[row_idx + base + k] = c0 + j;
               }
             }
           }
+#pragma unroll
+          for (int hh = 0; hh < G; ++hh) {
+            uint32_t v[HALF];
+            tmem_ld32(lane_addr + DCOL + hh * 64 + hf * HALF, v);
+            tmem_wait_ld();
+            float* dst = s_sel + (((long long)b * s.Hq + g * G + hh) * s.N + i) * K;
+            uint32_t rem = sel;
+            for (int k = 0; __any_sync(0xffffffffu, k < nmine); ++k) {
+              const int j = (__ffs(rem) - 1) & 31;  // 31 once this lane has no more (unused)
+              rem &= rem - 1u;
+              const float x = __uint_as_float(pick32(v, j));
+              if (k < nmine && base + k < K) dst[base + k] = __fmaf_rn(x, scale, sm.bt[par][hh][hf * HALF + j]);
+            }
+          }
         }
-        nsel += n0 + n1;
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.dempty[sd]);
+        if (lane == 0) mbar_arrive(&sm.dempty);
       }
     }
     if (valid && ok && hf == 0) {
@@ -372,7 +394,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int x = nsel; x < K; ++x) {
         idx[row_idx + x] = -1;
 #pragma unroll
-        for (int h = 0; h < G; ++h) s_sel[(((long long)b * s.Hq + g * G + h) * s.N + i) * K + x] = -INFINITY;
+        for (int hh = 0; hh < G; ++hh) s_sel[(((long long)b * s.Hq + g * G + hh) * s.N + i) * K + x] = -INFINITY;
       }
     }
     tc_fence_before();
@@ -384,7 +406,18 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-size_t smem_bytes(int K) { return sizeof(SmemS) + 1024 + (size_t)(K + HALF) * EPI * sizeof(unsigned long long); }
+constexpr size_t kSmemBytes = sizeof(SmemS) + 1024;
+
+template <int KT>
+cudaError_t launch_kt(const Shape& s, const CUtensorMap& tmk, const void* q, const float* b_sum, int32_t* idx,
+                      float* s_sel, cudaStream_t st, const DevCtx& ctx) {
+  cudaError_t e = ensure_dynamic_smem((const void*)score_topk_tc_kernel<KT>, (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid((s.N + MQ - 1) / MQ, s.Hkv, s.B);
+  score_topk_tc_kernel<KT><<<grid, THREADS, kSmemBytes, st>>>(s, tmk, (const __nv_bfloat16*)q, b_sum, idx, s_sel,
+                                                               ctx);
+  return cudaGetLastError();
+}
 
 }  // namespace
 
@@ -392,19 +425,16 @@ size_t score_tc_workspace(const Shape&) { return 0; }
 
 cudaError_t launch_score_topk_tc(const Shape& s, const void* q, const void* k_sum, const float* b_sum, int32_t* idx,
                                  float* s_sel, cudaStream_t st, const DevCtx& ctx) {
-  if (s.d != D || s.G != G || s.K > KMAX || s.S != 64) return cudaErrorNotSupported;
+  if (s.d != D || s.G != G || s.K > KMAX || s.K < 1 || s.S != 64) return cudaErrorNotSupported;
   CUtensorMap tmk;
   const uint64_t dims[3] = {(uint64_t)D, (uint64_t)(s.C > 0 ? s.C : 1), (uint64_t)s.B * s.Hq};
   const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)(s.C > 0 ? s.C : 1) * D * 2};
   const uint32_t box[3] = {64, TCH, 1};
   cudaError_t e = make_tmap_bf16(&tmk, k_sum, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
-  e = ensure_dynamic_smem((const void*)score_topk_tc_kernel, (int)smem_bytes(KMAX));
-  if (e != cudaSuccess) return e;
-  dim3 grid((s.N + MQ - 1) / MQ, s.Hkv, s.B);
-  score_topk_tc_kernel<<<grid, THREADS, smem_bytes(s.K), st>>>(s, tmk, (const __nv_bfloat16*)q, b_sum, idx, s_sel,
-                                                                ctx);
-  return cudaGetLastError();
+  if (s.K <= 16) return launch_kt<16>(s, tmk, q, b_sum, idx, s_sel, st, ctx);
+  if (s.K <= 32) return launch_kt<32>(s, tmk, q, b_sum, idx, s_sel, st, ctx);
+  return launch_kt<64>(s, tmk, q, b_sum, idx, s_sel, st, ctx);
 }
 
 }  // namespace hils
