@@ -346,7 +346,7 @@ def main():
     t_summ = mean_ms(ev["summaries"])
     peak_tf = pk["bf16_tflops_sustained"]
     ach = attn_f / (t_attn / 1e3) / 1e12
-    roofline = {"kernel": "attn_union_kernel (hils_attn_prefill)", "bound": "tensor", "achieved": round(ach, 2),
+    roofline = {"kernel": "attn_ring_kernel (hils_attn_prefill)", "bound": "tensor", "achieved": round(ach, 2),
                 "peak": peak_tf, "unit": "TFLOP/s", "frac": round(ach / peak_tf, 4),
                 "traffic": traffic_for("attn_union.cu", "attn_union_kernel", w.name),
                 "peak_source": f"{pk_kind} bf16_tflops_sustained",
