@@ -265,7 +265,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       // copies still in flight (only after a timeout) land before the CTA exits
-      if (!ok)
+      if (!ok && ctx.inject != 1)
         for (int j = max(0, k - NSI); j < k; ++j) mbar_wait(&sm.full[j % NSI], (j / NSI) & 1, ctx);
     }
     __syncwarp();

@@ -165,10 +165,10 @@ def test_end_to_end_tiny_sequences():
         _e2e(w, prefill_inputs(w))
 
 
-@pytest.mark.parametrize("stage", ["score", "qcal"])
+@pytest.mark.parametrize("stage", ["score", "qcal", "attn"])
 def test_prefill_wait_timeout_reports_status(stage):
-    """The tensor-core kernels that wait on tile copies (scoring, Q-Cal) report a
-    wait that runs out; the prefill attention kernel has no device waits."""
+    """The kernels that wait on tile copies (scoring, Q-Cal, attention) report a
+    wait that runs out, return, and leave the context usable."""
     w = WORKLOADS["prefill_512k_qcal"].scaled(name="to", N=2048, Hq=4, Hkv=1, needles_per_head=0)
     x = {n: t.to(DEV) for n, t in prefill_inputs(w).items() if isinstance(t, torch.Tensor)}
     qc = (x["h"], x["w_down"], x["w_up"])
@@ -178,8 +178,11 @@ def test_prefill_wait_timeout_reports_status(stage):
     try:
         H.hils_set_wait_budget(2_000_000)
         H.hils_set_fault_injection(1)
-        H.hils_score_topk(pre.cfg, x["q"], pre.k_sum, pre.b_sum, pre.idx, pre.s_sel, pre.ws,
-                          qcal=qc if stage == "qcal" else None)
+        if stage == "attn":
+            H.hils_attn_prefill(pre.cfg, x["q"], x["k"], x["v"], pre.idx, pre.s_sel, pre.out)
+        else:
+            H.hils_score_topk(pre.cfg, x["q"], pre.k_sum, pre.b_sum, pre.idx, pre.s_sel, pre.ws,
+                              qcal=qc if stage == "qcal" else None)
         with pytest.raises(H.HilsError) as ei:
             H.hils_sync_status()
         assert ei.value.status == H.HILS_ERR_TIMEOUT
