@@ -16,7 +16,7 @@
 // the union -- the block's selections below its first window chunk (a
 // bitmap, in chunk order), then every chunk from there to the last
 // position's chunk -- as separate K and V tiles (16 KB each, 128-byte
-// swizzle, rows past the sequence read as zero) through an 11-slot
+// swizzle, rows past the sequence read as zero) through a 13-slot
 // shared-memory ring filled by the tensor-memory accelerator.  15 consumer
 // warps, one per pair of positions (8 rows), each walk only their own chunks
 // (the two selection lists merged, then their window) in stream order.  A
@@ -57,7 +57,7 @@ constexpr int D = 128, S = 64, G = 4;
 constexpr int CW = 15;                  // consumer warps, one per position pair
 constexpr int BP = 2 * CW;              // positions per CTA
 constexpr int THREADS = (CW + 1) * 32;  // + producer warp
-constexpr int NSI = 11;                 // ring slots (16 KB each)
+constexpr int NSI = 13;                 // ring slots (16 KB each)
 constexpr uint32_t BOX = 64 * 128;      // [64 keys x 64 d] bf16, 128-byte rows
 constexpr uint32_t ITEM = 2 * BOX;      // the K or V tile of one chunk
 constexpr int KMAX = 64;
@@ -67,7 +67,6 @@ constexpr int MAXI = 2048;              // stream chunks per CTA (>= BP * KMAX +
 
 struct __align__(1024) SmemR {
   unsigned char slot[NSI][2][BOX];
-  __nv_bfloat16 stg[CW][8][D];  // output staging, one 8-row tile per warp
   uint32_t bits[MAXW];          // the block's selections below lo
   uint32_t pre[MAXW];           // exclusive prefix of popc(bits)
   uint32_t users[MAXI / 4];     // warps using each stream chunk (bytes)
@@ -439,28 +438,17 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
 
     // ---- epilogue: thread holds d = 16 mt + gq (acc[mt][0/1]) and 16 mt + gq + 8
-    // (acc[mt][2/3]) of its rows 2c4, 2c4+1; stage bf16 rows, then store 16-byte units
-    if (ok) {
+    // (acc[mt][2/3]) of its rows 2c4, 2c4+1 (position my_pos, heads my_h, my_h + 1);
+    // the 8 lanes of a quad column write 16 consecutive bytes per store
+    if (ok && my_valid) {
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
-        const float inv = my_valid ? 1.f / den[r] : 0.f;
-        __nv_bfloat16* row = sm.stg[warp][2 * c4 + r];
+        const float inv = 1.f / den[r];
+        __nv_bfloat16* o = out + (((long long)b * s.Hq + g * G + my_h + r) * s.N + my_pos) * D;
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt) {
-          row[16 * mt + gq] = __float2bfloat16_rn(acc[mt][r] * inv);
-          row[16 * mt + gq + 8] = __float2bfloat16_rn(acc[mt][2 + r] * inv);
-        }
-      }
-      __syncwarp();
-#pragma unroll
-      for (int x = 0; x < 4; ++x) {
-        const int unit = lane + 32 * x;  // 0..127
-        const int n = unit >> 4, w16 = unit & 15;
-        const int pos = p0 + (n >> 2);
-        if (pos < s.N) {
-          const uint4 val = reinterpret_cast<const uint4*>(sm.stg[warp][n])[w16];
-          __nv_bfloat16* o = out + (((long long)b * s.Hq + g * G + (n & 3)) * s.N + pos) * D;
-          reinterpret_cast<uint4*>(o)[w16] = val;
+          o[16 * mt + gq] = __float2bfloat16_rn(acc[mt][r] * inv);
+          o[16 * mt + gq + 8] = __float2bfloat16_rn(acc[mt][2 + r] * inv);
         }
       }
     }

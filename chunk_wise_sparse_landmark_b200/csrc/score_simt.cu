@@ -143,48 +143,76 @@ template <typename T, int D, int G>
 __global__ void __launch_bounds__(256) decode_scores(Shape s, const T* __restrict__ q, const T* __restrict__ k_sum,
                                                      const float* __restrict__ b_sum, float* __restrict__ s_all,
                                                      float* __restrict__ g_all, int ncand) {
-  // lane layout: 16 lanes per (chunk, head) row for d=128 (8 elements each)
+  // lane layout: LPR lanes per (chunk, head) row (16 for d = 128: 8 elements each)
   constexpr int LPR = D / 8 >= 32 ? 32 : D / 8;  // lanes per row
   constexpr int EPL = D / LPR;                    // elements per lane
+  constexpr int RPW = 32 / LPR;                   // rows per warp instruction
+  // row groups per iteration: all their loads are issued before any is used,
+  // so that each warp keeps U * G vectors per lane in flight
+  constexpr int U = (sizeof(T) == 2 && EPL == 8) ? (G >= 8 ? 2 : 16 / G) : 1;
   __shared__ float qs[G][D];
   const int g = blockIdx.y, b = blockIdx.z;
   for (int e = threadIdx.x; e < G * D; e += blockDim.x)
     qs[e / D][e % D] = to_f32(q[((long long)b * s.Hq + g * G + e / D) * D + e % D]);
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  constexpr int RPW = 32 / LPR;  // rows per warp instruction
   const int sub = lane / LPR, l = lane % LPR;
+  const long long hrow = ((long long)b * s.Hq + g * G) * s.C;  // row of head g*G, chunk 0
   // the loop bound is warp-uniform so that every lane reaches the shuffles
-  for (int cb = blockIdx.x * nwarps * RPW + warp * RPW; cb < ncand; cb += gridDim.x * nwarps * RPW) {
-    const int c = cb + sub < ncand ? cb + sub : cb;
-    const bool own = cb + sub < ncand;
-    float gmax = -INFINITY;
+  for (int cb = (blockIdx.x * nwarps + warp) * U * RPW; cb < ncand; cb += gridDim.x * nwarps * U * RPW) {
+    if constexpr (sizeof(T) == 2 && EPL == 8) {
+      uint4 u[U][G];
+      float bs[U][G];
 #pragma unroll
-    for (int hg = 0; hg < G; ++hg) {
-      const int h = g * G + hg;
-      const T* kp = k_sum + (((long long)b * s.Hq + h) * s.C + c) * D + l * EPL;
-      float acc = 0.f;
-      if constexpr (sizeof(T) == 2 && EPL == 8) {
-        // one 16-byte vector of bf16 per lane
-        const uint4 u = __ldg(reinterpret_cast<const uint4*>(kp));
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      for (int x = 0; x < U; ++x) {
+        const int c = min(cb + x * RPW + sub, ncand - 1);  // rows past ncand re-read the last one
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          const float2 f = bf16x2_to_f32x2(w[x]);
-          acc = fmaf(qs[hg][l * EPL + 2 * x], f.x, acc);
-          acc = fmaf(qs[hg][l * EPL + 2 * x + 1], f.y, acc);
+        for (int hg = 0; hg < G; ++hg) {
+          u[x][hg] = __ldg(reinterpret_cast<const uint4*>(k_sum + (hrow + (long long)hg * s.C + c) * D + l * EPL));
+          bs[x][hg] = __ldg(b_sum + hrow + (long long)hg * s.C + c);
         }
-      } else {
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) acc = fmaf(qs[hg][l * EPL + e], to_f32(kp[e]), acc);
       }
 #pragma unroll
-      for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      const float sv = acc * s.scale + b_sum[((long long)b * s.Hq + h) * s.C + c];
-      gmax = fmaxf(gmax, sv);
-      if (l == 0 && own) s_all[((long long)b * s.Hq + h) * s.C + c] = sv;
+      for (int x = 0; x < U; ++x) {
+        const int c = cb + x * RPW + sub;
+        const bool own = c < ncand;
+        float gmax = -INFINITY;
+#pragma unroll
+        for (int hg = 0; hg < G; ++hg) {
+          const uint32_t w[4] = {u[x][hg].x, u[x][hg].y, u[x][hg].z, u[x][hg].w};
+          float acc = 0.f;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = bf16x2_to_f32x2(w[e]);
+            acc = fmaf(qs[hg][l * EPL + 2 * e], f.x, acc);
+            acc = fmaf(qs[hg][l * EPL + 2 * e + 1], f.y, acc);
+          }
+#pragma unroll
+          for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+          const float sv = acc * s.scale + bs[x][hg];
+          gmax = fmaxf(gmax, sv);
+          if (l == 0 && own) s_all[hrow + (long long)hg * s.C + c] = sv;
+        }
+        if (l == 0 && own) g_all[((long long)b * s.Hkv + g) * s.C + c] = gmax;
+      }
+    } else {
+      const int c = cb + sub < ncand ? cb + sub : cb;
+      const bool own = cb + sub < ncand;
+      float gmax = -INFINITY;
+#pragma unroll
+      for (int hg = 0; hg < G; ++hg) {
+        const T* kp = k_sum + (hrow + (long long)hg * s.C + c) * D + l * EPL;
+        float acc = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) acc = fmaf(qs[hg][l * EPL + e], to_f32(kp[e]), acc);
+#pragma unroll
+        for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        const float sv = acc * s.scale + b_sum[hrow + (long long)hg * s.C + c];
+        gmax = fmaxf(gmax, sv);
+        if (l == 0 && own) s_all[hrow + (long long)hg * s.C + c] = sv;
+      }
+      if (l == 0 && own) g_all[((long long)b * s.Hkv + g) * s.C + c] = gmax;
     }
-    if (l == 0 && own) g_all[((long long)b * s.Hkv + g) * s.C + c] = gmax;
   }
 }
 
@@ -300,7 +328,8 @@ cudaError_t go_decode(const Shape& s, const void* q, const void* k_sum, const fl
   float* g_all = s_all + (size_t)s.B * s.Hq * s.C;
   if (ncand > 0) {
     constexpr int LPR = D / 8 >= 32 ? 32 : D / 8;
-    const int rows_per_block = 8 * (32 / LPR);
+    constexpr int U = (sizeof(T) == 2 && D / LPR == 8) ? (G >= 8 ? 2 : 16 / G) : 1;
+    const int rows_per_block = 8 * U * (32 / LPR);
     int gx = (ncand + rows_per_block - 1) / rows_per_block;
     const int sms = device_sm_count();
     const int want = (sms * 8 + s.B * s.Hkv - 1) / (s.B * s.Hkv);
