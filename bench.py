@@ -360,7 +360,8 @@ def main():
             "config": {"workload": w.name, "batch": w.B, "seq_len": w.N, "n_q_heads": w.Hq, "n_kv_heads": w.Hkv,
                        "head_dim": w.d, "chunk": w.S, "window": w.W, "top_k": w.K,
                        "qcal_rank": w.qcal_rank, "parallelism": f"replica x{ws}",
-                       "l2": "inputs larger than L2 (q 1.07 GB, k/v 268 MB each)"},
+                       "l2": "inputs larger than L2 (q %.2f GB, k/v %.0f MB each)" % (
+                           w.B * w.Hq * w.N * w.d * 2 / 1e9, w.B * w.Hkv * w.N * w.d * 2 / 1e6)},
             "roofline": roofline, "kernels": per_kernel, "clocks": clocks,
             "gpu_launches": (3 + (1 if w.d_model else 0)) * args.steps}
     if not args.no_e2e:

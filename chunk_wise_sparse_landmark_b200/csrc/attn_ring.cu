@@ -75,15 +75,19 @@ struct __align__(1024) SmemR {
   int nb;                       // selections below lo = stream chunks from the bitmap
 };
 
+// shared-memory fragment loads; the "memory" clobber keeps them ahead of the
+// barrier arrive that hands their slot back to the copy engine
 HILS_DI void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
+               : "r"(addr)
+               : "memory");
 }
 HILS_DI void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
+               : "r"(addr)
+               : "memory");
 }
 HILS_DI uint32_t movmatrix_t(uint32_t x) {
   uint32_t y;
