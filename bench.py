@@ -236,26 +236,29 @@ def device_time(stream, fn, steps, dist_on):
 
 
 def e2e_prefill(w, x, pre, stream, steps, dist_on):
-    """Through the public API with host buffers: H2D of the step's inputs from
-    pinned memory, the prefill, D2H of the output, all inside the timed region."""
-    names = ["q", "k", "v", "q_lmk"] + (["h", "w_down", "w_up"] if w.d_model else [])
-    host = {n: x[n].to("cpu").pin_memory() for n in names}
-    devb = {n: torch.empty_like(x[n]) for n in names}
+    """Through the C ABI with host buffers (hils_prefill_host): every step copies
+    the inputs from pinned host memory to the device, runs the prefill and copies
+    the output back; the library pipelines the transfers with the kernels by
+    (sequence, KV group)."""
+    names = ["q", "k", "v", "q_lmk"]
+    host = {n: x[n].to("cpu").contiguous().pin_memory() for n in names}
+    qc = tuple(x[n].to("cpu").contiguous().pin_memory() for n in ("h", "w_down", "w_up")) if w.d_model else None
     out_h = torch.empty(pre.out.shape, dtype=pre.out.dtype).pin_memory()
+    ws = H.alloc_workspace(H.workspace_bytes(pre.cfg, H.HILS_WS_PREFILL_HOST, w.qcal_rank), pre.out.device)
     h2d = sum(t.numel() * t.element_size() for t in host.values())
+    h2d += sum(t.numel() * t.element_size() for t in qc) if qc else 0
     d2h = out_h.numel() * out_h.element_size()
 
     def step():
-        for n in names:
-            devb[n].copy_(host[n], non_blocking=True)
-        qc = (devb["h"], devb["w_down"], devb["w_up"]) if w.d_model else None
-        pre.run(devb["q"], devb["k"], devb["v"], devb["q_lmk"], qcal=qc, stream=stream)
-        out_h.copy_(pre.out, non_blocking=True)
+        H.hils_prefill_host(pre.cfg, host["q"], host["k"], host["v"], host["q_lmk"], out_h, ws, qcal=qc,
+                            stream=stream)
 
     with torch.cuda.stream(stream):
         step()
-    torch.cuda.synchronize()
+    H.hils_sync_status(stream)
     ms = device_time(stream, step, steps, dist_on)
+    H.hils_sync_status(stream)
+    del ws
     return ms / steps, h2d, d2h
 
 

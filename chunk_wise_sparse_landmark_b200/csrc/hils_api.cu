@@ -113,6 +113,90 @@ hils_status_t make_shape(const hils_config_t* cfg, Shape* s, bool decode) {
 
 size_t esize(const Shape& s) { return s.dtype == HILS_F32 ? 4 : 2; }
 
+// ------------------------------------------------ host-memory prefill path ---
+size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Offsets, in the caller's workspace, of the device copies of the inputs and of
+// every intermediate tensor of hils_prefill_host.
+struct HostLayout {
+  size_t q, k, v, qlmk, ksum, bsum, idx, ssel, out, h, wd, wu, qt, total;
+};
+HostLayout host_layout(const Shape& s, int rank) {
+  HostLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += up256(bytes);
+    return o;
+  };
+  const size_t e = esize(s);
+  L.q = take((size_t)s.B * s.Hq * s.N * s.d * e);
+  L.k = take((size_t)s.B * s.Hkv * s.N * s.d * e);
+  L.v = take((size_t)s.B * s.Hkv * s.N * s.d * e);
+  L.qlmk = take((size_t)s.B * s.Hq * s.C * s.d * e);
+  L.ksum = take((size_t)s.B * s.Hq * s.C * s.d * e);
+  L.bsum = take((size_t)s.B * s.Hq * s.C * 4);
+  L.idx = take((size_t)s.B * s.Hkv * s.N * s.K * 4);
+  L.ssel = take((size_t)s.B * s.Hq * s.N * s.K * 4);
+  L.out = take((size_t)s.B * s.Hq * s.N * s.d * e);
+  if (rank > 0) {
+    const size_t dm = (size_t)s.Hq * s.d;  // the supported Q-Cal width
+    L.h = take((size_t)s.B * s.N * dm * e);
+    L.wd = take((size_t)rank * dm * e);
+    L.wu = take((size_t)s.Hq * s.d * rank * e);
+    L.qt = take((size_t)s.B * s.Hq * s.N * s.d * e);
+  }
+  L.total = off;
+  return L;
+}
+
+// Two copy streams (uploads, downloads) and a pool of events per device.  The
+// whole enqueue sequence of one call holds g_pipe_mu, so concurrent calls never
+// record an event that another call is about to wait on.
+struct Pipe {
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t* ev = nullptr;
+  int nev = 0;
+};
+Pipe g_pipe[64];
+std::mutex g_pipe_mu;
+
+hils_status_t get_pipe(int dev, int nev, Pipe** pp) {
+  Pipe& p = g_pipe[dev];
+  cudaError_t e;
+  if (!p.in) {
+    e = cudaStreamCreateWithFlags(&p.in, cudaStreamNonBlocking);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamCreate");
+  }
+  if (!p.out) {
+    e = cudaStreamCreateWithFlags(&p.out, cudaStreamNonBlocking);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamCreate");
+  }
+  if (p.nev < nev) {
+    cudaEvent_t* ev = new cudaEvent_t[nev];
+    for (int i = 0; i < p.nev; ++i) ev[i] = p.ev[i];
+    for (int i = p.nev; i < nev; ++i) {
+      e = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming);
+      if (e != cudaSuccess) {
+        for (int j = p.nev; j < i; ++j) cudaEventDestroy(ev[j]);
+        delete[] ev;
+        return cuda_fail(e, "cudaEventCreate");
+      }
+    }
+    delete[] p.ev;
+    p.ev = ev;
+    p.nev = nev;
+  }
+  *pp = &p;
+  return HILS_OK;
+}
+
+#define HILS_CK(expr, where)                                \
+  do {                                                      \
+    cudaError_t _e = (expr);                                \
+    if (_e != cudaSuccess) return cuda_fail(_e, where);     \
+  } while (0)
+
 }  // namespace
 }  // namespace hils
 
@@ -156,6 +240,8 @@ size_t hils_workspace_bytes(const hils_config_t* cfg, int32_t which, int32_t qca
       return decode_score_workspace(s);
     case HILS_WS_ATTN_DECODE:
       return decode_attn_workspace(s);
+    case HILS_WS_PREFILL_HOST:
+      return host_layout(s, qcal_rank > 0 ? qcal_rank : 0).total;
   }
   return (size_t)-1;
 }
@@ -218,6 +304,129 @@ hils_status_t hils_attn_prefill(const hils_config_t* cfg, const void* q, const v
       return fail(HILS_ERR_INVALID_ARG, "hils_attn_prefill: bf16 q, k, v must be 32-byte aligned");
     HILS_LAUNCH(launch_attn_prefill_tc(s, q, k, v, idx, s_sel, out, st, ctx), "attn_prefill_tc");
   }
+  return HILS_OK;
+}
+
+hils_status_t hils_prefill_host(const hils_config_t* cfg, const void* h_q, const void* h_k, const void* h_v,
+                                const void* h_q_lmk, const hils_qcal_t* qcal, void* h_out, void* workspace,
+                                size_t ws_bytes, void* stream) {
+  Shape s;
+  HILS_TRY(make_shape(cfg, &s, false));
+  if (!h_q || !h_k || !h_v || !h_q_lmk || !h_out) return fail(HILS_ERR_INVALID_ARG, "hils_prefill_host: NULL host pointer");
+  const int rank = qcal ? qcal->rank : 0;
+  if (qcal) {
+    if (!qcal->h || !qcal->w_down || !qcal->w_up) return fail(HILS_ERR_INVALID_ARG, "Q-Cal: NULL host pointer");
+    if (s.dtype != HILS_BF16) return fail(HILS_ERR_UNSUPPORTED, "Q-Cal needs bf16");
+    if (qcal->rank < 16 || qcal->rank > 128 || qcal->rank % 16 || qcal->d_model != s.Hq * s.d)
+      return fail(HILS_ERR_UNSUPPORTED, "hils_prefill_host: Q-Cal rank %d / d_model %d not supported (d_model must be Hq*d)",
+                  qcal->rank, qcal->d_model);
+  }
+  const size_t need = hils_workspace_bytes(cfg, HILS_WS_PREFILL_HOST, rank);
+  if (ws_bytes < need || !aligned16(workspace))
+    return fail(HILS_ERR_INVALID_ARG, "hils_prefill_host: workspace needs %zu bytes (got %zu)", need, ws_bytes);
+  DevCtx ctx;
+  HILS_TRY(dev_ctx(&ctx));
+  int dev = 0;
+  HILS_CK(cudaGetDevice(&dev), "cudaGetDevice");
+  const HostLayout L = host_layout(s, rank);
+  unsigned char* W = (unsigned char*)workspace;
+  unsigned char *dq = W + L.q, *dk = W + L.k, *dv = W + L.v, *dql = W + L.qlmk, *dks = W + L.ksum, *dout = W + L.out;
+  float* dbs = (float*)(W + L.bsum);
+  int32_t* didx = (int32_t*)(W + L.idx);
+  float* dss = (float*)(W + L.ssel);
+  const unsigned char *hq = (const unsigned char*)h_q, *hk = (const unsigned char*)h_k, *hv = (const unsigned char*)h_v,
+                      *hql = (const unsigned char*)h_q_lmk;
+  unsigned char* hout = (unsigned char*)h_out;
+  const size_t e = esize(s);
+  const int P = s.B * s.Hkv;  // pieces: (sequence, KV group)
+  const size_t nq = (size_t)s.G * s.N * s.d * e, nkv = (size_t)s.N * s.d * e, nql = (size_t)s.G * s.C * s.d * e;
+  Shape sub = s;  // one piece: one sequence, one KV group and its G query heads
+  sub.B = 1;
+  sub.Hq = s.G;
+  sub.Hkv = 1;
+  auto piece = [&](int p, size_t* oq, size_t* okv, size_t* oql, size_t* obs, size_t* oidx, size_t* oss) {
+    const size_t b = p / s.Hkv, g = p % s.Hkv, h0 = b * s.Hq + g * s.G, kv = b * s.Hkv + g;
+    *oq = h0 * s.N * s.d * e;
+    *okv = kv * s.N * s.d * e;
+    *oql = h0 * s.C * s.d * e;
+    *obs = h0 * s.C;
+    *oidx = kv * s.N * s.K;
+    *oss = h0 * s.N * s.K;
+  };
+  std::lock_guard<std::mutex> lk(g_pipe_mu);
+  Pipe* pp = nullptr;
+  HILS_TRY(get_pipe(dev, 2 * P + 3, &pp));
+  cudaStream_t st = (cudaStream_t)stream, ci = pp->in, co = pp->out;
+  cudaEvent_t ev_start = pp->ev[0], ev_all = pp->ev[1], ev_done = pp->ev[2];
+  cudaEvent_t* ev_in = pp->ev + 3;
+  cudaEvent_t* ev_att = pp->ev + 3 + P;
+  // the copy streams start after the work already on `stream` (which may still use the workspace)
+  HILS_CK(cudaEventRecord(ev_start, st), "cudaEventRecord");
+  HILS_CK(cudaStreamWaitEvent(ci, ev_start, 0), "cudaStreamWaitEvent");
+  HILS_CK(cudaStreamWaitEvent(co, ev_start, 0), "cudaStreamWaitEvent");
+  if (!qcal) {
+    for (int p = 0; p < P; ++p) {
+      size_t oq, okv, oql, obs, oidx, oss;
+      piece(p, &oq, &okv, &oql, &obs, &oidx, &oss);
+      HILS_CK(cudaMemcpyAsync(dk + okv, hk + okv, nkv, cudaMemcpyHostToDevice, ci), "upload k");
+      HILS_CK(cudaMemcpyAsync(dql + oql, hql + oql, nql, cudaMemcpyHostToDevice, ci), "upload q_lmk");
+      HILS_CK(cudaMemcpyAsync(dq + oq, hq + oq, nq, cudaMemcpyHostToDevice, ci), "upload q");
+      HILS_CK(cudaMemcpyAsync(dv + okv, hv + okv, nkv, cudaMemcpyHostToDevice, ci), "upload v");
+      HILS_CK(cudaEventRecord(ev_in[p], ci), "cudaEventRecord");
+    }
+    for (int p = 0; p < P; ++p) {
+      size_t oq, okv, oql, obs, oidx, oss;
+      piece(p, &oq, &okv, &oql, &obs, &oidx, &oss);
+      HILS_CK(cudaStreamWaitEvent(st, ev_in[p], 0), "cudaStreamWaitEvent");
+      HILS_LAUNCH(launch_summaries(sub, dk + okv, dql + oql, dks + oql, dbs + obs, st, ctx), "summaries");
+      if (s.dtype == HILS_F32) {
+        HILS_LAUNCH(launch_score_topk_simt(sub, dq + oq, dks + oql, dbs + obs, didx + oidx, dss + oss, st, ctx),
+                    "score_topk_simt");
+        HILS_LAUNCH(launch_attn_prefill_simt(sub, dq + oq, dk + okv, dv + okv, didx + oidx, dss + oss, dout + oq, st, ctx),
+                    "attn_prefill_simt");
+      } else {
+        HILS_LAUNCH(launch_score_topk_tc(sub, dq + oq, dks + oql, dbs + obs, didx + oidx, dss + oss, st, ctx),
+                    "score_topk_tc");
+        HILS_LAUNCH(launch_attn_prefill_tc(sub, dq + oq, dk + okv, dv + okv, didx + oidx, dss + oss, dout + oq, st, ctx),
+                    "attn_prefill_tc");
+      }
+      HILS_CK(cudaEventRecord(ev_att[p], st), "cudaEventRecord");
+      HILS_CK(cudaStreamWaitEvent(co, ev_att[p], 0), "cudaStreamWaitEvent");
+      HILS_CK(cudaMemcpyAsync(hout + oq, dout + oq, nq, cudaMemcpyDeviceToHost, co), "download out");
+    }
+  } else {
+    // Q-Cal: the low-rank term t = W_down h is shared by all heads, so the
+    // scoring runs on the whole problem once every input is on the device
+    const size_t all_q = (size_t)s.B * s.Hq * s.N * s.d * e, all_kv = (size_t)s.B * s.Hkv * s.N * s.d * e;
+    const size_t all_ql = (size_t)s.B * s.Hq * s.C * s.d * e, dm = (size_t)s.Hq * s.d;
+    HILS_CK(cudaMemcpyAsync(dk, hk, all_kv, cudaMemcpyHostToDevice, ci), "upload k");
+    HILS_CK(cudaMemcpyAsync(dql, hql, all_ql, cudaMemcpyHostToDevice, ci), "upload q_lmk");
+    HILS_CK(cudaMemcpyAsync(W + L.h, qcal->h, (size_t)s.B * s.N * dm * e, cudaMemcpyHostToDevice, ci), "upload h");
+    HILS_CK(cudaMemcpyAsync(W + L.wd, qcal->w_down, (size_t)rank * dm * e, cudaMemcpyHostToDevice, ci), "upload W_down");
+    HILS_CK(cudaMemcpyAsync(W + L.wu, qcal->w_up, (size_t)s.Hq * s.d * rank * e, cudaMemcpyHostToDevice, ci),
+            "upload W_up");
+    HILS_CK(cudaMemcpyAsync(dq, hq, all_q, cudaMemcpyHostToDevice, ci), "upload q");
+    HILS_CK(cudaEventRecord(ev_all, ci), "cudaEventRecord");
+    HILS_CK(cudaMemcpyAsync(dv, hv, all_kv, cudaMemcpyHostToDevice, ci), "upload v");
+    HILS_CK(cudaEventRecord(ev_in[0], ci), "cudaEventRecord");
+    HILS_CK(cudaStreamWaitEvent(st, ev_all, 0), "cudaStreamWaitEvent");
+    HILS_LAUNCH(launch_summaries(s, dk, dql, dks, dbs, st, ctx), "summaries");
+    HILS_LAUNCH(launch_qcal_tc(s, dq, W + L.h, W + L.wd, W + L.wu, rank, (int)dm, W + L.qt, st, ctx), "qcal");
+    HILS_LAUNCH(launch_score_topk_tc(s, W + L.qt, dks, dbs, didx, dss, st, ctx), "score_topk_tc");
+    HILS_CK(cudaStreamWaitEvent(st, ev_in[0], 0), "cudaStreamWaitEvent");
+    for (int p = 0; p < P; ++p) {
+      size_t oq, okv, oql, obs, oidx, oss;
+      piece(p, &oq, &okv, &oql, &obs, &oidx, &oss);
+      HILS_LAUNCH(launch_attn_prefill_tc(sub, dq + oq, dk + okv, dv + okv, didx + oidx, dss + oss, dout + oq, st, ctx),
+                  "attn_prefill_tc");
+      HILS_CK(cudaEventRecord(ev_att[p], st), "cudaEventRecord");
+      HILS_CK(cudaStreamWaitEvent(co, ev_att[p], 0), "cudaStreamWaitEvent");
+      HILS_CK(cudaMemcpyAsync(hout + oq, dout + oq, nq, cudaMemcpyDeviceToHost, co), "download out");
+    }
+  }
+  // `stream` passes the call once the last download has landed
+  HILS_CK(cudaEventRecord(ev_done, co), "cudaEventRecord");
+  HILS_CK(cudaStreamWaitEvent(st, ev_done, 0), "cudaStreamWaitEvent");
   return HILS_OK;
 }
 

@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(_PKG, "libhils.so")
 
 HILS_OK, HILS_ERR_INVALID_ARG, HILS_ERR_UNSUPPORTED, HILS_ERR_CUDA, HILS_ERR_TIMEOUT = range(5)
 HILS_F32, HILS_BF16 = 0, 1
-HILS_WS_SCORE_PREFILL, HILS_WS_SCORE_DECODE, HILS_WS_ATTN_DECODE = 0, 1, 2
+HILS_WS_SCORE_PREFILL, HILS_WS_SCORE_DECODE, HILS_WS_ATTN_DECODE, HILS_WS_PREFILL_HOST = 0, 1, 2, 3
 
 EXPORTS = (
     "hils_build_summaries",
@@ -25,6 +25,7 @@ EXPORTS = (
     "hils_attn_prefill",
     "hils_attn_decode",
     "hils_attn_decode_noalloc",
+    "hils_prefill_host",
     "hils_workspace_bytes",
     "hils_sync_status",
     "hils_last_error",
@@ -82,6 +83,7 @@ def load() -> ctypes.CDLL:
         lib.hils_attn_prefill.argtypes = [C, P, P, P, P, P, P, P]
         lib.hils_attn_decode.argtypes = [C, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         lib.hils_attn_decode_noalloc.argtypes = [C, P, P, P, P, P, P, P]
+        lib.hils_prefill_host.argtypes = [C, P, P, P, P, ctypes.POINTER(QCal), P, P, ctypes.c_size_t, P]
         lib.hils_workspace_bytes.argtypes = [C, ctypes.c_int32, ctypes.c_int32]
         lib.hils_workspace_bytes.restype = ctypes.c_size_t
         lib.hils_sync_status.argtypes = [P]
@@ -92,7 +94,7 @@ def load() -> ctypes.CDLL:
         lib.hils_set_fault_injection.restype = None
         lib.hils_version.restype = ctypes.c_char_p
         for n in ("hils_build_summaries", "hils_score_topk", "hils_attn_prefill", "hils_attn_decode",
-                  "hils_attn_decode_noalloc", "hils_sync_status"):
+                  "hils_attn_decode_noalloc", "hils_prefill_host", "hils_sync_status"):
             getattr(lib, n).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -151,6 +153,23 @@ def hils_score_topk(cfg: Config, q, k_sum, b_sum, idx, s_sel, workspace=None, de
 def hils_attn_prefill(cfg: Config, q, k, v, idx, s_sel, out, stream=None):
     _check(load().hils_attn_prefill(ctypes.byref(cfg), _p(q), _p(k), _p(v), _p(idx), _p(s_sel), _p(out),
                                     _stream(stream)))
+
+
+def _ph(t: torch.Tensor):
+    """Host tensor argument (contiguous CPU memory; pinned for overlapping copies)."""
+    assert not t.is_cuda and t.is_contiguous(), "host tensors must be contiguous CPU tensors"
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def hils_prefill_host(cfg: Config, q, k, v, q_lmk, out, workspace, qcal=None, stream=None):
+    """The prefill path from host memory (q, k, v, q_lmk, qcal tensors and out on the host)."""
+    qc = None
+    if qcal is not None:
+        h, w_down, w_up = qcal
+        qc = ctypes.byref(QCal(_ph(h).value, _ph(w_down).value, _ph(w_up).value, w_down.shape[0], w_down.shape[1]))
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(load().hils_prefill_host(ctypes.byref(cfg), _ph(q), _ph(k), _ph(v), _ph(q_lmk), qc, _ph(out),
+                                    _p(workspace), ws_bytes, _stream(stream)))
 
 
 def hils_attn_decode(cfg: Config, q, k_cache, v_cache, idx, s_sel, out, workspace, stream=None):

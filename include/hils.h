@@ -178,10 +178,48 @@ hils_status_t hils_attn_decode_noalloc(const hils_config_t* cfg, const void* q, 
                                        const void* v_cache, const int32_t* idx, const float* s_sel, void* out,
                                        void* stream);
 
-enum { HILS_WS_SCORE_PREFILL = 0, HILS_WS_SCORE_DECODE = 1, HILS_WS_ATTN_DECODE = 2 };
+/*
+ * The whole prefill path from host memory: copies the inputs to the device,
+ * builds the summaries, scores and selects (hils_build_summaries,
+ * hils_score_topk) and attends (hils_attn_prefill), then copies the output
+ * back.  The pages have no counterpart of this call; it packages the three
+ * steps above with their transfers so that a caller holding the inputs in
+ * host memory gets the output in host memory.
+ *
+ * Every (sequence, KV group) is an independent piece of the computation (its
+ * G query heads, its keys and values, its chunk lists).  Without Q-Cal the
+ * call uploads, computes and downloads piece by piece on two internal copy
+ * streams, so that the transfers of one piece overlap the kernels of others;
+ * with Q-Cal (whose low-rank term is shared by all heads) it uploads all
+ * inputs, scores the whole problem, then attends and downloads by piece.
+ * The results are those of the three device calls.
+ *   h_q [B, Hq, N, d], h_k / h_v [B, Hkv, N, d], h_q_lmk [B, Hq, C, d]
+ *   (dtype, host); h_out [B, Hq, N, d] (dtype, host, written).
+ *   qcal: NULL, or the Q-Cal tensors in HOST memory (layouts of hils_qcal_t).
+ *   Host buffers should be page-locked (cudaHostAlloc / pinned); pageable
+ *   memory works but the copies then do not overlap the kernels.
+ *   workspace: device memory of at least
+ *              hils_workspace_bytes(cfg, HILS_WS_PREFILL_HOST, rank) bytes
+ *              (16-byte aligned); it holds the device copies of the inputs and
+ *              all intermediate tensors, and belongs to the call until
+ *              `stream` passes it.
+ * The call enqueues all work and returns: h_out is complete once `stream`
+ * has passed the call (hils_sync_status(stream) waits and reports device
+ * errors).  The host buffers must stay valid and unchanged until then.  The
+ * call waits on and records events of its internal streams, so it must not be
+ * captured into a CUDA graph.
+ */
+hils_status_t hils_prefill_host(const hils_config_t* cfg, const void* h_q, const void* h_k, const void* h_v,
+                                const void* h_q_lmk, const hils_qcal_t* qcal, void* h_out, void* workspace,
+                                size_t ws_bytes, void* stream);
+
+enum { HILS_WS_SCORE_PREFILL = 0, HILS_WS_SCORE_DECODE = 1, HILS_WS_ATTN_DECODE = 2, HILS_WS_PREFILL_HOST = 3 };
 
 /* Bytes of workspace the call `which` needs for this configuration (0 if none);
- * qcal_rank is the Q-Cal rank for HILS_WS_SCORE_PREFILL (0 = no Q-Cal).
+ * qcal_rank is the Q-Cal rank for HILS_WS_SCORE_PREFILL and
+ * HILS_WS_PREFILL_HOST (0 = no Q-Cal).  With Q-Cal, hils_prefill_host
+ * supports d_model = Hq * d only (so that this size is known from cfg) and
+ * returns HILS_ERR_UNSUPPORTED for any other width.
  * Returns (size_t)-1 for an invalid configuration. */
 size_t hils_workspace_bytes(const hils_config_t* cfg, int32_t which, int32_t qcal_rank);
 

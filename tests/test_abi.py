@@ -71,3 +71,20 @@ def test_workspace_sizes():
     ws = H.workspace_bytes(cfg, H.HILS_WS_SCORE_DECODE)
     assert ws == (16 * 32 * 8192 + 16 * 8 * 8192) * 4
     assert H.workspace_bytes(cfg, H.HILS_WS_ATTN_DECODE) > 0
+
+
+def test_prefill_host_workspace_and_host_checks():
+    """Workspace size of the host-memory prefill and its argument checks (no GPU needed)."""
+    lib = H.load()
+    B, N, Hq, Hkv, d, S, K = 1, 512, 4, 1, 64, 32, 4
+    cfg = H.make_config(B, N, Hq, Hkv, d, S, 64, K, "f32")
+    up = lambda n: (n + 255) // 256 * 256
+    C = N // S
+    want = (up(B * Hq * N * d * 4) + 2 * up(B * Hkv * N * d * 4) + 2 * up(B * Hq * C * d * 4) + up(B * Hq * C * 4)
+            + up(B * Hkv * N * K * 4) + up(B * Hq * N * K * 4) + up(B * Hq * N * d * 4))
+    assert lib.hils_workspace_bytes(ctypes.byref(cfg), H.HILS_WS_PREFILL_HOST, 0) == want
+    p = ctypes.c_void_p(0x1000)
+    st = lib.hils_prefill_host(ctypes.byref(cfg), None, p, p, p, None, p, p, want, None)
+    assert st == H.HILS_ERR_INVALID_ARG
+    st = lib.hils_prefill_host(ctypes.byref(cfg), p, p, p, p, None, p, p, want - 1, None)
+    assert st == H.HILS_ERR_INVALID_ARG and b"workspace" in lib.hils_last_error()
