@@ -5,27 +5,28 @@
 // outputs are weighted by exp(s^_{i,c}) / Z^_i and the chunk-aligned window by
 // Z_swa / Z^_i, Z^_i = sum_c exp(s^_{i,c}) + Z_swa.  The section's hardware
 // paragraph groups adjacent queries and attends the union of their chunks;
-// here a CTA groups 30 adjacent positions of one GQA group (120 query-head
+// here a CTA groups 14 adjacent positions of one GQA group (56 query-head
 // rows) and streams the union of their chunks once.
 //
 // Why this shape.  Moving 64-key chunk tiles from L2 to the SMs is what
 // bounds this operation.  Even when positions pick their top-K chunks
-// independently, 30 positions choosing K of n candidates cover only
-// n (1 - (1 - K/n)^30) distinct chunks (about 630 instead of 960 for K = 32,
-// n = 1024), and they share their window chunks.  One producer warp streams
-// the union -- the block's selections below its first window chunk (a
-// bitmap, in chunk order), then every chunk from there to the last
-// position's chunk -- as separate K and V tiles (16 KB each, 128-byte
-// swizzle, rows past the sequence read as zero) through a 13-slot
-// shared-memory ring filled by the tensor-memory accelerator.  15 consumer
+// independently, P positions choosing K of n candidates cover only
+// n (1 - (1 - K/n)^P) distinct chunks, and they share their window chunks.
+// One producer warp streams the union -- the block's selections below its
+// first window chunk (a bitmap, in chunk order), then every chunk from there
+// to the last position's chunk -- as separate K and V tiles (16 KB each,
+// 128-byte swizzle, rows past the sequence read as zero) through a 6-slot
+// shared-memory ring filled by the tensor-memory accelerator.  7 consumer
 // warps, one per pair of positions (8 rows), each walk only their own chunks
 // (the two selection lists merged, then their window) in stream order.  A
 // slot is released by the warps that use its tile: the producer knows each
 // tile's user count (taken from the walks before streaming starts) and
 // arrives for the other warps itself, so a slot is never held by warps that
-// skip it.  16 warps per SM (512 threads, 128 registers each) keep the
-// tensor pipe and the copy engine busy while single warps wait.  A block may
-// straddle two chunks, so each warp keeps its own window range.
+// skip it.  Two such CTAs share an SM (256 threads, 128 registers each, about
+// 100 KB of shared memory): measured on B200, two independent rings per SM
+// beat one CTA of 15 consumer warps with a 13-slot ring (97.5 vs 101.0 ms at
+// 128K), because one stream's stalls no longer idle the whole SM.  A block
+// may straddle two chunks, so each warp keeps its own window range.
 //
 // Ring protocol.  Item k (K or V tile of stream chunk k / 2) lives in slot
 // k % NSI; its round k / NSI is published in round_[slot] once the slot's
@@ -54,10 +55,10 @@ namespace hils {
 namespace {
 
 constexpr int D = 128, S = 64, G = 4;
-constexpr int CW = 15;                  // consumer warps, one per position pair
+constexpr int CW = 7;                   // consumer warps, one per position pair
 constexpr int BP = 2 * CW;              // positions per CTA
 constexpr int THREADS = (CW + 1) * 32;  // + producer warp
-constexpr int NSI = 13;                 // ring slots (16 KB each)
+constexpr int NSI = 6;                  // ring slots (16 KB each)
 constexpr uint32_t BOX = 64 * 128;      // [64 keys x 64 d] bf16, 128-byte rows
 constexpr uint32_t ITEM = 2 * BOX;      // the K or V tile of one chunk
 constexpr int KMAX = 64;
@@ -110,7 +111,7 @@ struct Walk {
   int slot0 = 0, slot1 = 0;  // positions in the two lists (s^ lookup)
 };
 
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(THREADS, 2)
     attn_ring_kernel(Shape s, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                      const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ idx,
                      const float* __restrict__ s_sel, __nv_bfloat16* __restrict__ out, DevCtx ctx) {
