@@ -215,6 +215,20 @@ def mean_ms(pairs):
     return sum(a.elapsed_time(b) for a, b in pairs) / max(1, len(pairs))
 
 
+def max_over_ranks(ms, dist_on, device="cuda"):
+    """The slowest rank's time: every rank contributes its own and gets the max."""
+    if not dist_on:
+        return ms
+    t = torch.tensor([float(ms)], device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank, world_size, ms):
+    """Units all ranks processed per second, over the max-over-ranks time (weak scaling)."""
+    return units_per_rank * world_size / (ms / 1e3)
+
+
 def device_time(stream, fn, steps, dist_on):
     """Barrier + sync, K steps between CUDA events, sync; max over ranks (ms)."""
     if dist_on:
@@ -227,12 +241,7 @@ def device_time(stream, fn, steps, dist_on):
             fn()
     b.record(stream)
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b)
-    if dist_on:
-        t = torch.tensor([ms], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-    return ms
+    return max_over_ranks(a.elapsed_time(b), dist_on)
 
 
 def e2e_prefill(w, x, pre, stream, steps, dist_on):
@@ -342,7 +351,7 @@ def main():
     clocks = clk.summary()
     ms_step = ms_total / args.steps
     tokens = w.B * w.N * ws
-    value = tokens / (ms_step / 1e3)
+    value = whole_job_rate(w.B * w.N, ws, ms_step)
     score_f, attn_f = prefill_flops(w)
     t_attn = mean_ms(ev["attn_prefill"])
     t_score = mean_ms(ev["score_topk"])
@@ -360,11 +369,7 @@ def main():
     line = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": w.name, "batch": w.B, "seq_len": w.N, "n_q_heads": w.Hq, "n_kv_heads": w.Hkv,
-                       "head_dim": w.d, "chunk": w.S, "window": w.W, "top_k": w.K,
-                       "qcal_rank": w.qcal_rank, "parallelism": f"replica x{ws}",
-                       "l2": "inputs larger than L2 (q %.2f GB, k/v %.0f MB each)" % (
-                           w.B * w.Hq * w.N * w.d * 2 / 1e9, w.B * w.Hkv * w.N * w.d * 2 / 1e6)},
+            "config": run_config(w, ws),
             "roofline": roofline, "kernels": per_kernel, "clocks": clocks,
             "gpu_launches": (3 + (1 if w.d_model else 0)) * args.steps}
     if not args.no_e2e:
@@ -384,7 +389,7 @@ def main():
         t_sc = mean_ms(dev_ev["score_topk"])
         hbm = pk["hbm_gbs"]
         line["decode"] = {
-            "workload": wd.name, "value": round(wd.B * ws / (d_ms / 1e3), 1), "unit": "seqs/s",
+            "workload": wd.name, "value": round(whole_job_rate(wd.B, ws, d_ms), 1), "unit": "seqs/s",
             "ms_per_step": round(d_ms, 4), "score_topk_ms": round(t_sc, 4), "attn_decode_ms": round(t_att, 4),
             "roofline": {"kernel": "attn_decode_partial (hils_attn_decode, KV gather)", "bound": "hbm",
                          "achieved": round(gb / (t_att / 1e3) / 1e9, 1), "peak": hbm, "unit": "GB/s",
@@ -412,6 +417,15 @@ def main():
         torch.distributed.destroy_process_group()
 
 
+def run_config(w, ws):
+    """The `config` object of both arms' JSON lines."""
+    return {"workload": w.name, "batch": w.B, "seq_len": w.N, "n_q_heads": w.Hq, "n_kv_heads": w.Hkv,
+            "head_dim": w.d, "chunk": w.S, "window": w.W, "top_k": w.K, "qcal_rank": w.qcal_rank,
+            "parallelism": f"replica x{ws}",
+            "l2": "inputs larger than L2 (q %.2f GB, k/v %.0f MB each)" % (
+                w.B * w.Hq * w.N * w.d * 2 / 1e9, w.B * w.Hkv * w.N * w.d * 2 / 1e6)}
+
+
 def reference_arm(args, ws, rank):
     """The oracle as the reference implementation, on the host cores."""
     if rank != 0:
@@ -424,10 +438,10 @@ def reference_arm(args, ws, rank):
         if it >= args.warmup:
             vals.append(v)
     v = statistics.mean(vals)
-    line = {"impl": "reference", "metric": METRIC, "value": round(v, 2), "unit": "tokens/s", "n_gpus": 1,
+    line = {"impl": "reference", "metric": METRIC, "value": round(v, 2), "unit": "tokens/s", "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * 8 / v, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "batch": w.B, "seq_len": w.N, "parallelism": "host cores"},
+            "config": run_config(w, ws),
             "cpu_baseline": {"value": round(v, 2), "unit": "tokens/s", "kind": "oracle", "cores": os.cpu_count(),
                              "sample": f"8 random positions of {w.name} per step, all heads"},
             "e2e": {"value": round(v, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
