@@ -28,11 +28,18 @@
 // 128K), because one stream's stalls no longer idle the whole SM.  A block
 // may straddle two chunks, so each warp keeps its own window range.
 //
-// Ring protocol.  Item k (K or V tile of stream chunk k / 2) lives in slot
-// k % NSI; its round k / NSI is published in round_[slot] once the slot's
-// previous round has been released, and only then does a consumer wait on
-// the slot's full barrier with that round's parity (a consumer may run many
-// items ahead of the producer, so the parity alone would be ambiguous).
+// Ring protocol.  The items are the chunks' K and V tiles in stream order,
+// except that chunk r's V tile follows chunk r + DV's K tile: it is needed
+// only after the chunk's S^T and softmax, and holding it in a slot meanwhile
+// costs ring capacity (measured: 96.2 -> 90.0 ms at 128K for DV = 1).  Each
+// consumer then meets at most DV of its items out of stream order, which is
+// deadlock-free while NSI > DV: the producer issues in stream order, and an
+// item's slot is only reused after every earlier item in that slot was
+// released by its users.  Item k lives in slot k % NSI; its round k / NSI is
+// published in round_[slot] once the slot's previous round has been
+// released, and only then does a consumer wait on the slot's full barrier
+// with that round's parity (a consumer may run many items ahead of the
+// producer, so the parity alone would be ambiguous).
 //
 //   S^T (64 keys x 8 rows)   = K_c (keys x d)  . Q^T (d x rows)
 //   O^T (128 d x 8 rows)    += V_c^T (d x keys) . P^T (keys x rows)
@@ -102,6 +109,13 @@ HILS_DI void mbar_arrive_cnt(uint64_t* bar, uint32_t cnt) {
 }
 // byte address of 16-byte unit `unit` (0..7) of row `row` in a 128-byte-swizzled box
 HILS_DI uint32_t swz(uint32_t box, int row, int unit) { return box + row * 128 + ((unit ^ (row & 7)) << 4); }
+
+// Ring item numbers of stream chunk r's K and V tiles (n chunks): K_0 .. K_{DV-1},
+// then K_{r+DV}, V_r alternating, then the last DV V tiles.
+constexpr int DV = 1;
+static_assert(NSI > DV, "the delayed V tiles need more slots than the delay");
+HILS_DI int item_k(int r) { return r < DV ? r : 2 * r - DV; }
+HILS_DI int item_v(int r, int n) { return r <= n - 1 - DV ? DV + 2 * r + 1 : n + r; }
 
 // A warp's chunks in stream order: the merged selection lists, then its window.
 struct Walk {
@@ -242,32 +256,50 @@ __global__ void __launch_bounds__(THREADS, 2)
       int k = 0;  // items issued
       int w = 0;
       uint32_t m = nwords > 0 ? sm.bits[0] : 0u;
+      auto chunk_at = [&](int r) -> int {  // stream chunks, taken in order
+        if (r >= nb) return lo + (r - nb);
+        while (m == 0u) m = sm.bits[++w];
+        const int c = 32 * w + __ffs(m) - 1;
+        m &= m - 1u;
+        return c;
+      };
+      auto users_at = [&](int r) -> int { return (int)((sm.users[r >> 2] >> (8 * (r & 3))) & 0xFFu); };
+      auto put = [&](bool is_v, int c, int users) {
+        const int x = k % NSI, mr = k / NSI;
+        if (mr > 0) ok = mbar_wait(&sm.empty[x], (mr - 1) & 1, ctx);
+        if (!ok) return;
+        *reinterpret_cast<volatile int*>(&sm.round_[x]) = mr;
+        if (ctx.inject != 1) {
+          const CUtensorMap* tm = is_v ? &tmv : &tmk;
+          mbar_arrive_expect_tx(&sm.full[x], ITEM);
+          tma_load_3d(sm.slot[x][0], tm, 0, c * S, bg, &sm.full[x]);
+          tma_load_3d(sm.slot[x][1], tm, 64, c * S, bg, &sm.full[x]);
+        }
+        // the warps that do not use this tile are counted as done with it
+        if (users < CW) mbar_arrive_cnt(&sm.empty[x], (uint32_t)(CW - users));
+        ++k;
+      };
+      // the last DV + 1 chunks (pc[DV] = the newest), a shift register with
+      // static indices so that it stays in registers
+      int pc[DV + 1], pu[DV + 1];
+#pragma unroll
+      for (int j = 0; j <= DV; ++j) pc[j] = pu[j] = 0;
       for (int r = 0; r < nchunks && ok; ++r) {
-        int c;
-        if (r < nb) {
-          while (m == 0u) m = sm.bits[++w];
-          c = 32 * w + __ffs(m) - 1;
-          m &= m - 1u;
-        } else {
-          c = lo + (r - nb);
+        const int c = chunk_at(r), u = users_at(r);
+        put(false, c, u);
+#pragma unroll
+        for (int j = 0; j < DV; ++j) {
+          pc[j] = pc[j + 1];
+          pu[j] = pu[j + 1];
         }
-        const int users = (int)((sm.users[r >> 2] >> (8 * (r & 3))) & 0xFFu);
-        for (int kv = 0; kv < 2 && ok; ++kv) {
-          const int x = k % NSI, mr = k / NSI;
-          if (mr > 0) ok = mbar_wait(&sm.empty[x], (mr - 1) & 1, ctx);
-          if (!ok) break;
-          *reinterpret_cast<volatile int*>(&sm.round_[x]) = mr;
-          if (ctx.inject != 1) {
-            const CUtensorMap* tm = kv ? &tmv : &tmk;
-            mbar_arrive_expect_tx(&sm.full[x], ITEM);
-            tma_load_3d(sm.slot[x][0], tm, 0, c * S, bg, &sm.full[x]);
-            tma_load_3d(sm.slot[x][1], tm, 64, c * S, bg, &sm.full[x]);
-          }
-          // the warps that do not use this tile are counted as done with it
-          if (users < CW) mbar_arrive_cnt(&sm.empty[x], (uint32_t)(CW - users));
-          ++k;
-        }
+        pc[DV] = c;
+        pu[DV] = u;
+        if (ok && r >= DV) put(true, pc[0], pu[0]);  // V tile of chunk r - DV
       }
+      // V tiles of the last DV chunks (chunk n - 1 - DV + j sits at pc[j])
+#pragma unroll
+      for (int j = 1; j <= DV; ++j)
+        if (ok && nchunks - 1 - DV + j >= 0) put(true, pc[j], pu[j]);
       // copies still in flight (only after a timeout) land before the CTA exits
       if (!ok && ctx.inject != 1)
         for (int j = max(0, k - NSI); j < k; ++j) mbar_wait(&sm.full[j % NSI], (j / NSI) & 1, ctx);
@@ -339,7 +371,8 @@ __global__ void __launch_bounds__(THREADS, 2)
         a2[0] = __ldg(ss0 + slot_me) * kLog2e;
         a2[1] = __ldg(ss0 + sstride + slot_me) * kLog2e;
       }
-      const int kit = 2 * rank(c);
+      const int rk = rank(c);
+      const int kit = item_k(rk), vit = item_v(rk, nchunks);
       // ---- K tile: S^T = K_c Q^T
       if (!acquire(kit)) {
         ok = false;
@@ -420,11 +453,11 @@ __global__ void __launch_bounds__(THREADS, 2)
         }
       }
       // ---- V tile: O^T += V^T P^T, 8 m-tiles (16 d) x 4 k-steps (16 keys)
-      if (!acquire(kit + 1)) {
+      if (!acquire(vit)) {
         ok = false;
         break;
       }
-      const uint32_t vb = smem_u32(sm.slot[(kit + 1) % NSI][0]);
+      const uint32_t vb = smem_u32(sm.slot[vit % NSI][0]);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
         const uint32_t b0 = movmatrix_t(pack_bf16x2(sc[kk][0], sc[kk][1]));
@@ -439,7 +472,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       }
       __syncwarp();
       fence_proxy_async_shared();
-      if (lane == 0) mbar_arrive(&sm.empty[(kit + 1) % NSI]);
+      if (lane == 0) mbar_arrive(&sm.empty[vit % NSI]);
     }
 
     // ---- epilogue: thread holds d = 16 mt + gq (acc[mt][0/1]) and 16 mt + gq + 8
