@@ -243,54 +243,24 @@ __global__ void __launch_bounds__(kSelThreads) decode_select(Shape s, const floa
   } else {
     // MSB-first radix select of the K-th largest key
     unsigned prefix = 0, need = K;
-    const int lane = tid & 31;
     for (int shift = 24; shift >= 0; shift -= 8) {
       for (int x = tid; x < 256; x += kSelThreads) hist[x] = 0;
       __syncthreads();
       const unsigned hi_mask = shift == 24 ? 0u : (0xffffffffu << (shift + 8));
-      // the loop bound is warp-uniform: every lane reaches the match
-      for (int c0 = tid - lane; c0 < ncand; c0 += kSelThreads) {
-        const int c = c0 + lane;
-        const unsigned key = c < ncand ? float_key(gr[c]) : 0u;
-        const bool in = c < ncand && (key & hi_mask) == (prefix & hi_mask);
-        // one atomic per distinct bin and warp (the leading digits cluster)
-        const unsigned bin = in ? (key >> shift) & 255u : 256u + lane;
-        const unsigned peers = __match_any_sync(0xffffffffu, bin);
-        if (in && (__ffs(peers) - 1) == lane) atomicAdd(&hist[bin], (unsigned)__popc(peers));
+      for (int c = tid; c < ncand; c += kSelThreads) {
+        const unsigned key = float_key(gr[c]);
+        if ((key & hi_mask) == (prefix & hi_mask)) atomicAdd(&hist[(key >> shift) & 255u], 1u);
       }
       __syncthreads();
-      if (tid < 32) {
-        // digit of the need-th largest key: lane l holds bins 8l .. 8l+7
-        unsigned h8[8], own = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          h8[j] = hist[8 * lane + j];
-          own += h8[j];
+      if (tid == 0) {
+        unsigned acc = 0;
+        int digit = 255;
+        for (; digit > 0; --digit) {
+          if (acc + hist[digit] >= need) break;
+          acc += hist[digit];
         }
-        unsigned suf = own;  // keys in bins >= 8 lane
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const unsigned t = __shfl_down_sync(0xffffffffu, suf, o);
-          if (lane + o < 32) suf += t;
-        }
-        const unsigned above = suf - own;  // keys in bins >= 8 (lane + 1)
-        int digit = -1;
-        unsigned acc = above;
-        if (above < need && suf >= need) {
-#pragma unroll
-          for (int j = 7; j >= 0; --j) {
-            if (digit < 0 && acc + h8[j] >= need) digit = j;
-            else if (digit < 0) acc += h8[j];
-          }
-        }
-        const unsigned who = __ballot_sync(0xffffffffu, digit >= 0);
-        const int src = __ffs(who) - 1;
-        const int dg = __shfl_sync(0xffffffffu, 8 * lane + digit, src);
-        const unsigned ac = __shfl_sync(0xffffffffu, acc, src);
-        if (lane == 0) {
-          prefix_sh = prefix | ((unsigned)dg << shift);
-          need_sh = need - ac;
-        }
+        prefix_sh = prefix | ((unsigned)digit << shift);
+        need_sh = need - acc;
       }
       __syncthreads();
       prefix = prefix_sh;
