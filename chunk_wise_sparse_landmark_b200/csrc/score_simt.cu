@@ -241,32 +241,93 @@ __global__ void __launch_bounds__(kSelThreads) decode_select(Shape s, const floa
     for (int c = tid; c < ncand; c += kSelThreads) sel[c] = c;
     if (tid == 0) nsel_sh = ncand;
   } else {
-    // MSB-first radix select of the K-th largest key
-    unsigned prefix = 0, need = K;
-    for (int shift = 24; shift >= 0; shift -= 8) {
+    // MSB-first radix select of the K-th largest key.  The bits above the
+    // highest one in which the smallest and largest keys differ are common to
+    // all keys, so the 8-bit digits start just below them: the scores of one
+    // sequence span a narrow range and the leading digits would otherwise all
+    // fall into one or two histogram bins.
+    const int lane = tid & 31, wid = tid >> 5;
+    unsigned kmin = 0xffffffffu, kmax = 0u;
+    for (int c = tid; c < ncand; c += kSelThreads) {
+      const unsigned key = float_key(gr[c]);
+      kmin = min(kmin, key);
+      kmax = max(kmax, key);
+    }
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    if (lane == 0) {
+      scan[2 * wid] = kmin;
+      scan[2 * wid + 1] = kmax;
+    }
+    __syncthreads();
+    if (wid == 0) {
+      unsigned a = lane < kSelThreads / 32 ? scan[2 * lane] : 0xffffffffu;
+      unsigned z = lane < kSelThreads / 32 ? scan[2 * lane + 1] : 0u;
+      a = __reduce_min_sync(0xffffffffu, a);
+      z = __reduce_max_sync(0xffffffffu, z);
+      if (lane == 0) {
+        prefix_sh = a;
+        need_sh = z;
+      }
+    }
+    __syncthreads();
+    const unsigned diff = prefix_sh ^ need_sh;
+    const unsigned kmax_all = need_sh;
+    __syncthreads();
+    unsigned need = K;
+    // bits above `top` are common to every key
+    const int top = diff ? 31 - __clz(diff) : -1;
+    unsigned prefix = top >= 31 ? 0u : (kmax_all & ~((2u << top) - 1u));
+    for (int hi_bit = top; hi_bit >= 0; hi_bit -= 8) {
+      const int shift = max(0, hi_bit - 7);
+      const unsigned dmask = (2u << (hi_bit - shift)) - 1u;  // digit bits [shift, hi_bit]
       for (int x = tid; x < 256; x += kSelThreads) hist[x] = 0;
       __syncthreads();
-      const unsigned hi_mask = shift == 24 ? 0u : (0xffffffffu << (shift + 8));
+      const unsigned hi_mask = hi_bit >= 31 ? 0u : (0xffffffffu << (hi_bit + 1));
       for (int c = tid; c < ncand; c += kSelThreads) {
         const unsigned key = float_key(gr[c]);
-        if ((key & hi_mask) == (prefix & hi_mask)) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+        if ((key & hi_mask) == (prefix & hi_mask)) atomicAdd(&hist[(key >> shift) & dmask], 1u);
       }
       __syncthreads();
-      if (tid == 0) {
-        unsigned acc = 0;
-        int digit = 255;
-        for (; digit > 0; --digit) {
-          if (acc + hist[digit] >= need) break;
-          acc += hist[digit];
+      if (wid == 0) {
+        // digit of the need-th largest key: lane l holds bins 8l .. 8l+7
+        unsigned h8[8], own = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          h8[j] = hist[8 * lane + j];
+          own += h8[j];
         }
-        prefix_sh = prefix | ((unsigned)digit << shift);
-        need_sh = need - acc;
+        unsigned suf = own;  // keys in bins >= 8 lane
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const unsigned t = __shfl_down_sync(0xffffffffu, suf, o);
+          if (lane + o < 32) suf += t;
+        }
+        const unsigned above = suf - own;  // keys in bins >= 8 (lane + 1)
+        int digit = -1;
+        unsigned acc = above;
+        if (above < need && suf >= need) {
+#pragma unroll
+          for (int j = 7; j >= 0; --j) {
+            if (digit < 0 && acc + h8[j] >= need) digit = j;
+            else if (digit < 0) acc += h8[j];
+          }
+        }
+        const unsigned who = __ballot_sync(0xffffffffu, digit >= 0);
+        const int src = who ? __ffs(who) - 1 : 0;
+        const int dg = __shfl_sync(0xffffffffu, 8 * lane + digit, src);
+        const unsigned ac = __shfl_sync(0xffffffffu, acc, src);
+        if (lane == 0) {
+          prefix_sh = prefix | ((unsigned)dg << shift);
+          need_sh = need - ac;
+        }
       }
       __syncthreads();
       prefix = prefix_sh;
       need = need_sh;
       __syncthreads();
     }
+    if (top < 0) prefix = kmax_all;  // all keys equal
     const unsigned thr = prefix;  // key of the K-th largest; `need` ties at thr are taken
     // strictly greater: order irrelevant (sorted afterwards)
     for (int c = tid; c < ncand; c += kSelThreads) {
