@@ -31,7 +31,7 @@
 // Ring protocol.  The items are the chunks' K and V tiles in stream order,
 // except that chunk r's V tile follows chunk r + DV's K tile: it is needed
 // only after the chunk's S^T and softmax, and holding it in a slot meanwhile
-// costs ring capacity (measured: 96.2 -> 90.0 ms at 128K for DV = 1).  Each
+// costs ring capacity (measured: 96.2 -> 91.1 ms at 128K for DV = 1).  Each
 // consumer then meets at most DV of its items out of stream order, which is
 // deadlock-free while NSI > DV: the producer issues in stream order, and an
 // item's slot is only reused after every earlier item in that slot was
