@@ -170,7 +170,8 @@ def run_prefill(w, dev, steps, warmup, stream):
             ev["score_topk"].append(timed(lambda: H.hils_score_topk(cfg, x["q"], pre.k_sum, pre.b_sum, pre.idx,
                                                                     pre.s_sel, pre.ws, False, qc, stream), stream))
             ev["attn_prefill"].append(timed(lambda: H.hils_attn_prefill(cfg, x["q"], x["k"], x["v"], pre.idx,
-                                                                        pre.s_sel, pre.out, stream), stream))
+                                                                        pre.s_sel, pre.out, pre.ws_attn, stream),
+                                            stream))
         else:
             pre.run(x["q"], x["k"], x["v"], x["q_lmk"], qcal=qc, stream=stream)
 
@@ -371,7 +372,7 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": run_config(w, ws),
             "roofline": roofline, "kernels": per_kernel, "clocks": clocks,
-            "gpu_launches": (3 + (1 if w.d_model else 0)) * args.steps}
+            "gpu_launches": (2 + (1 if w.d_model else 0) + 5 * attn_tiles(w)) * args.steps}
     if not args.no_e2e:
         e2e_ms, h2d, d2h = e2e_prefill(w, x, pre, stream, max(2, args.steps // 3), dist_on)
         line["e2e"] = {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
@@ -415,6 +416,16 @@ def main():
     if dist_on:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
+
+
+def attn_tiles(w) -> int:
+    """Position tiles of the chunk-major attention (hils.h, hils_attn_prefill):
+    the fewest tiles whose 1 KB partial records (one per position, KV group and
+    selected chunk) fit about 8 GiB each.  Each tile launches five kernels:
+    bucket count, scan and scatter, the chunk-major pass, the window pass."""
+    per_pos = w.B * w.Hkv * w.K * w.G * w.d * 2
+    cap = max(1, (8 << 30) // per_pos)
+    return (w.N + cap - 1) // cap
 
 
 def run_config(w, ws):

@@ -1,0 +1,563 @@
+// Selected-chunk attention, chunk-major, on the tcgen05 tensor cores (bf16
+// prefill, d = 128, S = 64, G = 4).
+//
+// hyper.ai summary of arXiv 2607.02980 (HiLS-Attention), section 方法
+// (Method): every selected chunk c of position i is attended on its own,
+//   O_{i,c} = sum_{j in c} softmax_{j in c}(q_i.k_j * scale) v_j,
+// and the chunk outputs are fused with weights exp(s^_{i,c}) / Z^_i.  O_{i,c}
+// depends on nothing but q_i and chunk c, so the pairs (i, c) can be computed
+// in any grouping.  This file groups them by chunk: the positions that chose
+// chunk c (of one KV group) are gathered 32 at a time (x 4 heads = 128 query
+// rows, the MMA's M), and chunk c's K and V tiles are loaded once for all of
+// them:
+//
+//   S (128 rows x 64 keys)  = Q_rows (128 x d) . K_c^T        tcgen05, fp32 in TMEM
+//   P = softmax over the 64 keys of each row, written as bf16 to shared memory
+//   O (128 rows x 128 d)    = P (128 x 64) . V_c (64 x d)     tcgen05, fp32 in TMEM
+//
+// O is stored as one bf16 record per (position, slot k of its selection list)
+// -- the "partial" -- and the window pass (attn_ring.cu) adds the window's
+// exact softmax terms and fuses the partials with the exp(s^) weights.
+//
+// Why chunk-major: on the pages' i.i.d.-like workloads adjacent positions
+// share almost none of their selected chunks, so a position-major kernel
+// moves a 32 KB K/V tile per (position pair, chunk) into shared memory and
+// reads it back for 8 query rows.  Grouped by chunk, a tile serves ~100+ rows
+// and the work becomes dense tensor-core tiles; the price is the gathered
+// query rows (1 KB per pair, mostly L2 hits) and the partial records (1 KB per
+// pair written here, read once by the window pass).
+//
+// Host-side bucketing (three small kernels per position tile): count the pairs
+// per (sequence, KV group, chunk) bucket, scan the counts into bucket offsets
+// and item offsets (one item = up to 32 positions of one bucket), scatter the
+// pairs into their buckets and write the item table.  The order of the pairs
+// inside a bucket depends on atomic arrival order, but no result does: every
+// output row is computed by the same instructions wherever it sits in a tile.
+//
+// CTA layout (one persistent CTA per SM, 448 threads, items dealt round-robin):
+//   warps 0-3   gather the 128 query rows of an item (cp.async, 128-byte
+//               swizzle, rows past the item's count zero-filled); 3 stages
+//   warp 4      TMA loads of the chunk's K and V tiles; 3 stages
+//   warp 5      tcgen05.mma issue (one thread); S and O double-buffered in TMEM
+//   warps 6-9   softmax: TMEM row -> max, exp2, normalised bf16 P row
+//   warps 10-13 epilogue: TMEM O row -> bf16 partial record
+// Every wait is bounded (status word + early return), see common.cuh.
+#include <algorithm>
+
+#include "launch.h"
+#include "tmap.h"
+
+namespace hils {
+namespace {
+
+constexpr int D = 128, S = 64, G = 4;
+constexpr int PPI = 32;          // positions per item
+constexpr int MR = PPI * G;      // query rows per item (MMA M)
+constexpr int NQS = 3;           // query-row stages
+constexpr int NKV = 3;           // K/V stages
+constexpr int NST = 2;           // S / P / O stages
+constexpr uint32_t QHALF = MR * 128;  // one 64-d half of the gathered rows (16 KB)
+constexpr uint32_t BOX = S * 128;     // [64 keys x 64 d] bf16 (8 KB)
+constexpr int THREADS = 14 * 32;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t OCOL = 0;     // O of stage st at OCOL + 128 st
+constexpr uint32_t SCOL = 256;   // S of stage st at SCOL + 64 st
+constexpr int KMAX = 64;
+
+struct __align__(1024) SmemC {
+  unsigned char q[NQS][2][QHALF];   // [d half][row][128 B], 128-byte swizzle
+  unsigned char k[NKV][2][BOX];     // [d half][key][128 B]
+  unsigned char v[NKV][2][BOX];     // [d half][key][128 B]
+  unsigned char p[NST][MR * 128];   // [row][64 keys x bf16]
+  uint64_t qfull[NQS], qempty[NQS], kvfull[NKV], kvempty[NKV];
+  uint64_t sfull[NST], sfree[NST], pfull[NST], pempty[NST], ofull[NST], ofree[NST], done;
+  uint32_t tmem;
+};
+constexpr size_t kSmemBytes = sizeof(SmemC) + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+
+HILS_DI void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+HILS_DI void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+HILS_DI void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+HILS_DI void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+// Shared-memory descriptor of an MN-major operand with the 128-byte swizzle:
+// 64 MN-elements per 128-byte row, rows of consecutive K 128 B apart in
+// 8-row (1024 B) atoms; `lbo` = bytes between 64-element MN blocks, `sbo` =
+// bytes between 8-row K groups.
+HILS_DI uint64_t sdesc_mn_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1u << 46;  // descriptor version (sm_100)
+  d |= (uint64_t)2u << 61;  // 128-byte swizzle
+  return d;
+}
+
+struct Item {
+  int bg, c, s0, n;
+};
+
+__global__ void __launch_bounds__(THREADS, 1)
+    attn_chunk_kernel(Shape s, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                      const __nv_bfloat16* __restrict__ q, const int* __restrict__ off, const int* __restrict__ ioff,
+                      const int2* __restrict__ items, const int* __restrict__ ent, int t0, int PT,
+                      __nv_bfloat16* __restrict__ part, DevCtx ctx) {
+  extern __shared__ unsigned char smem_raw[];
+  SmemC& sm = *reinterpret_cast<SmemC*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int U = s.B * s.Hkv * s.C;
+  const int nitems = __ldg(ioff + U);
+  const int bid = blockIdx.x, nb = gridDim.x;
+  const int nmine = nitems > bid ? (nitems - 1 - bid) / nb + 1 : 0;
+  auto item_of = [&](int it) -> Item {
+    const int2 e = __ldg(items + bid + it * nb);
+    Item r;
+    r.bg = e.x / s.C;
+    r.c = e.x - r.bg * s.C;
+    r.s0 = e.y;
+    r.n = min(PPI, __ldg(off + e.x + 1) - e.y);
+    return r;
+  };
+
+  if (tid == 0) {
+    for (int x = 0; x < NQS; ++x) {
+      mbar_init(&sm.qfull[x], 128);
+      mbar_init(&sm.qempty[x], 1);
+    }
+    for (int x = 0; x < NKV; ++x) {
+      mbar_init(&sm.kvfull[x], 1);
+      mbar_init(&sm.kvempty[x], 1);
+    }
+    for (int x = 0; x < NST; ++x) {
+      mbar_init(&sm.sfull[x], 1);
+      mbar_init(&sm.sfree[x], 4);
+      mbar_init(&sm.pfull[x], 4);
+      mbar_init(&sm.pempty[x], 1);
+      mbar_init(&sm.ofull[x], 1);
+      mbar_init(&sm.ofree[x], 4);
+    }
+    mbar_init(&sm.done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(&sm.tmem, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem;
+
+  if (warp < 4) {
+    // ------------------------------------------------- query-row gather ----
+    // copy x of 16: row 8x + t/16, 16-byte unit t%16 of its 256-byte q row
+    const int t = tid;
+    const int unit = t & 15, half = unit >> 3, u8 = unit & 7;
+    bool ok = true;
+    int it = 0;
+    for (; it < nmine; ++it) {
+      const int sq = it % NQS;
+      if (it >= NQS) ok = mbar_wait(&sm.qempty[sq], ((it / NQS) - 1) & 1, ctx);
+      if (!__all_sync(0xffffffffu, ok)) {
+        ok = false;
+        break;
+      }
+      const Item im = item_of(it);
+      const int e = lane < im.n ? __ldg(ent + im.s0 + lane) : 0;
+      const int b = im.bg / s.Hkv, g = im.bg - b * s.Hkv;
+      const __nv_bfloat16* qb = q + ((long long)(b * s.Hq + g * G) * s.N + t0) * D + unit * 8;
+      const uint32_t qs = smem_u32(sm.q[sq][half]);
+#pragma unroll 4
+      for (int x = 0; x < 16; ++x) {
+        const int row = 8 * x + (t >> 4);
+        const int j = row >> 2, h = row & 3;
+        const int ej = __shfl_sync(0xffffffffu, e, j);
+        const bool v = j < im.n;
+        const __nv_bfloat16* src = v ? qb + ((long long)h * s.N + (ej >> 6)) * D : q;
+        cp_async16(qs + row * 128 + ((u8 ^ (row & 7)) << 4), src, v ? 16u : 0u);
+      }
+      cp_async_commit();
+      if (it > 0) {
+        // the previous item's rows have landed: publish them to the tensor core
+        cp_async_wait<1>();
+        fence_proxy_async_shared();
+        mbar_arrive(&sm.qfull[(it - 1) % NQS]);
+      }
+    }
+    cp_async_wait<0>();
+    if (ok && it > 0) {
+      fence_proxy_async_shared();
+      mbar_arrive(&sm.qfull[(it - 1) % NQS]);
+    }
+  } else if (warp == 4) {
+    // --------------------------------------------------------- K/V loads ----
+    if (lane == 0) {
+      bool ok = true;
+      int it = 0;
+      if (nmine > 0) {
+        prefetch_tmap(&tmk);
+        prefetch_tmap(&tmv);
+      }
+      for (; it < nmine; ++it) {
+        const int sk = it % NKV;
+        if (it >= NKV) ok = mbar_wait(&sm.kvempty[sk], ((it / NKV) - 1) & 1, ctx);
+        if (!ok) break;
+        const Item im = item_of(it);
+        if (ctx.inject != 1) {
+          mbar_arrive_expect_tx(&sm.kvfull[sk], 4 * BOX);
+          tma_load_3d(sm.k[sk][0], &tmk, 0, im.c * S, im.bg, &sm.kvfull[sk]);
+          tma_load_3d(sm.k[sk][1], &tmk, 64, im.c * S, im.bg, &sm.kvfull[sk]);
+          tma_load_3d(sm.v[sk][0], &tmv, 0, im.c * S, im.bg, &sm.kvfull[sk]);
+          tma_load_3d(sm.v[sk][1], &tmv, 64, im.c * S, im.bg, &sm.kvfull[sk]);
+        }
+      }
+      // copies still in flight (only after a timeout) land before the CTA exits
+      if (!ok && ctx.inject != 1)
+        for (int j = max(0, it - NKV); j < it; ++j) mbar_wait(&sm.kvfull[j % NKV], (j / NKV) & 1, ctx);
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // --------------------------------------------------------- MMA issue ----
+    if (lane == 0) {
+      const uint32_t id1 = idesc_bf16_f32(MR, S);
+      const uint32_t id2 = idesc_bf16_f32(MR, D) | (1u << 16);  // B (V) is MN-major
+      auto mma1 = [&](int j) -> bool {
+        const int st = j % NST, sq = j % NQS, sk = j % NKV;
+        if (!mbar_wait(&sm.qfull[sq], (j / NQS) & 1, ctx)) return false;
+        if (!mbar_wait(&sm.kvfull[sk], (j / NKV) & 1, ctx)) return false;
+        if (j >= NST && !mbar_wait(&sm.sfree[st], ((j / NST) - 1) & 1, ctx)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t a = sdesc_k_sw128(smem_u32(sm.q[sq][kk >> 2]) + (kk & 3) * 32);
+          const uint64_t bd = sdesc_k_sw128(smem_u32(sm.k[sk][kk >> 2]) + (kk & 3) * 32);
+          mma_ss(tmem + SCOL + 64 * st, a, bd, id1, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&sm.sfull[st]);
+        tc_commit(&sm.qempty[sq]);
+        return true;
+      };
+      auto mma2 = [&](int j) -> bool {
+        const int st = j % NST, sk = j % NKV;
+        if (!mbar_wait(&sm.pfull[st], (j / NST) & 1, ctx)) return false;
+        if (j >= NST && !mbar_wait(&sm.ofree[st], ((j / NST) - 1) & 1, ctx)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t a = sdesc_k_sw128(smem_u32(sm.p[st]) + kk * 32);
+          const uint64_t bd = sdesc_mn_sw128(smem_u32(sm.v[sk][0]) + kk * 2048, BOX, 1024);
+          mma_ss(tmem + OCOL + 128 * st, a, bd, id2, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&sm.ofull[st]);
+        tc_commit(&sm.kvempty[sk]);
+        tc_commit(&sm.pempty[st]);
+        return true;
+      };
+      // S of item j + 1 is computed while the softmax of item j runs
+      bool ok = nmine == 0 || mma1(0);
+      for (int it = 0; it < nmine && ok; ++it) {
+        if (it + 1 < nmine) ok = mma1(it + 1);
+        if (ok) ok = mma2(it);
+      }
+      // every MMA issued above has completed before the columns are released
+      tc_commit(&sm.done);
+      mbar_wait(&sm.done, 0, ctx);
+    }
+    __syncwarp();
+  } else if (warp < 10) {
+    // ----------------------------------------------------------- softmax ----
+    const int qw = warp & 3, row = 32 * qw + lane;
+    const uint32_t lrow = (uint32_t)(32 * qw) << 16;
+    const float sl2 = s.scale * kLog2e;
+    bool ok = true;
+    for (int it = 0; it < nmine; ++it) {
+      const int st = it % NST;
+      ok = mbar_wait(&sm.sfull[st], (it / NST) & 1, ctx);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      uint32_t r0[32], r1[32];
+      tmem_ld32(tmem + lrow + SCOL + 64 * st, r0);
+      tmem_ld32(tmem + lrow + SCOL + 64 * st + 32, r1);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.sfree[st]);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) mx = fmaxf(mx, fmaxf(__uint_as_float(r0[j]), __uint_as_float(r1[j])));
+      const float base = mx * sl2;
+      float l = 0.f;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float e0 = exp2f(fmaf(__uint_as_float(r0[j]), sl2, -base));
+        const float e1 = exp2f(fmaf(__uint_as_float(r1[j]), sl2, -base));
+        r0[j] = __float_as_uint(e0);
+        r1[j] = __float_as_uint(e1);
+        l += e0 + e1;
+      }
+      const float inv = 1.f / l;
+      if (it >= NST) ok = mbar_wait(&sm.pempty[st], ((it / NST) - 1) & 1, ctx);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const uint32_t pb = smem_u32(sm.p[st]) + row * 128;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        // 16-byte unit u = keys 8u .. 8u + 7
+        uint32_t w[4];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          const int kx = 8 * u + 2 * x;
+          const float a = __uint_as_float(kx < 32 ? r0[kx] : r1[kx - 32]) * inv;
+          const float c = __uint_as_float(kx + 1 < 32 ? r0[kx + 1] : r1[kx + 1 - 32]) * inv;
+          w[x] = pack_bf16x2(a, c);
+        }
+        st_shared_v4(pb + ((u ^ (row & 7)) << 4), w[0], w[1], w[2], w[3]);
+      }
+      fence_proxy_async_shared();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.pfull[st]);
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue ----
+    // Partial record of (position, slot k): [head][128] bf16, each head's 128
+    // values stored in four 32-value blocks; inside block a, element
+    // 4 r + t holds d = 32 a + r + 8 t (r = 0..7, t = 0..3), the order in
+    // which the window pass's MMA fragments consume them.
+    const int qw = warp & 3, row = 32 * qw + lane, jr = row >> 2, h = row & 3;
+    const uint32_t lrow = (uint32_t)(32 * qw) << 16;
+    bool ok = true;
+    for (int it = 0; it < nmine; ++it) {
+      const int st = it % NST;
+      const Item im = item_of(it);
+      const bool valid = jr < im.n;
+      const int e = valid ? __ldg(ent + im.s0 + jr) : 0;
+      __nv_bfloat16* dst = part + (((long long)im.bg * PT + (e >> 6)) * s.K + (e & 63)) * (G * D) + h * D;
+      ok = mbar_wait(&sm.ofull[st], (it / NST) & 1, ctx);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lrow + OCOL + 128 * st + 32 * a, v);
+        tmem_wait_ld();
+        uint32_t w[16];
+#pragma unroll
+        for (int x = 0; x < 16; ++x) {
+          const int d0 = (x >> 1) + 16 * (x & 1);
+          w[x] = pack_bf16x2(__uint_as_float(v[d0]), __uint_as_float(v[d0 + 8]));
+        }
+        if (valid) {
+          uint4* o = reinterpret_cast<uint4*>(dst + 32 * a);
+          o[0] = make_uint4(w[0], w[1], w[2], w[3]);
+          o[1] = make_uint4(w[4], w[5], w[6], w[7]);
+          o[2] = make_uint4(w[8], w[9], w[10], w[11]);
+          o[3] = make_uint4(w[12], w[13], w[14], w[15]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.ofree[st]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 5) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+// ------------------------------------------------------------ bucketing ----
+// The pairs of a position tile [t0, t0 + np): entry x = ((bg * np + pl) * K + k).
+HILS_DI bool pair_of(const Shape& s, const int32_t* __restrict__ idx, int t0, int np, long long x, int& u, int& pl,
+                     int& k) {
+  k = (int)(x % s.K);
+  const long long r = x / s.K;
+  pl = (int)(r % np);
+  const int bg = (int)(r / np);
+  const int p = t0 + pl;
+  const int c = __ldg(idx + ((long long)bg * s.N + p) * s.K + k);
+  const int ncand = max(0, p / S - s.nw + 1);
+  u = bg * s.C + c;
+  return c >= 0 && c < ncand;
+}
+
+__global__ void bucket_count_kernel(Shape s, const int32_t* __restrict__ idx, int t0, int np, int* __restrict__ cnt) {
+  const long long total = (long long)s.B * s.Hkv * np * s.K;
+  for (long long x = blockIdx.x * (long long)blockDim.x + threadIdx.x; x < total; x += (long long)gridDim.x * blockDim.x) {
+    int u, pl, k;
+    if (pair_of(s, idx, t0, np, x, u, pl, k)) atomicAdd(cnt + u, 1);
+  }
+}
+
+// One block: exclusive scans of the bucket counts (pair offsets) and of their
+// item counts ceil(n / 32) (item offsets); cnt becomes the scatter cursor.
+__global__ void __launch_bounds__(1024) bucket_scan_kernel(int U, int* __restrict__ cnt, int* __restrict__ off,
+                                                           int* __restrict__ ioff) {
+  __shared__ int wa[32], wb[32];
+  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+  const int per = (U + 1023) / 1024;
+  const int u0 = min(U, t * per), u1 = min(U, u0 + per);
+  int sa = 0, sb = 0;
+  for (int u = u0; u < u1; ++u) {
+    const int n = cnt[u];
+    sa += n;
+    sb += (n + PPI - 1) / PPI;
+  }
+  int ia = sa, ib = sb;  // inclusive warp scans
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int xa = __shfl_up_sync(0xffffffffu, ia, o), xb = __shfl_up_sync(0xffffffffu, ib, o);
+    if (lane >= o) {
+      ia += xa;
+      ib += xb;
+    }
+  }
+  if (lane == 31) {
+    wa[w] = ia;
+    wb[w] = ib;
+  }
+  __syncthreads();
+  if (w == 0) {
+    int xa = wa[lane], xb = wb[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int ya = __shfl_up_sync(0xffffffffu, xa, o), yb = __shfl_up_sync(0xffffffffu, xb, o);
+      if (lane >= o) {
+        xa += ya;
+        xb += yb;
+      }
+    }
+    wa[lane] = xa;  // inclusive over warps
+    wb[lane] = xb;
+  }
+  __syncthreads();
+  int ea = ia - sa + (w > 0 ? wa[w - 1] : 0), eb = ib - sb + (w > 0 ? wb[w - 1] : 0);
+  for (int u = u0; u < u1; ++u) {
+    const int n = cnt[u];
+    off[u] = ea;
+    ioff[u] = eb;
+    cnt[u] = ea;
+    ea += n;
+    eb += (n + PPI - 1) / PPI;
+  }
+  if (t == 1023) {
+    off[U] = ea;
+    ioff[U] = eb;
+  }
+}
+
+__global__ void bucket_scatter_kernel(Shape s, const int32_t* __restrict__ idx, int t0, int np,
+                                      const int* __restrict__ off, const int* __restrict__ ioff, int* __restrict__ cur,
+                                      int* __restrict__ ent, int2* __restrict__ items) {
+  const long long total = (long long)s.B * s.Hkv * np * s.K;
+  for (long long x = blockIdx.x * (long long)blockDim.x + threadIdx.x; x < total; x += (long long)gridDim.x * blockDim.x) {
+    int u, pl, k;
+    if (!pair_of(s, idx, t0, np, x, u, pl, k)) continue;
+    const int slot = atomicAdd(cur + u, 1);
+    ent[slot] = (pl << 6) | k;
+    const int rel = slot - __ldg(off + u);
+    if (rel % PPI == 0) items[__ldg(ioff + u) + rel / PPI] = make_int2(u, slot);
+  }
+}
+
+size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// workspace pieces, in order
+struct ChunkWs {
+  size_t cnt, off, ioff, ent, items, part, total;
+  int PT;
+};
+
+// Positions per tile: the fewest tiles whose partial records fit about
+// kPartBudget bytes each, of equal size rounded up to a multiple of the window
+// pass's block (14 positions).
+constexpr size_t kPartBudget = size_t(8) << 30;
+constexpr int kRingBlock = 14;
+
+ChunkWs chunk_ws(const Shape& s) {
+  ChunkWs w{};
+  const size_t per_pos = (size_t)s.B * s.Hkv * s.K * G * D * 2;
+  const long long cap = std::max<long long>(1, (long long)(kPartBudget / per_pos));
+  const long long ntiles = (s.N + cap - 1) / cap;
+  const long long pt = (s.N + ntiles - 1) / ntiles;
+  w.PT = (int)((pt + kRingBlock - 1) / kRingBlock * kRingBlock);
+  const size_t U = (size_t)s.B * s.Hkv * s.C;
+  const size_t pairs = (size_t)s.B * s.Hkv * w.PT * s.K;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t r = o;
+    o += up256(bytes);
+    return r;
+  };
+  w.cnt = take((U + 1) * 4);
+  w.off = take((U + 1) * 4);
+  w.ioff = take((U + 1) * 4);
+  w.ent = take(pairs * 4);
+  w.items = take((pairs / PPI + U + 1) * 8);
+  w.part = take(pairs * G * D * 2);
+  w.total = o;
+  return w;
+}
+
+}  // namespace
+
+size_t attn_prefill_tc_workspace(const Shape& s) {
+  if (s.d != D || s.S != S || s.G != G || s.K > KMAX) return 0;
+  return chunk_ws(s).total;
+}
+
+cudaError_t launch_attn_prefill_chunked(const Shape& s, const void* q, const void* k, const void* v,
+                                        const int32_t* idx, const float* s_sel, void* out, void* ws,
+                                        cudaStream_t st, const DevCtx& ctx) {
+  if (s.d != D || s.S != S || s.G != G || s.K > KMAX) return cudaErrorNotSupported;
+  const ChunkWs w = chunk_ws(s);
+  unsigned char* W = (unsigned char*)ws;
+  int* cnt = (int*)(W + w.cnt);
+  int* off = (int*)(W + w.off);
+  int* ioff = (int*)(W + w.ioff);
+  int* ent = (int*)(W + w.ent);
+  int2* items = (int2*)(W + w.items);
+  __nv_bfloat16* part = (__nv_bfloat16*)(W + w.part);
+  const int U = s.B * s.Hkv * s.C;
+
+  CUtensorMap tmk, tmv;
+  const uint64_t dims[3] = {(uint64_t)D, (uint64_t)s.N, (uint64_t)s.B * s.Hkv};
+  const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)s.N * D * 2};
+  const uint32_t box[3] = {64, (uint32_t)S, 1};
+  cudaError_t e = make_tmap_bf16(&tmk, k, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e != cudaSuccess) return e;
+  e = make_tmap_bf16(&tmv, v, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e != cudaSuccess) return e;
+  e = ensure_dynamic_smem((const void*)attn_chunk_kernel, (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int sms = device_sm_count();
+
+  for (int t0 = 0; t0 < s.N; t0 += w.PT) {
+    const int np = std::min(w.PT, s.N - t0);
+    if (U > 0) {
+      e = cudaMemsetAsync(cnt, 0, (size_t)U * 4, st);
+      if (e != cudaSuccess) return e;
+      const long long pairs = (long long)s.B * s.Hkv * np * s.K;
+      const int grid = (int)std::min<long long>((pairs + 255) / 256, (long long)sms * 16);
+      bucket_count_kernel<<<grid, 256, 0, st>>>(s, idx, t0, np, cnt);
+      bucket_scan_kernel<<<1, 1024, 0, st>>>(U, cnt, off, ioff);
+      bucket_scatter_kernel<<<grid, 256, 0, st>>>(s, idx, t0, np, off, ioff, cnt, ent, items);
+      attn_chunk_kernel<<<sms, THREADS, kSmemBytes, st>>>(s, tmk, tmv, (const __nv_bfloat16*)q, off, ioff, items, ent,
+                                                          t0, w.PT, part, ctx);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
+    e = launch_attn_window_merge(s, q, k, v, idx, s_sel, out, U > 0 ? part : nullptr, t0, t0 + np, w.PT, st, ctx);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace hils

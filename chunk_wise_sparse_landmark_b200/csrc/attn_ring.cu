@@ -128,17 +128,19 @@ struct Walk {
 __global__ void __launch_bounds__(THREADS, 2)
     attn_ring_kernel(Shape s, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                      const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ idx,
-                     const float* __restrict__ s_sel, __nv_bfloat16* __restrict__ out, DevCtx ctx) {
+                     const float* __restrict__ s_sel, __nv_bfloat16* __restrict__ out,
+                     const __nv_bfloat16* __restrict__ part, int t0, int t1, int PT, DevCtx ctx) {
   extern __shared__ unsigned char smem_raw[];
   SmemR& sm = *reinterpret_cast<SmemR*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = blockIdx.y, b = blockIdx.z;
   const int bg = b * s.Hkv + g;
-  const int i0 = blockIdx.x * BP;
+  const int i0 = t0 + blockIdx.x * BP;
+  const int nend = min(s.N, t1);  // this launch's positions: [t0, nend)
   const int K = s.K;
   // stream: selected chunks below lo (bitmap, ascending), then every chunk lo..hi
   const int lo = max(0, i0 / S - s.nw + 1);    // first window chunk of the block
-  const int hi = (min(i0 + BP, s.N) - 1) / S;  // chunk of the block's last position
+  const int hi = (min(i0 + BP, nend) - 1) / S;  // chunk of the block's last position
   const int nwords = (lo + 31) >> 5;
 
   for (int x = tid; x < nwords; x += THREADS) sm.bits[x] = 0u;
@@ -157,8 +159,8 @@ __global__ void __launch_bounds__(THREADS, 2)
 
   // consumer state (warp < CW): positions p0, p0 + 1 (same chunk: p0 is even)
   const int p0 = i0 + 2 * warp;
-  const bool valid0 = warp < CW && p0 < s.N;
-  const bool valid1 = warp < CW && p0 + 1 < s.N;
+  const bool valid0 = warp < CW && p0 < nend;
+  const bool valid1 = warp < CW && p0 + 1 < nend;
   const int cur = p0 / S;
   const int ncand = max(0, cur - s.nw + 1);
   const int wc0 = ncand;  // this warp's window chunks wc0..cur
@@ -179,6 +181,12 @@ __global__ void __launch_bounds__(THREADS, 2)
     l0b = l0b < ncand ? l0b : -1;
     l1a = l1a < ncand ? l1a : -1;
     l1b = l1b < ncand ? l1b : -1;
+  }
+  // with partial records the selected chunks were attended elsewhere: the
+  // lists are kept for the fusion at the end and the stream is the window only
+  const int m0a = l0a, m0b = l0b, m1a = l1a, m1b = l1b;
+  if (part) l0a = l0b = l1a = l1b = -1;
+  if (warp < CW) {
     if (l0a >= 0 && l0a < lo) atomicOr(&sm.bits[l0a >> 5], 1u << (l0a & 31));
     if (l0b >= 0 && l0b < lo) atomicOr(&sm.bits[l0b >> 5], 1u << (l0b & 31));
     if (l1a >= 0 && l1a < lo) atomicOr(&sm.bits[l1a >> 5], 1u << (l1a & 31));
@@ -475,6 +483,36 @@ __global__ void __launch_bounds__(THREADS, 2)
       if (lane == 0) mbar_arrive(&sm.empty[vit % NSI]);
     }
 
+    // ---- selected chunks from their partial records O_c (attn_chunk.cu):
+    // acc += e^{s^ - m} O_c, den += e^{s^ - m}.  Block a of a record's head row
+    // holds d = 32 a + r + 8 t at element 4 r + t, so the 8-byte word at
+    // 32 a + 4 gq is this thread's d = 16 (2a) + gq (+8) and 16 (2a + 1) + gq (+8).
+    if (part && ok) {
+      const __nv_bfloat16* rec = part + (((long long)bg * PT + (my_pos - t0)) * K) * (G * D) + 4 * gq;
+#pragma unroll 2
+      for (int x = 0; x < K; ++x) {
+        const int ca = entry(m0a, m0b, x), cb = entry(m1a, m1b, x);
+        if (my_valid && (my_q == 0 ? ca : cb) >= 0) {
+          const __nv_bfloat16* rx = rec + (long long)x * (G * D);
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const float wgt = exp2f(__ldg(ss0 + r * sstride + x) * kLog2e - m2[r]);
+            den[r] += wgt;
+            const __nv_bfloat16* rh = rx + (my_h + r) * D;
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+              const uint2 u = __ldg(reinterpret_cast<const uint2*>(rh + 32 * a));
+              const float2 f0 = bf16x2_to_f32x2(u.x), f1 = bf16x2_to_f32x2(u.y);
+              acc[2 * a][r] = fmaf(wgt, f0.x, acc[2 * a][r]);
+              acc[2 * a][2 + r] = fmaf(wgt, f0.y, acc[2 * a][2 + r]);
+              acc[2 * a + 1][r] = fmaf(wgt, f1.x, acc[2 * a + 1][r]);
+              acc[2 * a + 1][2 + r] = fmaf(wgt, f1.y, acc[2 * a + 1][2 + r]);
+            }
+          }
+        }
+      }
+    }
+
     // ---- epilogue: thread holds d = 16 mt + gq (acc[mt][0/1]) and 16 mt + gq + 8
     // (acc[mt][2/3]) of its rows 2c4, 2c4+1 (position my_pos, heads my_h, my_h + 1);
     // the 8 lanes of a quad column write 16 consecutive bytes per store
@@ -497,9 +535,11 @@ constexpr size_t kSmemBytes = sizeof(SmemR) + 1024;
 
 }  // namespace
 
-cudaError_t launch_attn_prefill_tc(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
-                                   const float* s_sel, void* out, cudaStream_t st, const DevCtx& ctx) {
+cudaError_t launch_attn_window_merge(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
+                                     const float* s_sel, void* out, const void* part, int t0, int t1, int PT,
+                                     cudaStream_t st, const DevCtx& ctx) {
   if (s.d != D || s.S != S || s.G != G || s.K > KMAX || s.C > MAXC || s.nw > 32) return cudaErrorNotSupported;
+  if (t0 % 2 || t1 <= t0) return cudaErrorInvalidValue;
   CUtensorMap tmk, tmv;
   const uint64_t dims[3] = {(uint64_t)D, (uint64_t)s.N, (uint64_t)s.B * s.Hkv};
   const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)s.N * D * 2};
@@ -510,10 +550,16 @@ cudaError_t launch_attn_prefill_tc(const Shape& s, const void* q, const void* k,
   if (e != cudaSuccess) return e;
   e = ensure_dynamic_smem((const void*)attn_ring_kernel, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid((s.N + BP - 1) / BP, s.Hkv, s.B);
+  dim3 grid((t1 - t0 + BP - 1) / BP, s.Hkv, s.B);
   attn_ring_kernel<<<grid, THREADS, kSmemBytes, st>>>(s, tmk, tmv, (const __nv_bfloat16*)q, idx, s_sel,
-                                                      (__nv_bfloat16*)out, ctx);
+                                                      (__nv_bfloat16*)out, (const __nv_bfloat16*)part, t0, t1, PT,
+                                                      ctx);
   return cudaGetLastError();
+}
+
+cudaError_t launch_attn_prefill_tc(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
+                                   const float* s_sel, void* out, cudaStream_t st, const DevCtx& ctx) {
+  return launch_attn_window_merge(s, q, k, v, idx, s_sel, out, nullptr, 0, s.N, 0, st, ctx);
 }
 
 }  // namespace hils

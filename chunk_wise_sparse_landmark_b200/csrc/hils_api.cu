@@ -119,8 +119,16 @@ size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 // Offsets, in the caller's workspace, of the device copies of the inputs and of
 // every intermediate tensor of hils_prefill_host.
 struct HostLayout {
-  size_t q, k, v, qlmk, ksum, bsum, idx, ssel, out, h, wd, wu, qt, total;
+  size_t q, k, v, qlmk, ksum, bsum, idx, ssel, out, attn, h, wd, wu, qt, total;
 };
+// one (sequence, KV group) piece of a shape: its G query heads and one KV head
+Shape piece_shape(const Shape& s) {
+  Shape sub = s;
+  sub.B = 1;
+  sub.Hq = s.G;
+  sub.Hkv = 1;
+  return sub;
+}
 HostLayout host_layout(const Shape& s, int rank) {
   HostLayout L{};
   size_t off = 0;
@@ -139,6 +147,7 @@ HostLayout host_layout(const Shape& s, int rank) {
   L.idx = take((size_t)s.B * s.Hkv * s.N * s.K * 4);
   L.ssel = take((size_t)s.B * s.Hq * s.N * s.K * 4);
   L.out = take((size_t)s.B * s.Hq * s.N * s.d * e);
+  L.attn = take(s.dtype == HILS_BF16 ? attn_prefill_tc_workspace(piece_shape(s)) : 0);
   if (rank > 0) {
     const size_t dm = (size_t)s.Hq * s.d;  // the supported Q-Cal width
     L.h = take((size_t)s.B * s.N * dm * e);
@@ -242,6 +251,8 @@ size_t hils_workspace_bytes(const hils_config_t* cfg, int32_t which, int32_t qca
       return decode_attn_workspace(s);
     case HILS_WS_PREFILL_HOST:
       return host_layout(s, qcal_rank > 0 ? qcal_rank : 0).total;
+    case HILS_WS_ATTN_PREFILL:
+      return s.dtype == HILS_BF16 ? attn_prefill_tc_workspace(s) : 0;
   }
   return (size_t)-1;
 }
@@ -289,19 +300,29 @@ hils_status_t hils_score_topk(const hils_config_t* cfg, const void* q, const hil
 }
 
 hils_status_t hils_attn_prefill(const hils_config_t* cfg, const void* q, const void* k, const void* v,
-                                const int32_t* idx, const float* s_sel, void* out, void* stream) {
+                                const int32_t* idx, const float* s_sel, void* out, void* workspace,
+                                size_t ws_bytes, void* stream) {
   Shape s;
   HILS_TRY(make_shape(cfg, &s, false));
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(s_sel) || !aligned16(out))
     return fail(HILS_ERR_INVALID_ARG, "hils_attn_prefill: NULL or unaligned pointer");
+  const bool bf16 = s.dtype == HILS_BF16;
+  const bool chunked = bf16 && (workspace || ws_bytes > 0);
+  if (bf16 && (((uintptr_t)q | (uintptr_t)k | (uintptr_t)v) & 31u))
+    return fail(HILS_ERR_INVALID_ARG, "hils_attn_prefill: bf16 q, k, v must be 32-byte aligned");
+  if (chunked) {
+    const size_t need = attn_prefill_tc_workspace(s);
+    if (ws_bytes < need || !aligned16(workspace))
+      return fail(HILS_ERR_INVALID_ARG, "hils_attn_prefill: workspace needs %zu bytes (got %zu)", need, ws_bytes);
+  }
   DevCtx ctx;
   HILS_TRY(dev_ctx(&ctx));
   cudaStream_t st = (cudaStream_t)stream;
-  if (s.dtype == HILS_F32) {
+  if (!bf16) {
     HILS_LAUNCH(launch_attn_prefill_simt(s, q, k, v, idx, s_sel, out, st, ctx), "attn_prefill_simt");
+  } else if (chunked) {
+    HILS_LAUNCH(launch_attn_prefill_chunked(s, q, k, v, idx, s_sel, out, workspace, st, ctx), "attn_prefill_chunked");
   } else {
-    if (((uintptr_t)q | (uintptr_t)k | (uintptr_t)v) & 31u)
-      return fail(HILS_ERR_INVALID_ARG, "hils_attn_prefill: bf16 q, k, v must be 32-byte aligned");
     HILS_LAUNCH(launch_attn_prefill_tc(s, q, k, v, idx, s_sel, out, st, ctx), "attn_prefill_tc");
   }
   return HILS_OK;
@@ -340,10 +361,8 @@ hils_status_t hils_prefill_host(const hils_config_t* cfg, const void* h_q, const
   const size_t e = esize(s);
   const int P = s.B * s.Hkv;  // pieces: (sequence, KV group)
   const size_t nq = (size_t)s.G * s.N * s.d * e, nkv = (size_t)s.N * s.d * e, nql = (size_t)s.G * s.C * s.d * e;
-  Shape sub = s;  // one piece: one sequence, one KV group and its G query heads
-  sub.B = 1;
-  sub.Hq = s.G;
-  sub.Hkv = 1;
+  const Shape sub = piece_shape(s);  // one piece: one sequence, one KV group and its G query heads
+  unsigned char* dattn = W + L.attn;
   auto piece = [&](int p, size_t* oq, size_t* okv, size_t* oql, size_t* obs, size_t* oidx, size_t* oss) {
     const size_t b = p / s.Hkv, g = p % s.Hkv, h0 = b * s.Hq + g * s.G, kv = b * s.Hkv + g;
     *oq = h0 * s.N * s.d * e;
@@ -387,8 +406,9 @@ hils_status_t hils_prefill_host(const hils_config_t* cfg, const void* h_q, const
       } else {
         HILS_LAUNCH(launch_score_topk_tc(sub, dq + oq, dks + oql, dbs + obs, didx + oidx, dss + oss, st, ctx),
                     "score_topk_tc");
-        HILS_LAUNCH(launch_attn_prefill_tc(sub, dq + oq, dk + okv, dv + okv, didx + oidx, dss + oss, dout + oq, st, ctx),
-                    "attn_prefill_tc");
+        HILS_LAUNCH(launch_attn_prefill_chunked(sub, dq + oq, dk + okv, dv + okv, didx + oidx, dss + oss, dout + oq,
+                                                dattn, st, ctx),
+                    "attn_prefill_chunked");
       }
       HILS_CK(cudaEventRecord(ev_att[p], st), "cudaEventRecord");
       HILS_CK(cudaStreamWaitEvent(co, ev_att[p], 0), "cudaStreamWaitEvent");
@@ -417,8 +437,9 @@ hils_status_t hils_prefill_host(const hils_config_t* cfg, const void* h_q, const
     for (int p = 0; p < P; ++p) {
       size_t oq, okv, oql, obs, oidx, oss;
       piece(p, &oq, &okv, &oql, &obs, &oidx, &oss);
-      HILS_LAUNCH(launch_attn_prefill_tc(sub, dq + oq, dk + okv, dv + okv, didx + oidx, dss + oss, dout + oq, st, ctx),
-                  "attn_prefill_tc");
+      HILS_LAUNCH(launch_attn_prefill_chunked(sub, dq + oq, dk + okv, dv + okv, didx + oidx, dss + oss, dout + oq,
+                                              dattn, st, ctx),
+                  "attn_prefill_chunked");
       HILS_CK(cudaEventRecord(ev_att[p], st), "cudaEventRecord");
       HILS_CK(cudaStreamWaitEvent(co, ev_att[p], 0), "cudaStreamWaitEvent");
       HILS_CK(cudaMemcpyAsync(hout + oq, dout + oq, nq, cudaMemcpyDeviceToHost, co), "download out");

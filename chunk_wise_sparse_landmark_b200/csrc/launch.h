@@ -43,9 +43,22 @@ cudaError_t launch_score_topk_decode(const Shape& s, const void* q, const void* 
 cudaError_t launch_attn_prefill_simt(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
                                      const float* s_sel, void* out, cudaStream_t st, const DevCtx& ctx);
 
-// bf16 tensor-core prefill attention (d=128, S=64)
+// bf16 prefill attention (d=128, S=64), one pass that streams each block's
+// chunk union (no workspace)
 cudaError_t launch_attn_prefill_tc(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
                                    const float* s_sel, void* out, cudaStream_t st, const DevCtx& ctx);
+// the window pass over positions [t0, t1); with `part` (partial records of the
+// selected chunks, tile of PT positions) it attends the window only and fuses
+// the records, without it it also streams the selected chunks
+cudaError_t launch_attn_window_merge(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
+                                     const float* s_sel, void* out, const void* part, int t0, int t1, int PT,
+                                     cudaStream_t st, const DevCtx& ctx);
+// bf16 prefill attention, chunk-major selected chunks (tcgen05) + window pass,
+// by position tiles; workspace of attn_prefill_tc_workspace(s) bytes
+size_t attn_prefill_tc_workspace(const Shape& s);
+cudaError_t launch_attn_prefill_chunked(const Shape& s, const void* q, const void* k, const void* v,
+                                        const int32_t* idx, const float* s_sel, void* out, void* ws,
+                                        cudaStream_t st, const DevCtx& ctx);
 
 // decode attention (all dtypes): split-KV partials + merge
 size_t decode_attn_workspace(const Shape& s);

@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(_PKG, "libhils.so")
 
 HILS_OK, HILS_ERR_INVALID_ARG, HILS_ERR_UNSUPPORTED, HILS_ERR_CUDA, HILS_ERR_TIMEOUT = range(5)
 HILS_F32, HILS_BF16 = 0, 1
-HILS_WS_SCORE_PREFILL, HILS_WS_SCORE_DECODE, HILS_WS_ATTN_DECODE, HILS_WS_PREFILL_HOST = 0, 1, 2, 3
+HILS_WS_SCORE_PREFILL, HILS_WS_SCORE_DECODE, HILS_WS_ATTN_DECODE, HILS_WS_PREFILL_HOST, HILS_WS_ATTN_PREFILL = range(5)
 
 EXPORTS = (
     "hils_build_summaries",
@@ -80,7 +80,7 @@ def load() -> ctypes.CDLL:
         P, C = ctypes.c_void_p, ctypes.POINTER(Config)
         lib.hils_build_summaries.argtypes = [C, P, P, P, P, P]
         lib.hils_score_topk.argtypes = [C, P, ctypes.POINTER(QCal), P, P, P, P, P, ctypes.c_size_t, ctypes.c_int32, P]
-        lib.hils_attn_prefill.argtypes = [C, P, P, P, P, P, P, P]
+        lib.hils_attn_prefill.argtypes = [C, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         lib.hils_attn_decode.argtypes = [C, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         lib.hils_attn_decode_noalloc.argtypes = [C, P, P, P, P, P, P, P]
         lib.hils_prefill_host.argtypes = [C, P, P, P, P, ctypes.POINTER(QCal), P, P, ctypes.c_size_t, P]
@@ -150,9 +150,12 @@ def hils_score_topk(cfg: Config, q, k_sum, b_sum, idx, s_sel, workspace=None, de
                                   _p(workspace), ws_bytes, 1 if decode else 0, _stream(stream)))
 
 
-def hils_attn_prefill(cfg: Config, q, k, v, idx, s_sel, out, stream=None):
+def hils_attn_prefill(cfg: Config, q, k, v, idx, s_sel, out, workspace=None, stream=None):
+    """workspace: None (bf16: the pass without scratch) or a device buffer of
+    workspace_bytes(cfg, HILS_WS_ATTN_PREFILL) bytes."""
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(load().hils_attn_prefill(ctypes.byref(cfg), _p(q), _p(k), _p(v), _p(idx), _p(s_sel), _p(out),
-                                    _stream(stream)))
+                                    _p(workspace), ws_bytes, _stream(stream)))
 
 
 def _ph(t: torch.Tensor):
@@ -219,11 +222,12 @@ class Prefill:
         self.s_sel = torch.empty((B, Hq, N, K), dtype=torch.float32, device=device)
         self.out = torch.empty((B, Hq, N, d), dtype=dt, device=device)
         self.ws = alloc_workspace(workspace_bytes(cfg, HILS_WS_SCORE_PREFILL, qcal_rank), device)
+        self.ws_attn = alloc_workspace(workspace_bytes(cfg, HILS_WS_ATTN_PREFILL), device)
 
     def run(self, q, k, v, q_lmk, qcal=None, stream=None):
         hils_build_summaries(self.cfg, k, q_lmk, self.k_sum, self.b_sum, stream)
         hils_score_topk(self.cfg, q, self.k_sum, self.b_sum, self.idx, self.s_sel, self.ws, False, qcal, stream)
-        hils_attn_prefill(self.cfg, q, k, v, self.idx, self.s_sel, self.out, stream)
+        hils_attn_prefill(self.cfg, q, k, v, self.idx, self.s_sel, self.out, self.ws_attn, stream)
         return self.out
 
 

@@ -134,9 +134,22 @@ hils_status_t hils_score_topk(const hils_config_t* cfg, const void* q, const hil
  *   out [B, Hq, N, d] (dtype, out).
  * idx entries must be -1 or candidates of their position (checked on device:
  * an out-of-range entry is skipped and recorded in the status word).
+ *   workspace: device scratch of at least
+ *              hils_workspace_bytes(cfg, HILS_WS_ATTN_PREFILL, 0) bytes
+ *              (16-byte aligned; 0 bytes for dtype F32).  With it, bf16 runs
+ *              attend the selected chunks chunk by chunk (the positions that
+ *              chose a chunk share one load of its K and V tiles), write one
+ *              bf16 partial record per (position, selected chunk) into the
+ *              workspace and fuse the records in the window pass, by tiles of
+ *              positions whose records fit the workspace (about 8 GiB).
+ *              workspace = NULL with ws_bytes = 0 selects the pass that needs
+ *              no scratch: each block of 14 positions streams the union of its
+ *              chunks (slower on long contexts; same results within the bf16
+ *              tolerance).  The call owns the workspace until the stream passes it.
  */
 hils_status_t hils_attn_prefill(const hils_config_t* cfg, const void* q, const void* k, const void* v,
-                                const int32_t* idx, const float* s_sel, void* out, void* stream);
+                                const int32_t* idx, const float* s_sel, void* out, void* workspace,
+                                size_t ws_bytes, void* stream);
 
 /*
  * The same attention for one new token per sequence (decode), at position
@@ -213,7 +226,13 @@ hils_status_t hils_prefill_host(const hils_config_t* cfg, const void* h_q, const
                                 const void* h_q_lmk, const hils_qcal_t* qcal, void* h_out, void* workspace,
                                 size_t ws_bytes, void* stream);
 
-enum { HILS_WS_SCORE_PREFILL = 0, HILS_WS_SCORE_DECODE = 1, HILS_WS_ATTN_DECODE = 2, HILS_WS_PREFILL_HOST = 3 };
+enum {
+  HILS_WS_SCORE_PREFILL = 0,
+  HILS_WS_SCORE_DECODE = 1,
+  HILS_WS_ATTN_DECODE = 2,
+  HILS_WS_PREFILL_HOST = 3,
+  HILS_WS_ATTN_PREFILL = 4
+};
 
 /* Bytes of workspace the call `which` needs for this configuration (0 if none);
  * qcal_rank is the Q-Cal rank for HILS_WS_SCORE_PREFILL and

@@ -59,7 +59,7 @@ def test_null_and_unaligned_pointers_rejected():
     assert lib.hils_build_summaries(ctypes.byref(cfg), None, None, None, None, None) == H.HILS_ERR_INVALID_ARG
     p = ctypes.c_void_p(0x1000)
     bad = ctypes.c_void_p(0x1004)
-    assert lib.hils_attn_prefill(ctypes.byref(cfg), p, p, p, p, p, bad, None) == H.HILS_ERR_INVALID_ARG
+    assert lib.hils_attn_prefill(ctypes.byref(cfg), p, p, p, p, p, bad, None, 0, None) == H.HILS_ERR_INVALID_ARG
     assert b"unaligned" in lib.hils_last_error()
     # workspace too small for decode attention
     assert lib.hils_attn_decode(ctypes.byref(cfg), p, p, p, p, p, p, p, 0, None) == H.HILS_ERR_INVALID_ARG
@@ -71,6 +71,36 @@ def test_workspace_sizes():
     ws = H.workspace_bytes(cfg, H.HILS_WS_SCORE_DECODE)
     assert ws == (16 * 32 * 8192 + 16 * 8 * 8192) * 4
     assert H.workspace_bytes(cfg, H.HILS_WS_ATTN_DECODE) > 0
+
+
+def test_attn_prefill_workspace_size():
+    """Chunk-major attention scratch: bucket counts / offsets / item offsets
+    (U + 1 ints each, U = B Hkv C buckets), the pairs of one position tile
+    (ints), the item table (int2, at most pairs / 32 + U + 1 items) and one
+    1 KB bf16 partial record per pair; the fewest equal tiles whose records
+    fit about 8 GiB, rounded up to a multiple of 14 positions."""
+    up = lambda n: (n + 255) // 256 * 256
+    B, N, Hq, Hkv, K = 1, 131072, 32, 8, 32
+    cfg = H.make_config(B, N, Hq, Hkv, 128, 64, 512, K, "bf16")
+    per_pos = B * Hkv * K * 4 * 128 * 2
+    cap = (8 << 30) // per_pos
+    ntiles = -(-N // cap)
+    PT = -(-(-(-N // ntiles)) // 14) * 14
+    assert (ntiles, PT) == (4, 32774)
+    U, pairs = B * Hkv * (N // 64), B * Hkv * PT * K
+    want = 3 * up((U + 1) * 4) + up(pairs * 4) + up((pairs // 32 + U + 1) * 8) + up(pairs * 1024)
+    assert H.workspace_bytes(cfg, H.HILS_WS_ATTN_PREFILL) == want
+    # short sequences: one tile of N rounded up to 14 positions
+    small = H.make_config(2, 1000, 8, 2, 128, 64, 128, 8, "bf16")
+    PT, U = 1008, 2 * 2 * (1000 // 64)
+    pairs = 2 * 2 * PT * 8
+    want = 3 * up((U + 1) * 4) + up(pairs * 4) + up((pairs // 32 + U + 1) * 8) + up(pairs * 1024)
+    assert H.workspace_bytes(small, H.HILS_WS_ATTN_PREFILL) == want
+    assert H.workspace_bytes(H.make_config(1, 512, 4, 1, 64, 32, 64, 4, "f32"), H.HILS_WS_ATTN_PREFILL) == 0
+    lib = H.load()
+    p = ctypes.c_void_p(0x1000)
+    st = lib.hils_attn_prefill(ctypes.byref(small), p, p, p, p, p, p, p, want - 1, None)
+    assert st == H.HILS_ERR_INVALID_ARG and b"workspace" in lib.hils_last_error()
 
 
 def test_prefill_host_workspace_and_host_checks():

@@ -37,7 +37,9 @@ def sample_rows(w, needles=(), n_random=256, seed=0):
     return [(b, p) for b in range(w.B) for p in pos]
 
 
-def _run_forced(w, x):
+def _run_forced(w, x, chunked=True):
+    """chunked: the chunk-major pass with its workspace; otherwise the pass
+    without scratch (each block streams its chunk union)."""
     dm = _dims(w)
     q, k, v, ql = (to_np(x[n]) for n in ("q", "k", "v", "q_lmk"))
     ks, bs = oracle.summaries(dm, k, ql)
@@ -48,8 +50,11 @@ def _run_forced(w, x):
     ssel_t = torch.from_numpy(ssel32.reshape(w.B, w.N, w.Hq, w.K).transpose(0, 2, 1, 3).copy()).to(DEV)
     d = {n: x[n].to(DEV) for n in ("q", "k", "v")}
     out = torch.empty((w.B, w.Hq, w.N, w.d), dtype=torch.bfloat16, device=DEV)
-    H.hils_attn_prefill(H.config_of(w), d["q"], d["k"], d["v"], idx_t.int().contiguous(), ssel_t.contiguous(), out)
+    cfg = H.config_of(w)
+    ws = H.alloc_workspace(H.workspace_bytes(cfg, H.HILS_WS_ATTN_PREFILL), DEV) if chunked else None
+    H.hils_attn_prefill(cfg, d["q"], d["k"], d["v"], idx_t.int().contiguous(), ssel_t.contiguous(), out, ws)
     H.hils_sync_status()
+    del ws
     rows = sample_rows(w, x["needles"])
     ridx = np.array([b * w.N + p for b, p in rows])
     ref = oracle.attend(dm, rows, q, k, v, idx[ridx], ssel32[ridx].astype(np.float64))
@@ -57,31 +62,61 @@ def _run_forced(w, x):
     return np.abs(got - ref).max(), got, ref
 
 
-def test_attn_forced_selection_8k():
+PASSES = pytest.mark.parametrize("chunked", [True, False], ids=["chunk_major", "union_stream"])
+
+
+@PASSES
+def test_attn_forced_selection_8k(chunked):
     w = WORKLOADS["prefill_8k"]
-    err, _, _ = _run_forced(w, prefill_inputs(w))
+    err, _, _ = _run_forced(w, prefill_inputs(w), chunked)
     assert err <= TOL_BF16, err
 
 
-def test_attn_forced_selection_ragged_tail_and_batch():
+@PASSES
+def test_attn_forced_selection_ragged_tail_and_batch(chunked):
     w = WORKLOADS["prefill_8k"].scaled(name="ragged", B=2, N=4096 + 45, Hq=8, Hkv=2, K=8, needles_per_head=2)
-    err, _, _ = _run_forced(w, prefill_inputs(w))
+    err, _, _ = _run_forced(w, prefill_inputs(w), chunked)
     assert err <= TOL_BF16, err
 
 
-def test_attn_forced_selection_long_context_reduced():
+@PASSES
+def test_attn_forced_selection_long_context_reduced(chunked):
     # the 128K workload's K and window on a shorter sequence and fewer heads
     w = WORKLOADS["prefill_128k"].scaled(name="p128r", N=32768, Hq=8, Hkv=2, needles_per_head=8)
-    err, _, _ = _run_forced(w, prefill_inputs(w))
+    err, _, _ = _run_forced(w, prefill_inputs(w), chunked)
     assert err <= TOL_BF16, err
 
 
-def test_attn_forced_selection_wide_window_k64():
+@PASSES
+def test_attn_forced_selection_wide_window_k64(chunked):
     # the 512K workload's K = 64 and W = 1024 on a short sequence
     w = WORKLOADS["prefill_512k_qcal"].scaled(name="k64r", N=16384, Hq=4, Hkv=1, d_model=0, qcal_rank=0,
                                               needles_per_head=4)
+    err, _, _ = _run_forced(w, prefill_inputs(w), chunked)
+    assert err <= TOL_BF16, err
+
+
+def test_attn_forced_selection_several_position_tiles():
+    """B Hkv K = 1024 partial records per position: 8 GiB hold 8192 positions,
+    so this sequence runs as two position tiles (4508 + 4492)."""
+    w = WORKLOADS["prefill_512k_qcal"].scaled(name="tiles", B=4, N=9000, Hq=16, Hkv=4, d_model=0, qcal_rank=0,
+                                              needles_per_head=2)
+    assert w.B * w.Hkv * w.K == 1024
     err, _, _ = _run_forced(w, prefill_inputs(w))
     assert err <= TOL_BF16, err
+
+
+def test_attn_chunk_major_is_deterministic_and_matches_union_stream():
+    """Bucket order inside the chunk-major pass follows atomic arrival order;
+    the output must not: two runs agree bit for bit.  The two passes compute
+    the same quantity (within the bf16 tolerance)."""
+    w = WORKLOADS["prefill_8k"].scaled(name="det", N=6000, Hq=8, Hkv=2, needles_per_head=2)
+    x = prefill_inputs(w)
+    _, a, _ = _run_forced(w, x, True)
+    _, b, _ = _run_forced(w, x, True)
+    _, c, _ = _run_forced(w, x, False)
+    assert np.array_equal(a, b)
+    assert np.abs(a - c).max() <= TOL_BF16
 
 
 def test_attn_constant_values_pass_through():
@@ -179,7 +214,7 @@ def test_prefill_wait_timeout_reports_status(stage):
         H.hils_set_wait_budget(2_000_000)
         H.hils_set_fault_injection(1)
         if stage == "attn":
-            H.hils_attn_prefill(pre.cfg, x["q"], x["k"], x["v"], pre.idx, pre.s_sel, pre.out)
+            H.hils_attn_prefill(pre.cfg, x["q"], x["k"], x["v"], pre.idx, pre.s_sel, pre.out, pre.ws_attn)
         else:
             H.hils_score_topk(pre.cfg, x["q"], pre.k_sum, pre.b_sum, pre.idx, pre.s_sel, pre.ws,
                               qcal=qc if stage == "qcal" else None)
