@@ -12,7 +12,7 @@
 // them:
 //
 //   S (128 rows x 64 keys)  = Q_rows (128 x d) . K_c^T        tcgen05, fp32 in TMEM
-//   P = softmax over the 64 keys of each row, written as bf16 to shared memory
+//   P = softmax over the 64 keys of each row, bf16, written back into TMEM
 //   O (128 rows x 128 d)    = P (128 x 64) . V_c (64 x d)     tcgen05, fp32 in TMEM
 //
 // O is stored as one bf16 record per (position, slot k of its selection list)
@@ -34,14 +34,32 @@
 // inside a bucket depends on atomic arrival order, but no result does: every
 // output row is computed by the same instructions wherever it sits in a tile.
 //
-// CTA layout (one persistent CTA per SM, 448 threads, items dealt round-robin):
-//   warps 0-3   gather the 128 query rows of an item (cp.async, 128-byte
-//               swizzle, rows past the item's count zero-filled); 3 stages
-//   warp 4      TMA loads of the chunk's K and V tiles; 3 stages
-//   warp 5      tcgen05.mma issue (one thread); S and O double-buffered in TMEM
-//   warps 6-9   softmax: TMEM row -> max, exp2, normalised bf16 P row
-//   warps 10-13 epilogue: TMEM O row -> bf16 partial record
-// Every wait is bounded (status word + early return), see common.cuh.
+// CTA layout (one persistent CTA per SM, 576 threads, items dealt round-robin):
+//   warp 0      TMA loads of the chunk's K and V tiles (128-byte swizzle); 6 stages
+//   warp 1      tcgen05.mma issue (one thread); S and O double-buffered in TMEM
+//   warps 2-9   query rows: two groups of four warps take alternate items;
+//               each thread owns one row (its TMEM lane), loads its 256 bytes
+//               with 32-byte global loads and stores them into TMEM, where
+//               they are the A operand of S = Q K^T (no shared-memory staging
+//               and no swizzle for the gathered rows)
+//   warps 10-13 softmax: TMEM S row -> max, exp2 -> normalised bf16 P row,
+//               written back into the first half of the row's S columns; the
+//               second MMA reads P from TMEM (no shared-memory traffic)
+//   warps 14-17 epilogue: TMEM O row -> bf16 partial record
+// 18 warps: the register file is split across the four sub-partitions, so
+// 96 registers per thread is the most that fits.
+//
+// Measured on B200 (clock stamps per role, 128K workload): every role runs at
+// the same period of ~5.5K cycles per item.  Staging the gathered rows in
+// shared memory with 16-byte cp.async held only ~20 KB in flight per SM and
+// set that period; with 32-byte loads into registers and P in TMEM the
+// gather and the softmax take ~3K cycles each and the period is set by the
+// tensor pipe (issue to completion: ~2.3K cycles for the 8 MMAs of S, ~6K for
+// the 4 of O behind them), far above the ~130 cycles per instruction that one
+// issuing thread reaches alone.  Copy-engine gathers issued from all lanes of
+// a warp (one tile::gather4 or one 256-byte bulk copy per row) did not
+// complete on B200 and are not used.  Every wait is bounded (status word +
+// early return), see common.cuh.
 #include <algorithm>
 
 #include "launch.h"
@@ -53,39 +71,40 @@ namespace {
 constexpr int D = 128, S = 64, G = 4;
 constexpr int PPI = 32;          // positions per item
 constexpr int MR = PPI * G;      // query rows per item (MMA M)
-constexpr int NQS = 3;           // query-row stages
-constexpr int NKV = 3;           // K/V stages
+constexpr int NQS = 2;           // query-row stages (TMEM), one per row group
+constexpr int NKV = 6;           // K/V stages
 constexpr int NST = 2;           // S / P / O stages
-constexpr uint32_t QHALF = MR * 128;  // one 64-d half of the gathered rows (16 KB)
 constexpr uint32_t BOX = S * 128;     // [64 keys x 64 d] bf16 (8 KB)
-constexpr int THREADS = 14 * 32;
+constexpr int THREADS = 18 * 32;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t OCOL = 0;     // O of stage st at OCOL + 128 st
 constexpr uint32_t SCOL = 256;   // S of stage st at SCOL + 64 st
+constexpr uint32_t QCOL = 384;   // query rows of stage sq at QCOL + 64 sq (bf16 pairs)
 constexpr int KMAX = 64;
 
 struct __align__(1024) SmemC {
-  unsigned char q[NQS][2][QHALF];   // [d half][row][128 B], 128-byte swizzle
   unsigned char k[NKV][2][BOX];     // [d half][key][128 B]
   unsigned char v[NKV][2][BOX];     // [d half][key][128 B]
-  unsigned char p[NST][MR * 128];   // [row][64 keys x bf16]
   uint64_t qfull[NQS], qempty[NQS], kvfull[NKV], kvempty[NKV];
-  uint64_t sfull[NST], sfree[NST], pfull[NST], pempty[NST], ofull[NST], ofree[NST], done;
+  uint64_t sfull[NST], sfree[NST], pfull[NST], ofull[NST], ofree[NST], done;
   uint32_t tmem;
 };
 constexpr size_t kSmemBytes = sizeof(SmemC) + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
-HILS_DI void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+HILS_DI void ldg32(const void* p, uint32_t (&w)[8]) {
+  asm volatile("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+               : "l"(p));
 }
-HILS_DI void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-HILS_DI void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-HILS_DI void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+// 32 lanes x 16 consecutive 32-bit columns <- 16 registers per thread
+HILS_DI void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
 }
 // Shared-memory descriptor of an MN-major operand with the 128-byte swizzle:
 // 64 MN-elements per 128-byte row, rows of consecutive K 128 B apart in
@@ -107,8 +126,8 @@ struct Item {
 
 __global__ void __launch_bounds__(THREADS, 1)
     attn_chunk_kernel(Shape s, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
-                      const __nv_bfloat16* __restrict__ q, const int* __restrict__ off, const int* __restrict__ ioff,
-                      const int2* __restrict__ items, const int* __restrict__ ent, int t0, int PT,
+                      const __nv_bfloat16* __restrict__ q, const int* __restrict__ ioff,
+                      const int4* __restrict__ items, const int* __restrict__ ent, int t0, int PT,
                       __nv_bfloat16* __restrict__ part, DevCtx ctx) {
   extern __shared__ unsigned char smem_raw[];
   SmemC& sm = *reinterpret_cast<SmemC*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -117,19 +136,22 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int nitems = __ldg(ioff + U);
   const int bid = blockIdx.x, nb = gridDim.x;
   const int nmine = nitems > bid ? (nitems - 1 - bid) / nb + 1 : 0;
+  // item record: bucket u = bg * C + c, first pair s0, pair count n (<= 32)
   auto item_of = [&](int it) -> Item {
-    const int2 e = __ldg(items + bid + it * nb);
-    Item r;
-    r.bg = e.x / s.C;
-    r.c = e.x - r.bg * s.C;
-    r.s0 = e.y;
-    r.n = min(PPI, __ldg(off + e.x + 1) - e.y);
+    Item r{0, 0, 0, 0};
+    if (it < nmine) {
+      const int4 e = __ldg(items + bid + it * nb);
+      r.bg = e.x / s.C;
+      r.c = e.x - r.bg * s.C;
+      r.s0 = e.y;
+      r.n = e.z;
+    }
     return r;
   };
 
   if (tid == 0) {
     for (int x = 0; x < NQS; ++x) {
-      mbar_init(&sm.qfull[x], 128);
+      mbar_init(&sm.qfull[x], 4);
       mbar_init(&sm.qempty[x], 1);
     }
     for (int x = 0; x < NKV; ++x) {
@@ -138,16 +160,15 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int x = 0; x < NST; ++x) {
       mbar_init(&sm.sfull[x], 1);
-      mbar_init(&sm.sfree[x], 4);
+      mbar_init(&sm.sfree[x], 1);
       mbar_init(&sm.pfull[x], 4);
-      mbar_init(&sm.pempty[x], 1);
       mbar_init(&sm.ofull[x], 1);
       mbar_init(&sm.ofree[x], 4);
     }
     mbar_init(&sm.done, 1);
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == 1) {
     tmem_alloc(&sm.tmem, TMEM_COLS);
     tmem_relinquish();
   }
@@ -156,48 +177,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem;
 
-  if (warp < 4) {
-    // ------------------------------------------------- query-row gather ----
-    // copy x of 16: row 8x + t/16, 16-byte unit t%16 of its 256-byte q row
-    const int t = tid;
-    const int unit = t & 15, half = unit >> 3, u8 = unit & 7;
-    bool ok = true;
-    int it = 0;
-    for (; it < nmine; ++it) {
-      const int sq = it % NQS;
-      if (it >= NQS) ok = mbar_wait(&sm.qempty[sq], ((it / NQS) - 1) & 1, ctx);
-      if (!__all_sync(0xffffffffu, ok)) {
-        ok = false;
-        break;
-      }
-      const Item im = item_of(it);
-      const int e = lane < im.n ? __ldg(ent + im.s0 + lane) : 0;
-      const int b = im.bg / s.Hkv, g = im.bg - b * s.Hkv;
-      const __nv_bfloat16* qb = q + ((long long)(b * s.Hq + g * G) * s.N + t0) * D + unit * 8;
-      const uint32_t qs = smem_u32(sm.q[sq][half]);
-#pragma unroll 4
-      for (int x = 0; x < 16; ++x) {
-        const int row = 8 * x + (t >> 4);
-        const int j = row >> 2, h = row & 3;
-        const int ej = __shfl_sync(0xffffffffu, e, j);
-        const bool v = j < im.n;
-        const __nv_bfloat16* src = v ? qb + ((long long)h * s.N + (ej >> 6)) * D : q;
-        cp_async16(qs + row * 128 + ((u8 ^ (row & 7)) << 4), src, v ? 16u : 0u);
-      }
-      cp_async_commit();
-      if (it > 0) {
-        // the previous item's rows have landed: publish them to the tensor core
-        cp_async_wait<1>();
-        fence_proxy_async_shared();
-        mbar_arrive(&sm.qfull[(it - 1) % NQS]);
-      }
-    }
-    cp_async_wait<0>();
-    if (ok && it > 0) {
-      fence_proxy_async_shared();
-      mbar_arrive(&sm.qfull[(it - 1) % NQS]);
-    }
-  } else if (warp == 4) {
+  if (warp == 0) {
     // --------------------------------------------------------- K/V loads ----
     if (lane == 0) {
       bool ok = true;
@@ -206,11 +186,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         prefetch_tmap(&tmk);
         prefetch_tmap(&tmv);
       }
+      Item nx = item_of(0);
       for (; it < nmine; ++it) {
         const int sk = it % NKV;
+        const Item im = nx;
+        nx = item_of(it + 1);
         if (it >= NKV) ok = mbar_wait(&sm.kvempty[sk], ((it / NKV) - 1) & 1, ctx);
         if (!ok) break;
-        const Item im = item_of(it);
         if (ctx.inject != 1) {
           mbar_arrive_expect_tx(&sm.kvfull[sk], 4 * BOX);
           tma_load_3d(sm.k[sk][0], &tmk, 0, im.c * S, im.bg, &sm.kvfull[sk]);
@@ -224,7 +206,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int j = max(0, it - NKV); j < it; ++j) mbar_wait(&sm.kvfull[j % NKV], (j / NKV) & 1, ctx);
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 1) {
     // --------------------------------------------------------- MMA issue ----
     if (lane == 0) {
       const uint32_t id1 = idesc_bf16_f32(MR, S);
@@ -237,9 +219,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t a = sdesc_k_sw128(smem_u32(sm.q[sq][kk >> 2]) + (kk & 3) * 32);
           const uint64_t bd = sdesc_k_sw128(smem_u32(sm.k[sk][kk >> 2]) + (kk & 3) * 32);
-          mma_ss(tmem + SCOL + 64 * st, a, bd, id1, kk > 0 ? 1u : 0u);
+          mma_ts(tmem + SCOL + 64 * st, tmem + QCOL + 64 * sq + 8 * kk, bd, id1, kk > 0 ? 1u : 0u);
         }
         tc_commit(&sm.sfull[st]);
         tc_commit(&sm.qempty[sq]);
@@ -252,13 +233,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t a = sdesc_k_sw128(smem_u32(sm.p[st]) + kk * 32);
           const uint64_t bd = sdesc_mn_sw128(smem_u32(sm.v[sk][0]) + kk * 2048, BOX, 1024);
-          mma_ss(tmem + OCOL + 128 * st, a, bd, id2, kk > 0 ? 1u : 0u);
+          mma_ts(tmem + OCOL + 128 * st, tmem + SCOL + 64 * st + 8 * kk, bd, id2, kk > 0 ? 1u : 0u);
         }
         tc_commit(&sm.ofull[st]);
         tc_commit(&sm.kvempty[sk]);
-        tc_commit(&sm.pempty[st]);
+        tc_commit(&sm.sfree[st]);  // P (in the S columns) has been read
         return true;
       };
       // S of item j + 1 is computed while the softmax of item j runs
@@ -273,6 +253,49 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     __syncwarp();
   } else if (warp < 10) {
+    // -------------------------------------------------------- query rows ----
+    // Group wg (warps 2-5 or 6-9) takes items wg, wg + 2, ...; thread = TMEM
+    // lane = row r = 4 j + h: head h of the item's position j (rows past the
+    // item's count are zero).  The 256-byte row is loaded before the stage is
+    // known to be free, so the loads of one item overlap the wait for it.
+    // Item metadata: records two items ahead, entries one item ahead.
+    const int wg = (warp - 2) >> 2, qw = warp & 3, row = 32 * qw + lane, jr = row >> 2, h = row & 3;
+    const uint32_t lrow = (uint32_t)(32 * qw) << 16;
+    Item m0 = item_of(wg), m1 = item_of(wg + 2);
+    int e0 = jr < m0.n ? __ldg(ent + m0.s0 + jr) : 0;
+    for (int it = wg; it < nmine; it += 2) {
+      const int sq = it % NQS, li = it / NQS;
+      const bool valid = jr < m0.n;
+      const int b = m0.bg / s.Hkv, g = m0.bg - b * s.Hkv;
+      const __nv_bfloat16* src = q + ((long long)(b * s.Hq + g * G + h) * s.N + t0 + (e0 >> 6)) * D;
+      uint32_t w[64];
+#pragma unroll
+      for (int x = 0; x < 8; ++x) {
+        uint32_t t8[8];
+        if (valid) {
+          ldg32(src + 16 * x, t8);
+        } else {
+#pragma unroll
+          for (int y = 0; y < 8; ++y) t8[y] = 0u;
+        }
+#pragma unroll
+        for (int y = 0; y < 8; ++y) w[8 * x + y] = t8[y];
+      }
+      e0 = jr < m1.n ? __ldg(ent + m1.s0 + jr) : 0;
+      m0 = m1;
+      m1 = item_of(it + 4);
+      const bool ok = li == 0 || mbar_wait(&sm.qempty[sq], (li - 1) & 1, ctx);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      uint32_t* w0 = w;
+      tmem_st32(tmem + lrow + QCOL + 64 * sq, *reinterpret_cast<uint32_t(*)[32]>(w0));
+      tmem_st32(tmem + lrow + QCOL + 64 * sq + 32, *reinterpret_cast<uint32_t(*)[32]>(w0 + 32));
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.qfull[sq]);
+    }
+  } else if (warp < 14) {
     // ----------------------------------------------------------- softmax ----
     const int qw = warp & 3, row = 32 * qw + lane;
     const uint32_t lrow = (uint32_t)(32 * qw) << 16;
@@ -287,9 +310,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       tmem_ld32(tmem + lrow + SCOL + 64 * st, r0);
       tmem_ld32(tmem + lrow + SCOL + 64 * st + 32, r1);
       tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.sfree[st]);
       float mx = -INFINITY;
 #pragma unroll
       for (int j = 0; j < 32; ++j) mx = fmaxf(mx, fmaxf(__uint_as_float(r0[j]), __uint_as_float(r1[j])));
@@ -304,61 +324,58 @@ __global__ void __launch_bounds__(THREADS, 1)
         l += e0 + e1;
       }
       const float inv = 1.f / l;
-      if (it >= NST) ok = mbar_wait(&sm.pempty[st], ((it / NST) - 1) & 1, ctx);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      const uint32_t pb = smem_u32(sm.p[st]) + row * 128;
+      // P row: keys 2c, 2c + 1 in column c (bf16 pairs), over S's first 32
+      // columns; keys 0-31 (r0) and 32-63 (r1) in two 16-column stores
+      uint32_t pw[16];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        // 16-byte unit u = keys 8u .. 8u + 7
-        uint32_t w[4];
+      for (int c = 0; c < 16; ++c) pw[c] = pack_bf16x2(__uint_as_float(r0[2 * c]) * inv, __uint_as_float(r0[2 * c + 1]) * inv);
+      tmem_st16(tmem + lrow + SCOL + 64 * st, pw);
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          const int kx = 8 * u + 2 * x;
-          const float a = __uint_as_float(kx < 32 ? r0[kx] : r1[kx - 32]) * inv;
-          const float c = __uint_as_float(kx + 1 < 32 ? r0[kx + 1] : r1[kx + 1 - 32]) * inv;
-          w[x] = pack_bf16x2(a, c);
-        }
-        st_shared_v4(pb + ((u ^ (row & 7)) << 4), w[0], w[1], w[2], w[3]);
-      }
-      fence_proxy_async_shared();
+      for (int c = 0; c < 16; ++c) pw[c] = pack_bf16x2(__uint_as_float(r1[2 * c]) * inv, __uint_as_float(r1[2 * c + 1]) * inv);
+      tmem_st16(tmem + lrow + SCOL + 64 * st + 16, pw);
+      tmem_wait_st();
+      tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.pfull[st]);
     }
   } else {
     // ---------------------------------------------------------- epilogue ----
-    // Partial record of (position, slot k): [head][128] bf16, each head's 128
-    // values stored in four 32-value blocks; inside block a, element
-    // 4 r + t holds d = 32 a + r + 8 t (r = 0..7, t = 0..3), the order in
-    // which the window pass's MMA fragments consume them.
+    // Partial record of (position, slot k): [head][128] bf16; in a head's row,
+    // element 16 r + 4 a + t holds d = 32 a + r + 8 t (r = 0..7, a = 0..3,
+    // t = 0..3): the 32 bytes at 16 r are what one thread of the window
+    // pass's MMA fragments consumes.  Item metadata is fetched ahead.
     const int qw = warp & 3, row = 32 * qw + lane, jr = row >> 2, h = row & 3;
     const uint32_t lrow = (uint32_t)(32 * qw) << 16;
-    bool ok = true;
+    Item m0 = item_of(0), m1 = item_of(1);
+    int e0 = jr < m0.n ? __ldg(ent + m0.s0 + jr) : 0;
     for (int it = 0; it < nmine; ++it) {
       const int st = it % NST;
-      const Item im = item_of(it);
+      const Item im = m0;
+      const int e = e0;
+      e0 = jr < m1.n ? __ldg(ent + m1.s0 + jr) : 0;
+      m0 = m1;
+      m1 = item_of(it + 2);
       const bool valid = jr < im.n;
-      const int e = valid ? __ldg(ent + im.s0 + jr) : 0;
       __nv_bfloat16* dst = part + (((long long)im.bg * PT + (e >> 6)) * s.K + (e & 63)) * (G * D) + h * D;
-      ok = mbar_wait(&sm.ofull[st], (it / NST) & 1, ctx);
+      const bool ok = mbar_wait(&sm.ofull[st], (it / NST) & 1, ctx);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
 #pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        uint32_t v[32];
-        tmem_ld32(tmem + lrow + OCOL + 128 * st + 32 * a, v);
+      for (int pr = 0; pr < 2; ++pr) {
+        uint32_t v0[32], v1[32];
+        tmem_ld32(tmem + lrow + OCOL + 128 * st + 64 * pr, v0);
+        tmem_ld32(tmem + lrow + OCOL + 128 * st + 64 * pr + 32, v1);
         tmem_wait_ld();
-        uint32_t w[16];
-#pragma unroll
-        for (int x = 0; x < 16; ++x) {
-          const int d0 = (x >> 1) + 16 * (x & 1);
-          w[x] = pack_bf16x2(__uint_as_float(v[d0]), __uint_as_float(v[d0 + 8]));
-        }
         if (valid) {
-          uint4* o = reinterpret_cast<uint4*>(dst + 32 * a);
-          o[0] = make_uint4(w[0], w[1], w[2], w[3]);
-          o[1] = make_uint4(w[4], w[5], w[6], w[7]);
-          o[2] = make_uint4(w[8], w[9], w[10], w[11]);
-          o[3] = make_uint4(w[12], w[13], w[14], w[15]);
+#pragma unroll
+          for (int r = 0; r < 8; ++r) {
+            uint4 o;
+            o.x = pack_bf16x2(__uint_as_float(v0[r]), __uint_as_float(v0[r + 8]));
+            o.y = pack_bf16x2(__uint_as_float(v0[r + 16]), __uint_as_float(v0[r + 24]));
+            o.z = pack_bf16x2(__uint_as_float(v1[r]), __uint_as_float(v1[r + 8]));
+            o.w = pack_bf16x2(__uint_as_float(v1[r + 16]), __uint_as_float(v1[r + 24]));
+            *reinterpret_cast<uint4*>(dst + 16 * r + 8 * pr) = o;
+          }
         }
       }
       tc_fence_before();
@@ -370,7 +387,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) tmem_dealloc(tmem, TMEM_COLS);
+  if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
 }
 
 // ------------------------------------------------------------ bucketing ----
@@ -455,7 +472,7 @@ __global__ void __launch_bounds__(1024) bucket_scan_kernel(int U, int* __restric
 
 __global__ void bucket_scatter_kernel(Shape s, const int32_t* __restrict__ idx, int t0, int np,
                                       const int* __restrict__ off, const int* __restrict__ ioff, int* __restrict__ cur,
-                                      int* __restrict__ ent, int2* __restrict__ items) {
+                                      int* __restrict__ ent, int4* __restrict__ items) {
   const long long total = (long long)s.B * s.Hkv * np * s.K;
   for (long long x = blockIdx.x * (long long)blockDim.x + threadIdx.x; x < total; x += (long long)gridDim.x * blockDim.x) {
     int u, pl, k;
@@ -463,7 +480,8 @@ __global__ void bucket_scatter_kernel(Shape s, const int32_t* __restrict__ idx, 
     const int slot = atomicAdd(cur + u, 1);
     ent[slot] = (pl << 6) | k;
     const int rel = slot - __ldg(off + u);
-    if (rel % PPI == 0) items[__ldg(ioff + u) + rel / PPI] = make_int2(u, slot);
+    if (rel % PPI == 0)
+      items[__ldg(ioff + u) + rel / PPI] = make_int4(u, slot, min(PPI, __ldg(off + u + 1) - slot), 0);
   }
 }
 
@@ -500,7 +518,7 @@ ChunkWs chunk_ws(const Shape& s) {
   w.off = take((U + 1) * 4);
   w.ioff = take((U + 1) * 4);
   w.ent = take(pairs * 4);
-  w.items = take((pairs / PPI + U + 1) * 8);
+  w.items = take((pairs / PPI + U + 1) * 16);
   w.part = take(pairs * G * D * 2);
   w.total = o;
   return w;
@@ -523,7 +541,7 @@ cudaError_t launch_attn_prefill_chunked(const Shape& s, const void* q, const voi
   int* off = (int*)(W + w.off);
   int* ioff = (int*)(W + w.ioff);
   int* ent = (int*)(W + w.ent);
-  int2* items = (int2*)(W + w.items);
+  int4* items = (int4*)(W + w.items);
   __nv_bfloat16* part = (__nv_bfloat16*)(W + w.part);
   const int U = s.B * s.Hkv * s.C;
 
@@ -549,8 +567,8 @@ cudaError_t launch_attn_prefill_chunked(const Shape& s, const void* q, const voi
       bucket_count_kernel<<<grid, 256, 0, st>>>(s, idx, t0, np, cnt);
       bucket_scan_kernel<<<1, 1024, 0, st>>>(U, cnt, off, ioff);
       bucket_scatter_kernel<<<grid, 256, 0, st>>>(s, idx, t0, np, off, ioff, cnt, ent, items);
-      attn_chunk_kernel<<<sms, THREADS, kSmemBytes, st>>>(s, tmk, tmv, (const __nv_bfloat16*)q, off, ioff, items, ent,
-                                                          t0, w.PT, part, ctx);
+      attn_chunk_kernel<<<sms, THREADS, kSmemBytes, st>>>(s, tmk, tmv, (const __nv_bfloat16*)q, ioff, items, ent, t0,
+                                                          w.PT, part, ctx);
       e = cudaGetLastError();
       if (e != cudaSuccess) return e;
     }

@@ -72,6 +72,7 @@ constexpr int KMAX = 64;
 constexpr int MAXC = 8192;              // candidate chunks covered by the bitmap
 constexpr int MAXW = MAXC / 32;
 constexpr int MAXI = 2048;              // stream chunks per CTA (>= BP * KMAX + window)
+constexpr int MSL = 3;                  // partial-record slots loaded at a time
 
 struct __align__(1024) SmemR {
   unsigned char slot[NSI][2][BOX];
@@ -125,6 +126,7 @@ struct Walk {
   int slot0 = 0, slot1 = 0;  // positions in the two lists (s^ lookup)
 };
 
+template <bool PART>
 __global__ void __launch_bounds__(THREADS, 2)
     attn_ring_kernel(Shape s, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                      const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ idx,
@@ -185,7 +187,7 @@ __global__ void __launch_bounds__(THREADS, 2)
   // with partial records the selected chunks were attended elsewhere: the
   // lists are kept for the fusion at the end and the stream is the window only
   const int m0a = l0a, m0b = l0b, m1a = l1a, m1b = l1b;
-  if (part) l0a = l0b = l1a = l1b = -1;
+  if (PART) l0a = l0b = l1a = l1b = -1;
   if (warp < CW) {
     if (l0a >= 0 && l0a < lo) atomicOr(&sm.bits[l0a >> 5], 1u << (l0a & 31));
     if (l0b >= 0 && l0b < lo) atomicOr(&sm.bits[l0b >> 5], 1u << (l0b & 31));
@@ -484,32 +486,53 @@ __global__ void __launch_bounds__(THREADS, 2)
     }
 
     // ---- selected chunks from their partial records O_c (attn_chunk.cu):
-    // acc += e^{s^ - m} O_c, den += e^{s^ - m}.  Block a of a record's head row
-    // holds d = 32 a + r + 8 t at element 4 r + t, so the 8-byte word at
-    // 32 a + 4 gq is this thread's d = 16 (2a) + gq (+8) and 16 (2a + 1) + gq (+8).
-    if (part && ok) {
-      const __nv_bfloat16* rec = part + (((long long)bg * PT + (my_pos - t0)) * K) * (G * D) + 4 * gq;
-#pragma unroll 2
-      for (int x = 0; x < K; ++x) {
-        const int ca = entry(m0a, m0b, x), cb = entry(m1a, m1b, x);
-        if (my_valid && (my_q == 0 ? ca : cb) >= 0) {
+    // acc += e^{s^ - m} O_c, den += e^{s^ - m}.  In a record's head row the 32
+    // bytes at element 16 gq hold this thread's values, d = 32 a + gq + 8 t at
+    // element 16 gq + 4 a + t (a, t = 0..3), i.e. d = 16 mt + gq (+ 8) for
+    // mt = 2a + t/2.  MSL slots are loaded at a time (predicated, no branch)
+    // so that their HBM round trips overlap.
+    if (PART && ok) {
+      const __nv_bfloat16* rec = part + (((long long)bg * PT + (my_pos - t0)) * K) * (G * D) + 16 * gq;
+      for (int x0 = 0; x0 < K; x0 += MSL) {
+        uint4 w[MSL][2][2];
+        float wg[MSL][2];
+#pragma unroll
+        for (int j = 0; j < MSL; ++j) {
+          const int x = x0 + j;
+          const int ca = entry(m0a, m0b, x), cb = entry(m1a, m1b, x);
+          const bool v = my_valid && (my_q == 0 ? ca : cb) >= 0;
           const __nv_bfloat16* rx = rec + (long long)x * (G * D);
 #pragma unroll
           for (int r = 0; r < 2; ++r) {
-            const float wgt = exp2f(__ldg(ss0 + r * sstride + x) * kLog2e - m2[r]);
-            den[r] += wgt;
-            const __nv_bfloat16* rh = rx + (my_h + r) * D;
+            float sv = -INFINITY;
+            if (v) sv = __ldg(ss0 + r * sstride + x);
+            wg[j][r] = sv;
 #pragma unroll
-            for (int a = 0; a < 4; ++a) {
-              const uint2 u = __ldg(reinterpret_cast<const uint2*>(rh + 32 * a));
-              const float2 f0 = bf16x2_to_f32x2(u.x), f1 = bf16x2_to_f32x2(u.y);
-              acc[2 * a][r] = fmaf(wgt, f0.x, acc[2 * a][r]);
-              acc[2 * a][2 + r] = fmaf(wgt, f0.y, acc[2 * a][2 + r]);
-              acc[2 * a + 1][r] = fmaf(wgt, f1.x, acc[2 * a + 1][r]);
-              acc[2 * a + 1][2 + r] = fmaf(wgt, f1.y, acc[2 * a + 1][2 + r]);
+            for (int hh = 0; hh < 2; ++hh) {
+              uint4 u = make_uint4(0u, 0u, 0u, 0u);
+              if (v) u = __ldg(reinterpret_cast<const uint4*>(rx + (my_h + r) * D + 8 * hh));
+              w[j][r][hh] = u;
             }
           }
         }
+#pragma unroll
+        for (int j = 0; j < MSL; ++j)
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const float wgt = exp2f(wg[j][r] * kLog2e - m2[r]);  // 0 for skipped slots
+            den[r] += wgt;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const uint32_t ww[4] = {w[j][r][hh].x, w[j][r][hh].y, w[j][r][hh].z, w[j][r][hh].w};
+#pragma unroll
+              for (int q2 = 0; q2 < 4; ++q2) {  // a = 2 hh + q2 / 2, t pair = q2 % 2
+                const int a = 2 * hh + (q2 >> 1), mt = 2 * a + (q2 & 1);
+                const float2 f = bf16x2_to_f32x2(ww[q2]);
+                acc[mt][r] = fmaf(wgt, f.x, acc[mt][r]);
+                acc[mt][2 + r] = fmaf(wgt, f.y, acc[mt][2 + r]);
+              }
+            }
+          }
       }
     }
 
@@ -548,12 +571,12 @@ cudaError_t launch_attn_window_merge(const Shape& s, const void* q, const void* 
   if (e != cudaSuccess) return e;
   e = make_tmap_bf16(&tmv, v, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
-  e = ensure_dynamic_smem((const void*)attn_ring_kernel, (int)kSmemBytes);
+  auto kern = part ? attn_ring_kernel<true> : attn_ring_kernel<false>;
+  e = ensure_dynamic_smem((const void*)kern, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid((t1 - t0 + BP - 1) / BP, s.Hkv, s.B);
-  attn_ring_kernel<<<grid, THREADS, kSmemBytes, st>>>(s, tmk, tmv, (const __nv_bfloat16*)q, idx, s_sel,
-                                                      (__nv_bfloat16*)out, (const __nv_bfloat16*)part, t0, t1, PT,
-                                                      ctx);
+  kern<<<grid, THREADS, kSmemBytes, st>>>(s, tmk, tmv, (const __nv_bfloat16*)q, idx, s_sel, (__nv_bfloat16*)out,
+                                          (const __nv_bfloat16*)part, t0, t1, PT, ctx);
   return cudaGetLastError();
 }
 
