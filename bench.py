@@ -130,18 +130,26 @@ def decode_bytes(w):
     return score, gather, q_out
 
 
-def traffic_for(kernel_file: str, kernel: str, workload: str):
-    """DRAM bytes per launch from a committed ncu capture (profiles/traffic.json),
-    or None if absent or if the kernel's source changed since the capture."""
+def source_sha(kernel_files) -> str:
+    """Hash of the kernel sources a traffic figure was measured with."""
+    if isinstance(kernel_files, str):
+        kernel_files = [kernel_files]
+    h = hashlib.sha256()
+    for f in kernel_files:
+        h.update(open(os.path.join(ROOT, "chunk_wise_sparse_landmark_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel_files, kernel: str, workload: str):
+    """DRAM bytes per launch (or per call) from a committed ncu capture
+    (profiles/traffic.json), or None if absent or if a source changed since."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     try:
         d = json.load(open(p))
         e = d[kernel][workload]
-        src = os.path.join(ROOT, "chunk_wise_sparse_landmark_b200", "csrc", kernel_file)
-        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-        return e["bytes_per_launch"] if e.get("source_sha") == h else None
+        return e["bytes_per_launch"] if e.get("source_sha") == source_sha(kernel_files) else None
     except Exception:
         return None
 
@@ -365,7 +373,7 @@ def main():
                           f"{attn_tiles(w)} position tiles)",
                 "bound": "tensor", "achieved": round(ach, 2),
                 "peak": peak_tf, "unit": "TFLOP/s", "frac": round(ach / peak_tf, 4),
-                "traffic": traffic_for("attn_chunk.cu", "attn_chunk_kernel", w.name),
+                "traffic": traffic_for(["attn_chunk.cu", "attn_ring.cu"], "hils_attn_prefill", w.name),
                 "peak_source": f"{pk_kind} bf16_tflops_sustained",
                 "algorithmic_flop_per_launch": attn_f}
     per_kernel = {"summaries_ms": round(t_summ, 4), "score_topk_ms": round(t_score, 4),
