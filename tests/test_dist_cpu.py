@@ -54,3 +54,18 @@ def test_both_arms_share_the_config_object():
     w = bench.WORKLOADS["prefill_128k"]
     c = bench.run_config(w, 2)
     assert c["workload"] == "prefill_128k" and c["seq_len"] == 131072 and c["parallelism"] == "replica x2"
+
+
+def test_attention_tiles_and_traffic_lookup():
+    """Tile counts of the chunk-major attention (fewest tiles of <= 8 GiB of
+    1 KB records) and the traffic record, which is used only while the
+    measured kernel sources are unchanged."""
+    from chunk_wise_sparse_landmark_b200.inputs import WORKLOADS
+    assert bench.attn_tiles(WORKLOADS["prefill_128k"]) == 4
+    assert bench.attn_tiles(WORKLOADS["prefill_512k_qcal"]) == 32
+    assert bench.attn_tiles(WORKLOADS["prefill_8k"]) == 1
+    files = ["attn_chunk.cu", "attn_ring.cu"]
+    t = bench.traffic_for(files, "hils_attn_prefill", "prefill_128k")
+    assert t is None or t > 0
+    assert bench.traffic_for(["attn_chunk.cu"], "hils_attn_prefill", "prefill_128k") is None  # other sources
+    assert bench.traffic_for(files, "hils_attn_prefill", "no_such_workload") is None
