@@ -97,6 +97,12 @@ HILS_DI void ldg32(const void* p, uint32_t (&w)[8]) {
                : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
                : "l"(p));
 }
+// 32-byte global store (address 32-byte aligned)
+HILS_DI void stg32(void* p, const uint32_t (&w)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+               "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
 // 32 lanes x 16 consecutive 32-bit columns <- 16 registers per thread
 HILS_DI void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
@@ -341,9 +347,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else {
     // ---------------------------------------------------------- epilogue ----
     // Partial record of (position, slot k): [head][128] bf16; in a head's row,
-    // element 16 r + 4 a + t holds d = 32 a + r + 8 t (r = 0..7, a = 0..3,
-    // t = 0..3): the 32 bytes at 16 r are what one thread of the window
-    // pass's MMA fragments consumes.  Item metadata is fetched ahead.
+    // element 64 h2 + 8 r + 4 a + t holds d = 64 h2 + 32 a + r + 8 t (h2, a =
+    // 0..1, r = 0..7, t = 0..3).  Each 64-column half of the TMEM row is one
+    // contiguous 128-byte run written with 32-byte stores (measured: records
+    // written as 16-byte halves of sectors from separate passes cost ~13 ms of
+    // the 128K attention), and the 16 bytes at 64 h2 + 8 r are what one thread
+    // of the window pass's MMA fragments consumes.  Item metadata is fetched ahead.
     const int qw = warp & 3, row = 32 * qw + lane, jr = row >> 2, h = row & 3;
     const uint32_t lrow = (uint32_t)(32 * qw) << 16;
     Item m0 = item_of(0), m1 = item_of(1);
@@ -368,13 +377,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_wait_ld();
         if (valid) {
 #pragma unroll
-          for (int r = 0; r < 8; ++r) {
-            uint4 o;
-            o.x = pack_bf16x2(__uint_as_float(v0[r]), __uint_as_float(v0[r + 8]));
-            o.y = pack_bf16x2(__uint_as_float(v0[r + 16]), __uint_as_float(v0[r + 24]));
-            o.z = pack_bf16x2(__uint_as_float(v1[r]), __uint_as_float(v1[r + 8]));
-            o.w = pack_bf16x2(__uint_as_float(v1[r + 16]), __uint_as_float(v1[r + 24]));
-            *reinterpret_cast<uint4*>(dst + 16 * r + 8 * pr) = o;
+          for (int r = 0; r < 8; r += 2) {
+            uint32_t o[8];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              o[4 * u + 0] = pack_bf16x2(__uint_as_float(v0[r + u]), __uint_as_float(v0[r + u + 8]));
+              o[4 * u + 1] = pack_bf16x2(__uint_as_float(v0[r + u + 16]), __uint_as_float(v0[r + u + 24]));
+              o[4 * u + 2] = pack_bf16x2(__uint_as_float(v1[r + u]), __uint_as_float(v1[r + u + 8]));
+              o[4 * u + 3] = pack_bf16x2(__uint_as_float(v1[r + u + 16]), __uint_as_float(v1[r + u + 24]));
+            }
+            stg32(dst + 64 * pr + 8 * r, o);
           }
         }
       }

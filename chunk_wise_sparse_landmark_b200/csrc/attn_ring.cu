@@ -486,13 +486,13 @@ __global__ void __launch_bounds__(THREADS, 2)
     }
 
     // ---- selected chunks from their partial records O_c (attn_chunk.cu):
-    // acc += e^{s^ - m} O_c, den += e^{s^ - m}.  In a record's head row the 32
-    // bytes at element 16 gq hold this thread's values, d = 32 a + gq + 8 t at
-    // element 16 gq + 4 a + t (a, t = 0..3), i.e. d = 16 mt + gq (+ 8) for
-    // mt = 2a + t/2.  MSL slots are loaded at a time (predicated, no branch)
+    // acc += e^{s^ - m} O_c, den += e^{s^ - m}.  In a record's head row the 16
+    // bytes at element 64 hh + 8 gq (hh = 0, 1) hold this thread's values
+    // d = 64 hh + 32 a + gq + 8 t at element 64 hh + 8 gq + 4 a + t (a = 0..1,
+    // t = 0..3), i.e. d = 16 mt + gq (+ 8) for mt = 4 hh + 2 a + t/2.  MSL slots are loaded at a time (predicated, no branch)
     // so that their HBM round trips overlap.
     if (PART && ok) {
-      const __nv_bfloat16* rec = part + (((long long)bg * PT + (my_pos - t0)) * K) * (G * D) + 16 * gq;
+      const __nv_bfloat16* rec = part + (((long long)bg * PT + (my_pos - t0)) * K) * (G * D) + 8 * gq;
       for (int x0 = 0; x0 < K; x0 += MSL) {
         uint4 w[MSL][2][2];
         float wg[MSL][2];
@@ -510,7 +510,7 @@ __global__ void __launch_bounds__(THREADS, 2)
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
               uint4 u = make_uint4(0u, 0u, 0u, 0u);
-              if (v) u = __ldg(reinterpret_cast<const uint4*>(rx + (my_h + r) * D + 8 * hh));
+              if (v) u = __ldg(reinterpret_cast<const uint4*>(rx + (my_h + r) * D + 64 * hh));
               w[j][r][hh] = u;
             }
           }
@@ -525,8 +525,8 @@ __global__ void __launch_bounds__(THREADS, 2)
             for (int hh = 0; hh < 2; ++hh) {
               const uint32_t ww[4] = {w[j][r][hh].x, w[j][r][hh].y, w[j][r][hh].z, w[j][r][hh].w};
 #pragma unroll
-              for (int q2 = 0; q2 < 4; ++q2) {  // a = 2 hh + q2 / 2, t pair = q2 % 2
-                const int a = 2 * hh + (q2 >> 1), mt = 2 * a + (q2 & 1);
+              for (int q2 = 0; q2 < 4; ++q2) {  // a = q2 / 2, t pair = q2 % 2
+                const int mt = 4 * hh + q2;
                 const float2 f = bf16x2_to_f32x2(ww[q2]);
                 acc[mt][r] = fmaf(wgt, f.x, acc[mt][r]);
                 acc[mt][2 + r] = fmaf(wgt, f.y, acc[mt][2 + r]);
