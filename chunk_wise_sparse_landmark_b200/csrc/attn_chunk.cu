@@ -49,17 +49,18 @@
 // 18 warps: the register file is split across the four sub-partitions, so
 // 96 registers per thread is the most that fits.
 //
-// Measured on B200 (clock stamps per role, 128K workload): every role runs at
-// the same period of ~5.5K cycles per item.  Staging the gathered rows in
-// shared memory with 16-byte cp.async held only ~20 KB in flight per SM and
-// set that period; with 32-byte loads into registers and P in TMEM the
-// gather and the softmax take ~3K cycles each and the period is set by the
-// tensor pipe (issue to completion: ~2.3K cycles for the 8 MMAs of S, ~6K for
-// the 4 of O behind them), far above the ~130 cycles per instruction that one
-// issuing thread reaches alone.  Copy-engine gathers issued from all lanes of
-// a warp (one tile::gather4 or one 256-byte bulk copy per row) did not
-// complete on B200 and are not used.  Every wait is bounded (status word +
-// early return), see common.cuh.
+// Measured on B200 at 128K:
+//   - Staging the gathered rows in shared memory with 16-byte cp.async held
+//     only ~20 KB in flight per SM and set a period of ~5K cycles per item;
+//     32-byte loads into registers keep far more in flight.
+//   - A build that skipped the record stores ran 13 ms faster (36.1 -> 23.2 ms
+//     for the attention call) while the records were written as 16-byte halves
+//     of sectors from separate passes.  Writing each 64-column half of a row as
+//     one contiguous 128-byte run took the attention to 30.9 ms.
+//   - A second MMA-issuing thread changed nothing measurable.
+//   - Copy-engine gathers issued from all lanes of a warp (one tile::gather4 or
+//     one 256-byte bulk copy per row) did not complete, and are not used.
+// Every wait is bounded (status word + early return), see common.cuh.
 #include <algorithm>
 
 #include "launch.h"
