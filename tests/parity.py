@@ -17,11 +17,16 @@ import numpy as np
 EPS_SEL = 1e-2
 TOL_F32 = 1e-5
 TOL_BF16 = 1.5e-2
-# k' (bf16 runs): one bf16 rounding of the stored value (2^-8 relative) plus the
-# fp32 accumulation error of the tensor-core weighted sum of the chunk's 64 keys
-# (absolute, below 1e-4 for |k| of order 1).  Its effect on s^ is ~1e-4, far below
-# the 1e-2 selection gap.
-KSUM_ATOL = 1e-4
+# k' (bf16 runs): one bf16 rounding of the stored value (|k'| 2^-8 relative), plus
+# an absolute term.  The summary kernel splits each softmax weight p into a bf16
+# high part ph = bf16(p) and a low part p - ph, which the bf16 MMA rounds again:
+# |p - ph| <= 2^-8 p, so each weight enters with error <= 2^-16 p, and the
+# weighted key sum with error <= 2^-16 * max|k| (the weights sum to 1).  The
+# fp32 accumulation of the 64 products adds at most 63 * 2^-24 * max|k|.  The
+# largest |k| of the biggest workload (8.6e9 N(0,1) draws) is about 6.5, so the
+# two give 9.9e-5 + 2.4e-5 < 1.25e-4.  Its effect on s^ is ~1e-4, far below the
+# 1e-2 selection gap.
+KSUM_ATOL = 1.25e-4
 
 
 def to_np(t):

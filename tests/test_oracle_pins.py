@@ -290,6 +290,26 @@ def test_qcal_identity_projection(oracle_mod):
     np.testing.assert_allclose(qs, want, rtol=0, atol=1e-12)
 
 
+def test_golden_qcal_layout(oracle_mod):
+    """Hand-derived Q-Cal rows with non-square, non-symmetric W_down / W_up
+    (tests/golden): a transposed read of either matrix, a swapped head/dim
+    reshape or a wrong hidden-state row gives another answer."""
+    from oracle import Dims
+
+    g = json.load(open(GOLDEN))["qcal_layout"]
+    Hq, d = g["Hq"], g["d"]
+    dm = Dims(B=1, Hq=Hq, Hkv=1, N=2, d=d, S=1, W=1, K=1)
+    q = np.full((1, Hq, 2, d), g["q_value"], np.float32)
+    h = np.array(g["h"], np.float32).reshape(1, 2, g["d_model"])
+    wd = np.array(g["w_down"], np.float32)
+    wu = np.array(g["w_up"], np.float32)
+    assert wd.shape == (g["r"], g["d_model"]) and wu.shape == (Hq * d, g["r"])
+    qs = oracle_mod.qcal(dm, [(0, 0), (0, 1)], q, h, wd, wu)
+    for n, key in enumerate(("q_tilde_pos0", "q_tilde_pos1")):
+        want = np.array([[_ev(e) for e in row] for row in g["expected"][key]])
+        np.testing.assert_array_equal(qs[n], want)
+
+
 def test_P11_single_head_groups_select_by_sort(oracle_mod):
     from oracle import Dims
 
