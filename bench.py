@@ -130,6 +130,52 @@ def decode_bytes(w):
     return score, gather, q_out
 
 
+def attention_stats(w, idx):
+    """Executed work of the chunk-major attention, and the reuse measure of
+    grouping adjacent queries, from the selection the step produced.
+
+    * pairs: (position, KV group, selected chunk) triples; each is 4 heads x
+      (2 d S + 2 S d) FLOP of algorithmic selected-chunk work.
+    * items: per position tile and bucket (sequence, group, chunk), ceil(n/32)
+      items of 128 query rows; each executes 128 rows x 4 d S FLOP on tcgen05.
+    * window: each warp of the window pass covers 2 positions x 4 heads (8
+      rows) against every window chunk of its position pair (64 keys each,
+      causal keys masked inside the current chunk), 8 x 4 d S FLOP per chunk.
+    * union_over_k_m4: mean size of the union of the chunk sets of M = 4
+      adjacent positions divided by K (rows with full lists), the reuse measure
+      of grouping adjacent queries.
+    Counting runs on the GPU with torch after the timed region (measurement
+    only, not part of the path)."""
+    B, Hkv, N, K = idx.shape
+    S, nw, d = w.S, w.W // w.S, w.d
+    C = N // S
+    PT = attn_tile_positions(w)
+    valid = idx >= 0
+    pairs = int(valid.sum().item())
+    items = 0
+    for t0 in range(0, N, PT):
+        sl = idx[:, :, t0:t0 + PT]
+        bg = torch.arange(B * Hkv, device=idx.device).view(B, Hkv, 1, 1).expand_as(sl)
+        u = (bg * C + sl.clamp(min=0))[sl >= 0]
+        cnt = torch.bincount(u.long(), minlength=B * Hkv * C)
+        items += int(((cnt + 31) // 32).sum().item())
+    win_chunks = 0
+    for p0 in range(0, N, 2):
+        cur = p0 // S
+        win_chunks += cur - max(0, cur - nw + 1) + 1
+    exec_chunk = items * 128 * 4 * d * S
+    exec_win = B * Hkv * win_chunks * 8 * 4 * d * S
+    M = 4
+    nb = N // M
+    blk = idx[:, :, : nb * M].reshape(B, Hkv, nb, M * K)
+    full = (idx[:, :, : nb * M] >= 0).sum(-1).reshape(B, Hkv, nb, M).min(-1).values == K
+    srt, _ = torch.sort(blk, dim=-1)
+    distinct = ((srt[..., 1:] != srt[..., :-1]) & (srt[..., 1:] >= 0)).sum(-1) + (srt[..., 0] >= 0).long()
+    union_k = float((distinct[full].float() / K).mean().item()) if bool(full.any()) else None
+    return {"pairs": pairs, "items": items, "item_fill": round(pairs / max(1, 32 * items), 4),
+            "executed_flop_per_launch": exec_chunk + exec_win, "union_over_k_m4": union_k}
+
+
 def source_sha(kernel_files) -> str:
     """Hash of the kernel sources a traffic figure was measured with."""
     if isinstance(kernel_files, str):
@@ -317,6 +363,61 @@ def cpu_baseline_prefill(w, x, budget_s=15.0, rows=None, seed=0):
     return 1.0 / per_token, done, t_summ, t_rows
 
 
+def prefill_launches(w) -> int:
+    """Kernels one prefill step launches: summaries, [Q-Cal,] scoring, and per
+    attention position tile bucket count, scan, scatter, the chunk-major pass
+    and the window pass."""
+    return 2 + (1 if w.d_model else 0) + 5 * attn_tiles(w)
+
+
+def prefill_roofline(w, pre, ev, pk, pk_kind):
+    """Roofline of the dominant call (hils_attn_prefill) and per-kernel times of
+    a timed prefill run; the executed-work statistics come from its selection."""
+    score_f, attn_f = prefill_flops(w)
+    t_attn = mean_ms(ev["attn_prefill"])
+    t_score = mean_ms(ev["score_topk"])
+    t_summ = mean_ms(ev["summaries"])
+    peak_tf = pk["bf16_tflops_sustained"]
+    ach = attn_f / (t_attn / 1e3) / 1e12
+    st = attention_stats(w, pre.idx)
+    roofline = {"kernel": f"hils_attn_prefill (attn_chunk_kernel + attn_ring_kernel<1> + bucketing, "
+                          f"{attn_tiles(w)} position tiles)",
+                "bound": "tensor", "achieved": round(ach, 2),
+                "peak": peak_tf, "unit": "TFLOP/s", "frac": round(ach / peak_tf, 4),
+                "traffic": traffic_for(["attn_chunk.cu", "attn_ring.cu", "common.cuh"], "hils_attn_prefill", w.name),
+                "peak_source": f"{pk_kind} bf16_tflops_sustained",
+                "algorithmic_flop_per_launch": attn_f,
+                "executed_flop_per_launch": st["executed_flop_per_launch"],
+                "executed_tflops": round(st["executed_flop_per_launch"] / (t_attn / 1e3) / 1e12, 2),
+                "union_over_k_m4": st["union_over_k_m4"], "pairs": st["pairs"], "items": st["items"],
+                "item_fill": st["item_fill"]}
+    per_kernel = {"summaries_ms": round(t_summ, 4), "score_topk_ms": round(t_score, 4),
+                  "attn_prefill_ms": round(t_attn, 4),
+                  "score_tflops_alg": round(score_f / (t_score / 1e3) / 1e12, 2),
+                  "score_frac": round(score_f / (t_score / 1e3) / 1e12 / peak_tf, 4)}
+    return roofline, per_kernel
+
+
+def extra_prefill(w, dev, stream, args, ws, dist_on, pk, pk_kind):
+    """Another prefill workload timed the same way (device-resident inputs,
+    W >= 3 warm-up steps, K timed steps between CUDA events, max over ranks),
+    reported beside the main line."""
+    steps = max(3, args.steps // 2)
+    x, pre, step, ev = run_prefill(w, dev, steps, args.warmup, stream)
+    with Clocks(int(os.environ.get("LOCAL_RANK", "0"))) as clk:
+        ms_total = device_time(stream, lambda: step(True), steps, dist_on)
+    H.hils_sync_status(stream)
+    ms_step = ms_total / steps
+    roofline, per_kernel = prefill_roofline(w, pre, ev, pk, pk_kind)
+    out = {"workload": w.name, "value": round(whole_job_rate(w.B * w.N, ws, ms_step), 1), "unit": "tokens/s",
+           "ms_per_step": round(ms_step, 3), "steps": steps, "warmup": args.warmup, "config": run_config(w, ws),
+           "roofline": roofline, "kernels": per_kernel, "clocks": clk.summary(),
+           "gpu_launches": prefill_launches(w) * steps}
+    del x, pre
+    torch.cuda.empty_cache()
+    return out
+
+
 # ------------------------------------------------------------------ main -----
 
 def main():
@@ -330,6 +431,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-qcal", action="store_true", help="skip the 512K Q-Cal prefill reported beside the line")
     ap.add_argument("--seq-len", type=int, default=0, help="override N of the prefill workload (profiling)")
     ap.add_argument("--decode-seq-len", type=int, default=0, help="override L of the decode workload (profiling)")
     args = ap.parse_args()
@@ -361,30 +463,13 @@ def main():
     ms_step = ms_total / args.steps
     tokens = w.B * w.N * ws
     value = whole_job_rate(w.B * w.N, ws, ms_step)
-    score_f, attn_f = prefill_flops(w)
-    t_attn = mean_ms(ev["attn_prefill"])
-    t_score = mean_ms(ev["score_topk"])
-    t_summ = mean_ms(ev["summaries"])
-    peak_tf = pk["bf16_tflops_sustained"]
-    ach = attn_f / (t_attn / 1e3) / 1e12
-    # the attention call: per position tile, bucketing (3 small kernels), the
-    # chunk-major tcgen05 kernel and the window pass; timed as one call
-    roofline = {"kernel": f"hils_attn_prefill (attn_chunk_kernel + attn_ring_kernel<1> + bucketing, "
-                          f"{attn_tiles(w)} position tiles)",
-                "bound": "tensor", "achieved": round(ach, 2),
-                "peak": peak_tf, "unit": "TFLOP/s", "frac": round(ach / peak_tf, 4),
-                "traffic": traffic_for(["attn_chunk.cu", "attn_ring.cu"], "hils_attn_prefill", w.name),
-                "peak_source": f"{pk_kind} bf16_tflops_sustained",
-                "algorithmic_flop_per_launch": attn_f}
-    per_kernel = {"summaries_ms": round(t_summ, 4), "score_topk_ms": round(t_score, 4),
-                  "attn_prefill_ms": round(t_attn, 4),
-                  "score_tflops_alg": round(score_f / (t_score / 1e3) / 1e12, 2)}
+    roofline, per_kernel = prefill_roofline(w, pre, ev, pk, pk_kind)
     line = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": run_config(w, ws),
             "roofline": roofline, "kernels": per_kernel, "clocks": clocks,
-            "gpu_launches": (2 + (1 if w.d_model else 0) + 5 * attn_tiles(w)) * args.steps}
+            "gpu_launches": prefill_launches(w) * args.steps}
     if not args.no_e2e:
         e2e_ms, h2d, d2h = e2e_prefill(w, x, pre, stream, max(2, args.steps // 3), dist_on)
         line["e2e"] = {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
@@ -417,6 +502,9 @@ def main():
                                    / (summ_ms / 1e3) / 1e9, 1),
             "gpu_launches": 4 * args.steps * 5}
         del xd, dec
+    if not args.no_qcal and args.workload != "prefill_512k_qcal" and not args.seq_len:
+        line["prefill_512k_qcal"] = extra_prefill(WORKLOADS["prefill_512k_qcal"], dev, stream, args, ws, dist_on, pk,
+                                                  pk_kind)
     if rank == 0 and not args.no_cpu:
         v, done, t_s, t_r = cpu_baseline_prefill(w, x)
         line["cpu_baseline"] = {"value": round(v, 2), "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
@@ -440,6 +528,13 @@ def attn_tiles(w) -> int:
     return (w.N + cap - 1) // cap
 
 
+def attn_tile_positions(w) -> int:
+    """Positions per tile: N split evenly over the tiles, rounded up to 14."""
+    nt = attn_tiles(w)
+    pt = -(-w.N // nt)
+    return -(-pt // 14) * 14
+
+
 def run_config(w, ws):
     """The `config` object of both arms' JSON lines."""
     return {"workload": w.name, "batch": w.B, "seq_len": w.N, "n_q_heads": w.Hq, "n_kv_heads": w.Hkv,
@@ -455,18 +550,20 @@ def reference_arm(args, ws, rank):
         return
     w = WORKLOADS[args.workload]
     x = prefill_inputs(w, device="cuda" if torch.cuda.is_available() else "cpu")
+    # every host core gets rows: the oracle spreads positions over its threads
+    nrows = max(16, 2 * (os.cpu_count() or 8))
     vals = []
     for it in range(args.warmup + args.steps):
-        v, done, _, _ = cpu_baseline_prefill(w, x, rows=8, seed=it)
+        v, done, _, _ = cpu_baseline_prefill(w, x, rows=nrows, seed=it)
         if it >= args.warmup:
             vals.append(v)
     v = statistics.mean(vals)
     line = {"impl": "reference", "metric": METRIC, "value": round(v, 2), "unit": "tokens/s", "n_gpus": ws,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * 8 / v, 2),
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * nrows / v, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": run_config(w, ws),
             "cpu_baseline": {"value": round(v, 2), "unit": "tokens/s", "kind": "oracle", "cores": os.cpu_count(),
-                             "sample": f"8 random positions of {w.name} per step, all heads"},
+                             "sample": f"{nrows} random positions of {w.name} per step, all heads"},
             "e2e": {"value": round(v, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 

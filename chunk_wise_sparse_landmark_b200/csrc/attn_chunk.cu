@@ -404,25 +404,34 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 // ------------------------------------------------------------ bucketing ----
-// The pairs of a position tile [t0, t0 + np): entry x = ((bg * np + pl) * K + k).
-HILS_DI bool pair_of(const Shape& s, const int32_t* __restrict__ idx, int t0, int np, long long x, int& u, int& pl,
-                     int& k) {
-  k = (int)(x % s.K);
-  const long long r = x / s.K;
+// The lists of a position tile [t0, t0 + np): list r = bg * np + pl holds the
+// K entries of position t0 + pl in KV group bg.  One warp reads one list
+// (lane j: entries j and j + 32) and keeps the entries that have the list
+// form (accept_list_warp, common.cuh); the window pass applies the same rule
+// before it fuses the records, so both agree on every pair.
+HILS_DI void list_of(const Shape& s, const int32_t* __restrict__ idx, int t0, int np, long long r, int& bg, int& pl,
+                     int& a, int& b, const DevCtx* report) {
+  const int lane = threadIdx.x & 31;
   pl = (int)(r % np);
-  const int bg = (int)(r / np);
+  bg = (int)(r / np);
   const int p = t0 + pl;
-  const int c = __ldg(idx + ((long long)bg * s.N + p) * s.K + k);
-  const int ncand = max(0, p / S - s.nw + 1);
-  u = bg * s.C + c;
-  return c >= 0 && c < ncand;
+  const int32_t* L = idx + ((long long)bg * s.N + p) * s.K;
+  a = lane < s.K ? __ldg(L + lane) : -1;
+  b = lane + 32 < s.K ? __ldg(L + lane + 32) : -1;
+  bool bad;
+  accept_list_warp(a, b, s.K, max(0, p / S - s.nw + 1), bad);
+  if (report && bad && lane == 0) raise_status(*report, kStatusBadIndex);
 }
 
-__global__ void bucket_count_kernel(Shape s, const int32_t* __restrict__ idx, int t0, int np, int* __restrict__ cnt) {
-  const long long total = (long long)s.B * s.Hkv * np * s.K;
-  for (long long x = blockIdx.x * (long long)blockDim.x + threadIdx.x; x < total; x += (long long)gridDim.x * blockDim.x) {
-    int u, pl, k;
-    if (pair_of(s, idx, t0, np, x, u, pl, k)) atomicAdd(cnt + u, 1);
+__global__ void bucket_count_kernel(Shape s, const int32_t* __restrict__ idx, int t0, int np, int* __restrict__ cnt,
+                                    DevCtx ctx) {
+  const long long lists = (long long)s.B * s.Hkv * np;
+  const long long wpb = blockDim.x >> 5;
+  for (long long r = blockIdx.x * wpb + (threadIdx.x >> 5); r < lists; r += (long long)gridDim.x * wpb) {
+    int bg, pl, a, b;
+    list_of(s, idx, t0, np, r, bg, pl, a, b, &ctx);
+    if (a >= 0) atomicAdd(cnt + bg * s.C + a, 1);
+    if (b >= 0) atomicAdd(cnt + bg * s.C + b, 1);
   }
 }
 
@@ -486,15 +495,23 @@ __global__ void __launch_bounds__(1024) bucket_scan_kernel(int U, int* __restric
 __global__ void bucket_scatter_kernel(Shape s, const int32_t* __restrict__ idx, int t0, int np,
                                       const int* __restrict__ off, const int* __restrict__ ioff, int* __restrict__ cur,
                                       int* __restrict__ ent, int4* __restrict__ items) {
-  const long long total = (long long)s.B * s.Hkv * np * s.K;
-  for (long long x = blockIdx.x * (long long)blockDim.x + threadIdx.x; x < total; x += (long long)gridDim.x * blockDim.x) {
-    int u, pl, k;
-    if (!pair_of(s, idx, t0, np, x, u, pl, k)) continue;
-    const int slot = atomicAdd(cur + u, 1);
-    ent[slot] = (pl << 6) | k;
-    const int rel = slot - __ldg(off + u);
-    if (rel % PPI == 0)
-      items[__ldg(ioff + u) + rel / PPI] = make_int4(u, slot, min(PPI, __ldg(off + u + 1) - slot), 0);
+  const long long lists = (long long)s.B * s.Hkv * np;
+  const long long wpb = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31;
+  for (long long r = blockIdx.x * wpb + (threadIdx.x >> 5); r < lists; r += (long long)gridDim.x * wpb) {
+    int bg, pl, a, b;
+    list_of(s, idx, t0, np, r, bg, pl, a, b, nullptr);  // the count pass reported bad entries
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int c = h ? b : a;
+      if (c < 0) continue;
+      const int u = bg * s.C + c;
+      const int slot = atomicAdd(cur + u, 1);
+      ent[slot] = (pl << 6) | (lane + 32 * h);
+      const int rel = slot - __ldg(off + u);
+      if (rel % PPI == 0)
+        items[__ldg(ioff + u) + rel / PPI] = make_int4(u, slot, min(PPI, __ldg(off + u + 1) - slot), 0);
+    }
   }
 }
 
@@ -575,9 +592,9 @@ cudaError_t launch_attn_prefill_chunked(const Shape& s, const void* q, const voi
     if (U > 0) {
       e = cudaMemsetAsync(cnt, 0, (size_t)U * 4, st);
       if (e != cudaSuccess) return e;
-      const long long pairs = (long long)s.B * s.Hkv * np * s.K;
-      const int grid = (int)std::min<long long>((pairs + 255) / 256, (long long)sms * 16);
-      bucket_count_kernel<<<grid, 256, 0, st>>>(s, idx, t0, np, cnt);
+      const long long lists = (long long)s.B * s.Hkv * np;
+      const int grid = (int)std::min<long long>((lists + 7) / 8, (long long)sms * 16);
+      bucket_count_kernel<<<grid, 256, 0, st>>>(s, idx, t0, np, cnt, ctx);
       bucket_scan_kernel<<<1, 1024, 0, st>>>(U, cnt, off, ioff);
       bucket_scatter_kernel<<<grid, 256, 0, st>>>(s, idx, t0, np, off, ioff, cnt, ent, items);
       attn_chunk_kernel<<<sms, THREADS, kSmemBytes, st>>>(s, tmk, tmv, (const __nv_bfloat16*)q, ioff, items, ent, t0,

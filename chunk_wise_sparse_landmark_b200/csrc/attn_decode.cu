@@ -77,9 +77,8 @@ __global__ void __launch_bounds__(kThreads) attn_decode_partial(Shape s, const T
       const int c = ir[u];
       sel = true;
       slot = u;
-      if (c < 0) return false;
-      if (c >= ncand) {
-        if (tid == 0) raise_status(ctx, kStatusBadIndex);
+      if (!list_entry_accepted(ir, u, ncand)) {  // the list form, common.cuh
+        if (c != -1 && tid == 0) raise_status(ctx, kStatusBadIndex);
         return false;
       }
       j0 = c * S;
@@ -295,9 +294,8 @@ __global__ void __launch_bounds__(kMmaWarps * 32) attn_decode_mma(Shape s, const
     int slot = -1;
     if (u < s.K) {
       const int c = ir[u];
-      if (c < 0) continue;
-      if (c >= ncand) {
-        if (lane == 0) raise_status(ctx, kStatusBadIndex);
+      if (!list_entry_accepted(ir, u, ncand)) {  // the list form, common.cuh
+        if (c != -1 && lane == 0) raise_status(ctx, kStatusBadIndex);
         continue;
       }
       sel = true;
@@ -454,7 +452,7 @@ cudaError_t go_g(const Shape& s, const void* q, const void* k, const void* v, co
     case 4: return go<T, D, S, 4>(s, q, k, v, idx, s_sel, out, ws, st, ctx);
     case 8: return go<T, D, S, 8>(s, q, k, v, idx, s_sel, out, ws, st, ctx);
   }
-  return cudaErrorInvalidValue;
+  return cudaErrorNotSupported;
 }
 
 }  // namespace
@@ -486,7 +484,7 @@ cudaError_t launch_attn_decode(const Shape& s, const void* q, const void* k, con
       case 8: return go_mma<8>(s, q, k, v, idx, s_sel, out, ws, nsplit, st, ctx);
     }
   }
-  return cudaErrorInvalidValue;
+  return cudaErrorNotSupported;
 }
 
 size_t decode_static_scratch_bytes() { return kStaticScratchFloats * sizeof(float); }

@@ -177,12 +177,12 @@ __global__ void __launch_bounds__(THREADS, 2)
       l1a = lane < K ? __ldg(L0 + K + lane) : -1;
       l1b = lane + 32 < K ? __ldg(L0 + K + lane + 32) : -1;
     }
-    // entries outside [0, ncand) are invalid: reported and dropped
-    if (l0a >= ncand || l0b >= ncand || l1a >= ncand || l1b >= ncand) raise_status(ctx, kStatusBadIndex);
-    l0a = l0a < ncand ? l0a : -1;
-    l0b = l0b < ncand ? l0b : -1;
-    l1a = l1a < ncand ? l1a : -1;
-    l1b = l1b < ncand ? l1b : -1;
+    // entries that break the list form (ascending candidates, then -1) are
+    // dropped and reported; the chunk-major bucketing drops the same ones
+    bool bad0, bad1;
+    accept_list_warp(l0a, l0b, K, ncand, bad0);
+    accept_list_warp(l1a, l1b, K, ncand, bad1);
+    if ((bad0 || bad1) && lane == 0) raise_status(ctx, kStatusBadIndex);
   }
   // with partial records the selected chunks were attended elsewhere: the
   // lists are kept for the fusion at the end and the stream is the window only
@@ -226,19 +226,30 @@ __global__ void __launch_bounds__(THREADS, 2)
     const int v = __shfl_sync(0xffffffffu, cu < 32 ? la : lb, cu & 31);
     return cu < K ? v : -1;
   };
+  // the accepted entries of the two lists (dropped ones left -1 holes)
+  const uint64_t vm0 = (uint64_t)__ballot_sync(0xffffffffu, l0a >= 0) |
+                       ((uint64_t)__ballot_sync(0xffffffffu, l0b >= 0) << 32);
+  const uint64_t vm1 = (uint64_t)__ballot_sync(0xffffffffu, l1a >= 0) |
+                       ((uint64_t)__ballot_sync(0xffffffffu, l1b >= 0) << 32);
+  // the first accepted entry at or after slot cu: its chunk (INT_MAX if none) and slot
+  auto next_at = [&](int la, int lb, uint64_t vm, int cu, int& x) -> int {
+    const uint64_t rest = cu < 64 ? (vm & (~0ull << cu)) : 0ull;
+    x = rest ? __ffsll((long long)rest) - 1 : 0;
+    const int v = __shfl_sync(0xffffffffu, x < 32 ? la : lb, x & 31);
+    return rest ? v : INT_MAX;
+  };
   auto step = [&](Walk& wk) {
-    int a0 = entry(l0a, l0b, wk.cu0), a1 = entry(l1a, l1b, wk.cu1);
-    a0 = a0 < 0 ? INT_MAX : a0;  // lists are ascending with -1 padding at the end
-    a1 = a1 < 0 ? INT_MAX : a1;
+    int x0, x1;
+    const int a0 = next_at(l0a, l0b, vm0, wk.cu0, x0), a1 = next_at(l1a, l1b, vm1, wk.cu1, x1);
     if (a0 != INT_MAX || a1 != INT_MAX) {
       wk.c = min(a0, a1);
       wk.win = false;
       wk.part0 = a0 == wk.c;
       wk.part1 = a1 == wk.c;
-      wk.slot0 = wk.cu0;
-      wk.slot1 = wk.cu1;
-      if (wk.part0) ++wk.cu0;
-      if (wk.part1) ++wk.cu1;
+      wk.slot0 = x0;
+      wk.slot1 = x1;
+      if (wk.part0) wk.cu0 = x0 + 1;
+      if (wk.part1) wk.cu1 = x1 + 1;
     } else if (valid0 && wc0 + wk.w <= cur) {
       wk.c = wc0 + wk.w++;
       wk.win = true;

@@ -77,13 +77,17 @@ __global__ void __launch_bounds__(256) attn_prefill_simt(Shape s, const float* _
   const int ncand = max(0, cur - s.nw + 1);
   const int32_t* ir = idx + (((long long)b * s.Hkv + g) * s.N + i) * s.K;
   const float* sr = s_sel + row * s.K;
+  // the list form (common.cuh, accept_list_warp): ascending candidates, then -1
+  int prev = -1;  // largest entry so far; a negative entry ends the list
   for (int x = 0; x < s.K; ++x) {
     const int c = ir[x];
-    if (c < 0) continue;
-    if (c >= ncand) {
-      if (lane == 0) raise_status(ctx, kStatusBadIndex);
+    const bool ok = c >= 0 && c < ncand && c > prev;
+    if (!ok) {
+      if (c != -1 && lane == 0) raise_status(ctx, kStatusBadIndex);
+      prev = c < 0 ? 0x7fffffff : max(prev, c);
       continue;
     }
+    prev = c;
     unit(c * s.S, c * s.S + s.S - 1, true, sr[x]);
   }
   float* o = out + row * D;
@@ -112,7 +116,7 @@ cudaError_t launch_attn_prefill_simt(const Shape& s, const void* q, const void* 
                                                     (float*)out, ctx);
       break;
     default:
-      return cudaErrorInvalidValue;
+      return cudaErrorNotSupported;
   }
   return cudaGetLastError();
 }

@@ -233,6 +233,60 @@ HILS_DI float warp_sum(float x) {
   return x;
 }
 
+// ------------------------------------------------------ chunk-list form ---
+// A selection list (one idx row) holds strictly ascending candidate chunks of
+// its position, c in [0, ncand), followed by -1 padding; hils_score_topk
+// writes exactly this form.  An entry is accepted iff it is a candidate and
+// lies above every earlier entry, a negative entry counting as +inf (so that
+// nothing after the first -1 is accepted).  Every attention kernel applies
+// this one rule, and reports (kStatusBadIndex) any entry other than -1 that
+// it drops, so that the passes agree on what they attend.
+//
+// Warp form: lane j holds entries j (a) and j + 32 (b); entries at or past K
+// are absent.  Returns the two entries with every rejected one replaced by -1
+// and sets `bad` (warp-uniform) if a non-padding entry was dropped.
+HILS_DI void accept_list_warp(int& a, int& b, int K, int ncand, bool& bad) {
+  const int lane = threadIdx.x & 31;
+  const bool pa = lane < K, pb = lane + 32 < K;
+  const int ka = (!pa || a < 0) ? 0x7fffffff : a;
+  const int kb = (!pb || b < 0) ? 0x7fffffff : b;
+  // exclusive prefix max of the keys over the list order a_0..a_31, b_0..b_31
+  int ia = ka, ib = kb;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int xa = __shfl_up_sync(0xffffffffu, ia, o), xb = __shfl_up_sync(0xffffffffu, ib, o);
+    if (lane >= o) {
+      ia = max(ia, xa);
+      ib = max(ib, xb);
+    }
+  }
+  const int tot_a = __shfl_sync(0xffffffffu, ia, 31);
+  int pa_ex = __shfl_up_sync(0xffffffffu, ia, 1), pb_ex = __shfl_up_sync(0xffffffffu, ib, 1);
+  if (lane == 0) {
+    pa_ex = -1;
+    pb_ex = tot_a;
+  } else {
+    pb_ex = max(pb_ex, tot_a);
+  }
+  const bool oka = pa && a >= 0 && a < ncand && a > pa_ex;
+  const bool okb = pb && b >= 0 && b < ncand && b > pb_ex;
+  const bool bada = pa && a != -1 && !oka, badb = pb && b != -1 && !okb;
+  bad = __any_sync(0xffffffffu, bada || badb);
+  a = oka ? a : -1;
+  b = okb ? b : -1;
+}
+
+// The same rule for entry x of a list in memory (sequential; K <= 64).
+HILS_DI bool list_entry_accepted(const int32_t* list, int x, int ncand) {
+  int prev = -1;
+  for (int y = 0; y < x; ++y) {
+    const int c = list[y];
+    prev = c < 0 ? 0x7fffffff : max(prev, c);
+  }
+  const int c = list[x];
+  return c >= 0 && c < ncand && c > prev;
+}
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 

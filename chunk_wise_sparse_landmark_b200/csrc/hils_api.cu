@@ -57,7 +57,44 @@ hils_status_t dev_ctx(DevCtx* ctx) {
 
 bool aligned16(const void* p) { return p && ((uintptr_t)p & 15u) == 0; }
 
-hils_status_t make_shape(const hils_config_t* cfg, Shape* s, bool decode) {
+// The operations whose shape coverage is checked on the host, before any
+// launch: a shape no kernel serves returns HILS_ERR_UNSUPPORTED.
+enum Op { kOpSummaries, kOpScorePrefill, kOpScoreDecode, kOpAttnPrefill, kOpAttnDecode, kOpPrefillHost, kOpNone };
+
+// Kernel coverage per operation (the dispatchers in the .cu files serve
+// exactly these shapes; anything else would reach no kernel).
+const char* uncovered(const Shape& s, Op op) {
+  if (s.dtype == HILS_F32) {
+    const bool d_ok = s.d == 32 || s.d == 64 || s.d == 128;
+    const bool s_ok = s.S == 16 || s.S == 32 || s.S == 64;
+    if (!d_ok) return "f32 needs d in {32, 64, 128}";
+    if (!s_ok) return "f32 needs S in {16, 32, 64}";
+    const bool summ = !(s.d == 32 && s.S == 64);
+    const bool score = !(s.d == 128 && s.G == 8);
+    const bool dec = (s.d == 64 || s.d == 128) && (s.S == 32 || s.S == 64);
+    switch (op) {
+      case kOpSummaries: return summ ? nullptr : "f32 summaries: no kernel for d = 32 with S = 64";
+      case kOpScorePrefill: return score ? nullptr : "f32 prefill scoring: no kernel for d = 128 with G = 8";
+      case kOpAttnDecode: return dec ? nullptr : "f32 decode attention needs d in {64, 128} and S in {32, 64}";
+      case kOpPrefillHost:
+        if (!summ) return "f32 summaries: no kernel for d = 32 with S = 64";
+        return score ? nullptr : "f32 prefill scoring: no kernel for d = 128 with G = 8";
+      default: return nullptr;
+    }
+  }
+  if (s.d != 128 || s.S != 64) return "bf16 needs d = 128 and S = 64";
+  switch (op) {
+    case kOpScorePrefill:
+    case kOpAttnPrefill:
+    case kOpPrefillHost:
+      if (s.G != 4) return "bf16 prefill needs G = Hq / Hkv = 4";
+      if (op != kOpScorePrefill && s.C > 8192) return "bf16 prefill attention needs N / S <= 8192";
+      return nullptr;
+    default: return nullptr;
+  }
+}
+
+hils_status_t make_shape(const hils_config_t* cfg, Shape* s, Op op) {
   if (!cfg) return fail(HILS_ERR_INVALID_ARG, "cfg is NULL");
   const hils_config_t& c = *cfg;
   if (c.batch < 1 || c.seq_len < 1 || c.n_q_heads < 1 || c.n_kv_heads < 1 || c.head_dim < 1 || c.chunk < 1 ||
@@ -88,13 +125,7 @@ hils_status_t make_shape(const hils_config_t* cfg, Shape* s, bool decode) {
   if (!g_ok) return fail(HILS_ERR_UNSUPPORTED, "G = Hq/Hkv = %d not in {1,2,4,8}", s->G);
   if (s->K > 64) return fail(HILS_ERR_UNSUPPORTED, "K = %d > 64", s->K);
   if (s->nw > 32) return fail(HILS_ERR_UNSUPPORTED, "W/S = %d > 32", s->nw);
-  if (c.dtype == HILS_F32) {
-    if (!(s->d == 32 || s->d == 64 || s->d == 128)) return fail(HILS_ERR_UNSUPPORTED, "f32: d=%d", s->d);
-    if (!(s->S == 16 || s->S == 32 || s->S == 64)) return fail(HILS_ERR_UNSUPPORTED, "f32: S=%d", s->S);
-  } else {
-    if (s->d != 128 || s->S != 64) return fail(HILS_ERR_UNSUPPORTED, "bf16 needs d=128, S=64 (got d=%d S=%d)", s->d, s->S);
-  }
-  (void)decode;
+  if (const char* why = uncovered(*s, op)) return fail(HILS_ERR_UNSUPPORTED, "%s", why);
   return HILS_OK;
 }
 
@@ -224,7 +255,7 @@ void hils_set_fault_injection(int32_t mode) { g_inject = mode == 1 ? 1 : 0; }
 hils_status_t hils_build_summaries(const hils_config_t* cfg, const void* k, const void* q_lmk, void* k_sum,
                                    float* b_sum, void* stream) {
   Shape s;
-  HILS_TRY(make_shape(cfg, &s, false));
+  HILS_TRY(make_shape(cfg, &s, kOpSummaries));
   if (!aligned16(k) || !aligned16(q_lmk) || !aligned16(k_sum) || !aligned16(b_sum))
     return fail(HILS_ERR_INVALID_ARG, "hils_build_summaries: NULL or unaligned pointer");
   if (s.dtype == HILS_BF16 && (((uintptr_t)k | (uintptr_t)q_lmk) & 31u))
@@ -237,7 +268,17 @@ hils_status_t hils_build_summaries(const hils_config_t* cfg, const void* k, cons
 
 size_t hils_workspace_bytes(const hils_config_t* cfg, int32_t which, int32_t qcal_rank) {
   Shape s;
-  if (make_shape(cfg, &s, which != HILS_WS_SCORE_PREFILL) != HILS_OK) return (size_t)-1;
+  const Op op = which == HILS_WS_SCORE_PREFILL ? kOpScorePrefill
+                : which == HILS_WS_SCORE_DECODE ? kOpScoreDecode
+                : which == HILS_WS_ATTN_DECODE  ? kOpAttnDecode
+                : which == HILS_WS_PREFILL_HOST ? kOpPrefillHost
+                : which == HILS_WS_ATTN_PREFILL ? kOpAttnPrefill
+                                                : kOpNone;
+  if (op == kOpNone) {
+    fail(HILS_ERR_INVALID_ARG, "unknown workspace kind %d", which);
+    return (size_t)-1;
+  }
+  if (make_shape(cfg, &s, op) != HILS_OK) return (size_t)-1;
   switch (which) {
     case HILS_WS_SCORE_PREFILL: {
       size_t b = 0;
@@ -261,7 +302,7 @@ hils_status_t hils_score_topk(const hils_config_t* cfg, const void* q, const hil
                               const float* b_sum, int32_t* idx, float* s_sel, void* workspace, size_t ws_bytes,
                               int32_t decode, void* stream) {
   Shape s;
-  HILS_TRY(make_shape(cfg, &s, decode != 0));
+  HILS_TRY(make_shape(cfg, &s, decode ? kOpScoreDecode : kOpScorePrefill));
   if (decode != 0 && decode != 1) return fail(HILS_ERR_INVALID_ARG, "decode must be 0 or 1");
   if (!aligned16(q) || !aligned16(k_sum) || !aligned16(b_sum) || !aligned16(idx) || !aligned16(s_sel))
     return fail(HILS_ERR_INVALID_ARG, "hils_score_topk: NULL or unaligned pointer");
@@ -269,22 +310,24 @@ hils_status_t hils_score_topk(const hils_config_t* cfg, const void* q, const hil
                                            qcal ? qcal->rank : 0);
   if (need > 0 && (ws_bytes < need || !aligned16(workspace)))
     return fail(HILS_ERR_INVALID_ARG, "hils_score_topk: workspace needs %zu bytes (got %zu)", need, ws_bytes);
+  if (qcal) {
+    if (decode) return fail(HILS_ERR_UNSUPPORTED, "Q-Cal is a prefill-only option");
+    if (!aligned16(qcal->h) || !aligned16(qcal->w_down) || !aligned16(qcal->w_up))
+      return fail(HILS_ERR_INVALID_ARG, "Q-Cal: NULL or unaligned pointer");
+    if (qcal->rank != 64 || qcal->d_model < 64 || qcal->d_model % 64)
+      return fail(HILS_ERR_UNSUPPORTED, "Q-Cal: rank %d / d_model %d not supported", qcal->rank, qcal->d_model);
+    if (s.dtype != HILS_BF16) return fail(HILS_ERR_UNSUPPORTED, "Q-Cal needs bf16");
+  }
   DevCtx ctx;
   HILS_TRY(dev_ctx(&ctx));
   cudaStream_t st = (cudaStream_t)stream;
   if (decode) {
-    if (qcal) return fail(HILS_ERR_UNSUPPORTED, "Q-Cal is a prefill-only option");
     HILS_LAUNCH(launch_score_topk_decode(s, q, k_sum, b_sum, idx, s_sel, workspace, st, ctx), "score_topk_decode");
     return HILS_OK;
   }
   const void* q_score = q;
   unsigned char* ws = (unsigned char*)workspace;
   if (qcal) {
-    if (!aligned16(qcal->h) || !aligned16(qcal->w_down) || !aligned16(qcal->w_up))
-      return fail(HILS_ERR_INVALID_ARG, "Q-Cal: NULL or unaligned pointer");
-    if (qcal->rank < 16 || qcal->rank > 128 || qcal->rank % 16 || qcal->d_model < 64 || qcal->d_model % 64)
-      return fail(HILS_ERR_UNSUPPORTED, "Q-Cal: rank %d / d_model %d not supported", qcal->rank, qcal->d_model);
-    if (s.dtype != HILS_BF16) return fail(HILS_ERR_UNSUPPORTED, "Q-Cal needs bf16");
     void* q_tilde = ws;
     ws += (size_t)s.B * s.Hq * s.N * s.d * esize(s);
     HILS_LAUNCH(launch_qcal_tc(s, q, qcal->h, qcal->w_down, qcal->w_up, qcal->rank, qcal->d_model, q_tilde, st, ctx),
@@ -303,7 +346,7 @@ hils_status_t hils_attn_prefill(const hils_config_t* cfg, const void* q, const v
                                 const int32_t* idx, const float* s_sel, void* out, void* workspace,
                                 size_t ws_bytes, void* stream) {
   Shape s;
-  HILS_TRY(make_shape(cfg, &s, false));
+  HILS_TRY(make_shape(cfg, &s, kOpAttnPrefill));
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(s_sel) || !aligned16(out))
     return fail(HILS_ERR_INVALID_ARG, "hils_attn_prefill: NULL or unaligned pointer");
   const bool bf16 = s.dtype == HILS_BF16;
@@ -332,13 +375,13 @@ hils_status_t hils_prefill_host(const hils_config_t* cfg, const void* h_q, const
                                 const void* h_q_lmk, const hils_qcal_t* qcal, void* h_out, void* workspace,
                                 size_t ws_bytes, void* stream) {
   Shape s;
-  HILS_TRY(make_shape(cfg, &s, false));
+  HILS_TRY(make_shape(cfg, &s, kOpPrefillHost));
   if (!h_q || !h_k || !h_v || !h_q_lmk || !h_out) return fail(HILS_ERR_INVALID_ARG, "hils_prefill_host: NULL host pointer");
   const int rank = qcal ? qcal->rank : 0;
   if (qcal) {
     if (!qcal->h || !qcal->w_down || !qcal->w_up) return fail(HILS_ERR_INVALID_ARG, "Q-Cal: NULL host pointer");
     if (s.dtype != HILS_BF16) return fail(HILS_ERR_UNSUPPORTED, "Q-Cal needs bf16");
-    if (qcal->rank < 16 || qcal->rank > 128 || qcal->rank % 16 || qcal->d_model != s.Hq * s.d)
+    if (qcal->rank != 64 || qcal->d_model != s.Hq * s.d)
       return fail(HILS_ERR_UNSUPPORTED, "hils_prefill_host: Q-Cal rank %d / d_model %d not supported (d_model must be Hq*d)",
                   qcal->rank, qcal->d_model);
   }
@@ -455,7 +498,7 @@ hils_status_t hils_attn_decode(const hils_config_t* cfg, const void* q, const vo
                                const int32_t* idx, const float* s_sel, void* out, void* workspace, size_t ws_bytes,
                                void* stream) {
   Shape s;
-  HILS_TRY(make_shape(cfg, &s, true));
+  HILS_TRY(make_shape(cfg, &s, kOpAttnDecode));
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(idx) || !aligned16(s_sel) ||
       !aligned16(out))
     return fail(HILS_ERR_INVALID_ARG, "hils_attn_decode: NULL or unaligned pointer");
@@ -473,7 +516,7 @@ hils_status_t hils_attn_decode_noalloc(const hils_config_t* cfg, const void* q, 
                                        const void* v_cache, const int32_t* idx, const float* s_sel, void* out,
                                        void* stream) {
   Shape s;
-  HILS_TRY(make_shape(cfg, &s, true));
+  HILS_TRY(make_shape(cfg, &s, kOpAttnDecode));
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(idx) || !aligned16(s_sel) ||
       !aligned16(out))
     return fail(HILS_ERR_INVALID_ARG, "hils_attn_decode_noalloc: NULL or unaligned pointer");

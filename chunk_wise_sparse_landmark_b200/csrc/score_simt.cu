@@ -132,7 +132,7 @@ cudaError_t go_prefill(const Shape& s, const void* q, const void* k_sum, const f
     score_topk_prefill_simt<D, G, 65><<<grid, kQB * G, 0, st>>>(s, (const float*)q, (const float*)k_sum, b_sum, idx,
                                                                  s_sel);
   else
-    return cudaErrorInvalidValue;
+    return cudaErrorNotSupported;
   return cudaGetLastError();
 }
 
@@ -411,7 +411,7 @@ cudaError_t go_decode_g(const Shape& s, const void* q, const void* k_sum, const 
     case 4: return go_decode<T, D, 4>(s, q, k_sum, b_sum, idx, s_sel, ws, st);
     case 8: return go_decode<T, D, 8>(s, q, k_sum, b_sum, idx, s_sel, ws, st);
   }
-  return cudaErrorInvalidValue;
+  return cudaErrorNotSupported;
 }
 
 }  // namespace
@@ -424,7 +424,7 @@ cudaError_t launch_score_topk_simt(const Shape& s, const void* q, const void* k_
   HILS_CASE(64, 1) HILS_CASE(64, 2) HILS_CASE(64, 4) HILS_CASE(64, 8)
   HILS_CASE(128, 1) HILS_CASE(128, 2) HILS_CASE(128, 4)
 #undef HILS_CASE
-  return cudaErrorInvalidValue;
+  return cudaErrorNotSupported;
 }
 
 size_t decode_score_workspace(const Shape& s) {
@@ -440,7 +440,7 @@ cudaError_t launch_score_topk_decode(const Shape& s, const void* q, const void* 
   } else {
     if (s.d == 128) return go_decode_g<__nv_bfloat16, 128>(s, q, k_sum, b_sum, idx, s_sel, ws, st);
   }
-  return cudaErrorInvalidValue;
+  return cudaErrorNotSupported;
 }
 
 }  // namespace hils

@@ -99,7 +99,7 @@ cudaError_t go_g(const Shape& s, const void* k, const void* q_lmk, void* k_sum, 
     case 4: return go<T, D, S, 4>(s, k, q_lmk, k_sum, b_sum, st);
     case 8: return go<T, D, S, 8>(s, k, q_lmk, k_sum, b_sum, st);
   }
-  return cudaErrorInvalidValue;
+  return cudaErrorNotSupported;
 }
 
 template <typename T>
@@ -115,7 +115,7 @@ cudaError_t go_t(const Shape& s, const void* k, const void* q_lmk, void* k_sum, 
   HILS_CASE(128, 16)
   HILS_CASE(32, 32)
 #undef HILS_CASE
-  return cudaErrorInvalidValue;
+  return cudaErrorNotSupported;
 }
 
 // ---------------------------------------------------------------------------

@@ -33,9 +33,17 @@
  *    thread-local message for the last non-OK status.  No C++ exception
  *    crosses this boundary.
  *
- * Supported kernels: dtype F32 (SIMT kernels, any d in {32,64,96,128},
- * S in {16,32,64}); dtype BF16 with d = 128 and S = 64 (tensor-core prefill
- * path; SIMT decode path).  K <= 64, n_w <= 32.
+ * Supported shapes (anything else returns HILS_ERR_UNSUPPORTED, checked on
+ * the host before any launch):
+ *  - every call: G in {1, 2, 4, 8}, K <= 64, n_w = W/S <= 32;
+ *  - dtype F32 (CUDA-core kernels with fp32 FMA): d in {32, 64, 128} and
+ *    S in {16, 32, 64}, except summaries with d = 32 and S = 64, prefill
+ *    scoring with d = 128 and G = 8, and decode attention with d = 32 or
+ *    S = 16;
+ *  - dtype BF16 (tensor-core kernels): d = 128 and S = 64; prefill scoring
+ *    and prefill attention need G = 4, and prefill attention N/S <= 8192;
+ *    decode works for every G (its attention gathers tiles into warp-level
+ *    MMAs); Q-Cal needs rank 64 and d_model a multiple of 64.
  */
 #ifndef HILS_H
 #define HILS_H
@@ -78,7 +86,7 @@ typedef struct {
   const void* h;       /* [B, N, d_model] hidden states (dtype); decode: [B, d_model] */
   const void* w_down;  /* [r, d_model] (dtype) */
   const void* w_up;    /* [Hq*d, r] (dtype); row hq*d+e feeds head hq, dim e */
-  int32_t rank;        /* r, a multiple of 16, <= 128 */
+  int32_t rank;        /* r; the kernels support r = 64 */
   int32_t d_model;     /* a multiple of 64 */
 } hils_qcal_t;
 
@@ -132,8 +140,12 @@ hils_status_t hils_score_topk(const hils_config_t* cfg, const void* q, const hil
  * raw q.
  *   q [B, Hq, N, d]; k, v [B, Hkv, N, d]; idx [B, Hkv, N, K]; s_sel [B, Hq, N, K];
  *   out [B, Hq, N, d] (dtype, out).
- * idx entries must be -1 or candidates of their position (checked on device:
- * an out-of-range entry is skipped and recorded in the status word).
+ * Each idx list must hold strictly ascending candidates of its position
+ * followed by -1 padding (the form hils_score_topk writes).  Checked on the
+ * device: an entry that is not a candidate, is not above every earlier entry
+ * of its list, or follows a -1 is skipped (both attention passes skip the same
+ * entries) and recorded in the status word, which hils_sync_status() reports
+ * as HILS_ERR_INVALID_ARG.
  *   workspace: device scratch of at least
  *              hils_workspace_bytes(cfg, HILS_WS_ATTN_PREFILL, 0) bytes
  *              (16-byte aligned; 0 bytes for dtype F32).  With it, bf16 runs
@@ -157,6 +169,8 @@ hils_status_t hils_attn_prefill(const hils_config_t* cfg, const void* q, const v
  * split across CTAs and merged by a second kernel.
  *   q [B, Hq, d]; k_cache, v_cache [B, Hkv, L, d]; idx [B, Hkv, K];
  *   s_sel [B, Hq, K]; out [B, Hq, d] (dtype, out).
+ *   idx lists have the form described at hils_attn_prefill and are checked
+ *   the same way.
  *   workspace: at least hils_workspace_bytes(cfg, HILS_WS_ATTN_DECODE, 0)
  *              bytes of device scratch for the per-split partial results.
  */
@@ -244,7 +258,8 @@ size_t hils_workspace_bytes(const hils_config_t* cfg, int32_t which, int32_t qca
 
 /* Synchronises `stream`, then reads and clears the calling device's status
  * word: HILS_OK, HILS_ERR_TIMEOUT (a bounded device wait ran out), or
- * HILS_ERR_INVALID_ARG (a kernel skipped an out-of-range index). */
+ * HILS_ERR_INVALID_ARG (a kernel skipped a chunk-list entry that was not a
+ * candidate, not ascending, or after the list's -1 padding). */
 hils_status_t hils_sync_status(void* stream);
 
 /* Thread-local text for the last non-OK status returned on this thread. */

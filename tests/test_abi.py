@@ -119,3 +119,49 @@ def test_prefill_host_workspace_and_host_checks():
     assert st == H.HILS_ERR_INVALID_ARG
     st = lib.hils_prefill_host(ctypes.byref(cfg), p, p, p, p, None, p, p, want - 1, None)
     assert st == H.HILS_ERR_INVALID_ARG and b"workspace" in lib.hils_last_error()
+
+
+@pytest.mark.parametrize(
+    "call,kw",
+    [
+        ("summaries", dict(d=32, S=64)),                      # f32 summaries: no (d=32, S=64) kernel
+        ("score_prefill", dict(d=128, S=64, Hq=8, Hkv=1)),    # f32 prefill scoring: no G=8 kernel at d=128
+        ("attn_decode", dict(d=32, S=32)),                    # f32 decode attention: d=32
+        ("attn_decode", dict(d=64, S=16)),                    # f32 decode attention: S=16
+        ("score_prefill", dict(dtype="bf16", d=128, S=64, Hq=8, Hkv=1)),  # bf16 prefill: G=4 only
+        ("attn_prefill", dict(dtype="bf16", d=128, S=64, Hq=8, Hkv=4)),   # bf16 prefill: G=4 only
+    ],
+)
+def test_shapes_without_a_kernel_are_unsupported_on_host(call, kw):
+    """Shapes that no kernel serves return HILS_ERR_UNSUPPORTED from the host
+    checks, before any device work (so this runs without a GPU)."""
+    base = dict(B=1, N=512, Hq=4, Hkv=1, d=64, S=32, W=64, K=4, dtype="f32")
+    base.update(kw)
+    if base["W"] < base["S"]:
+        base["W"] = base["S"]
+    base["W"] = max(base["W"], 2 * base["S"])
+    cfg = H.make_config(**base)
+    lib = H.load()
+    p = ctypes.c_void_p(0x1000)
+    if call == "summaries":
+        st = lib.hils_build_summaries(ctypes.byref(cfg), p, p, p, p, None)
+    elif call == "score_prefill":
+        st = lib.hils_score_topk(ctypes.byref(cfg), p, None, p, p, p, p, p, 1 << 30, 0, None)
+    elif call == "attn_prefill":
+        st = lib.hils_attn_prefill(ctypes.byref(cfg), p, p, p, p, p, p, None, 0, None)
+    else:
+        st = lib.hils_attn_decode(ctypes.byref(cfg), p, p, p, p, p, p, p, 1 << 30, None)
+    assert st == H.HILS_ERR_UNSUPPORTED, (st, lib.hils_last_error())
+    which = {"summaries": None, "score_prefill": H.HILS_WS_SCORE_PREFILL, "attn_prefill": H.HILS_WS_ATTN_PREFILL,
+             "attn_decode": H.HILS_WS_ATTN_DECODE}[call]
+    if which is not None:
+        assert lib.hils_workspace_bytes(ctypes.byref(cfg), which, 0) == ctypes.c_size_t(-1).value
+
+
+def test_qcal_rank_other_than_64_is_unsupported_on_host():
+    lib = H.load()
+    cfg = H.make_config(1, 1024, 4, 1, 128, 64, 128, 4, "bf16")
+    p = ctypes.c_void_p(0x1000)
+    qc = H.QCal(0x1000, 0x1000, 0x1000, 32, 4096)
+    st = lib.hils_score_topk(ctypes.byref(cfg), p, ctypes.byref(qc), p, p, p, p, p, 1 << 40, 0, None)
+    assert st == H.HILS_ERR_UNSUPPORTED, lib.hils_last_error()

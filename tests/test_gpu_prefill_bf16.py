@@ -245,6 +245,58 @@ def test_qcal_zero_up_projection_changes_nothing():
     H.hils_sync_status()
     assert torch.equal(base.idx, qc.idx)
     assert torch.equal(base.s_sel, qc.s_sel)
-    # the attention adds chunk contributions with shared-memory atomics, so two
-    # runs may round differently in the last bf16 bit
-    torch.testing.assert_close(base.out.float(), qc.out.float(), atol=1e-3, rtol=2.0 ** -7)
+    # the same selection through deterministic kernels: the same bits
+    assert torch.equal(base.out, qc.out)
+
+
+def _list_form(lst, ncand):
+    """The list form every attention pass accepts (include/hils.h): strictly
+    ascending candidates, then -1.  Entries that break it become -1."""
+    out, prev = [], -1
+    for c in lst:
+        out.append(int(c) if 0 <= c < ncand and c > prev else -1)
+        prev = 1 << 30 if c < 0 else max(prev, int(c))
+    return out
+
+
+@PASSES
+def test_bad_list_entries_are_dropped_and_reported(chunked):
+    """A duplicate, a -7 and a non-ascending pair in the bf16 path: those
+    entries (and, after the -7, the rest of its list) are dropped by both
+    passes, hils_sync_status reports HILS_ERR_INVALID_ARG, and every row
+    equals the oracle run on the cleaned lists."""
+    w = WORKLOADS["prefill_8k"].scaled(name="badidx", N=4096, Hq=8, Hkv=2, needles_per_head=0)
+    x = prefill_inputs(w)
+    dm = _dims(w)
+    q, k, v, ql = (to_np(x[n]) for n in ("q", "k", "v", "q_lmk"))
+    ks, bs = oracle.summaries(dm, k, ql)
+    rows_all = oracle.all_rows(w.B, w.N)
+    idx, ssel = oracle.select(dm, rows_all, q, k_sum=ks, b_sum=bs)  # [N, Hkv, K]
+    bad = idx.copy()
+    p_dup, p_neg, p_swap = 3000, 3500, 4095
+    assert (bad[[p_dup, p_neg, p_swap]] >= 0).all()  # full lists
+    bad[p_dup, 0, 5] = bad[p_dup, 0, 4]
+    bad[p_neg, 1, 2] = -7
+    bad[p_swap, 0, 7], bad[p_swap, 0, 8] = idx[p_swap, 0, 8], idx[p_swap, 0, 7]
+    clean = bad.copy()
+    for p in (p_dup, p_neg, p_swap):
+        for g in range(w.Hkv):
+            clean[p, g] = _list_form(bad[p, g], max(0, p // w.S - w.W // w.S + 1))
+    assert (clean != idx).sum() >= 1 + 13 + 1
+    idx_t = torch.from_numpy(bad.reshape(w.B, w.N, w.Hkv, w.K).transpose(0, 2, 1, 3).copy()).int().to(DEV)
+    ssel32 = ssel.astype(np.float32)
+    ssel_t = torch.from_numpy(ssel32.reshape(w.B, w.N, w.Hq, w.K).transpose(0, 2, 1, 3).copy()).to(DEV)
+    d = {n: x[n].to(DEV) for n in ("q", "k", "v")}
+    out = torch.empty((w.B, w.Hq, w.N, w.d), dtype=torch.bfloat16, device=DEV)
+    cfg = H.config_of(w)
+    ws = H.alloc_workspace(H.workspace_bytes(cfg, H.HILS_WS_ATTN_PREFILL), DEV) if chunked else None
+    H.hils_attn_prefill(cfg, d["q"], d["k"], d["v"], idx_t.contiguous(), ssel_t.contiguous(), out, ws)
+    with pytest.raises(H.HilsError) as ei:
+        H.hils_sync_status()
+    assert ei.value.status == H.HILS_ERR_INVALID_ARG
+    H.hils_sync_status()  # cleared
+    rows = [(0, p) for p in (0, 700, 2999, p_dup, p_neg, p_swap)]
+    ridx = np.array([p for _, p in rows])
+    ref = oracle.attend(dm, rows, q, k, v, clean[ridx], ssel32[ridx].astype(np.float64))
+    got = to_np(out).transpose(0, 2, 1, 3).reshape(w.N, w.Hq, w.d)[ridx]
+    assert np.abs(got - ref).max() <= TOL_BF16
