@@ -266,6 +266,20 @@ hils_status_t hils_build_summaries(const hils_config_t* cfg, const void* k, cons
   return HILS_OK;
 }
 
+hils_status_t hils_build_summaries_shared(const hils_config_t* cfg, const void* k, const void* q_shared,
+                                          void* k_sum, float* b_sum, void* stream) {
+  Shape s;
+  HILS_TRY(make_shape(cfg, &s, kOpSummaries));
+  if (!aligned16(k) || !aligned16(q_shared) || !aligned16(k_sum) || !aligned16(b_sum))
+    return fail(HILS_ERR_INVALID_ARG, "hils_build_summaries_shared: NULL or unaligned pointer");
+  if (s.dtype == HILS_BF16 && (((uintptr_t)k | (uintptr_t)q_shared) & 31u))
+    return fail(HILS_ERR_INVALID_ARG, "hils_build_summaries_shared: bf16 k and q_shared must be 32-byte aligned");
+  DevCtx ctx;
+  HILS_TRY(dev_ctx(&ctx));
+  HILS_LAUNCH(launch_summaries(s, k, q_shared, k_sum, b_sum, (cudaStream_t)stream, ctx, true), "summaries_shared");
+  return HILS_OK;
+}
+
 size_t hils_workspace_bytes(const hils_config_t* cfg, int32_t which, int32_t qcal_rank) {
   Shape s;
   const Op op = which == HILS_WS_SCORE_PREFILL ? kOpScorePrefill

@@ -17,9 +17,10 @@ struct Shape {
   int dtype;  // 0 f32, 1 bf16
 };
 
-// K1: landmark summaries (all dtypes)
+// K1: landmark summaries (all dtypes); shared_lmk: q_lmk is one query per head
+// [Hq, d] shared by every chunk and sequence (the landmark-free variant)
 cudaError_t launch_summaries(const Shape& s, const void* k, const void* q_lmk, void* k_sum, float* b_sum,
-                             cudaStream_t st, const DevCtx& ctx);
+                             cudaStream_t st, const DevCtx& ctx, bool shared_lmk = false);
 
 // fp32 SIMT prefill score + group max + top-K
 cudaError_t launch_score_topk_simt(const Shape& s, const void* q, const void* k_sum, const float* b_sum, int32_t* idx,

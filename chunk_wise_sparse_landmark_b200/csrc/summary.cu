@@ -20,10 +20,18 @@ namespace {
 
 constexpr int kThreads = 256;
 
+// Element offset of the landmark query of (sequence b, query head h, chunk c):
+// per-chunk queries use strides (Hq C d, C d, d); the landmark-free variant's
+// one shared query per head uses (0, d, 0).
+struct LmkStrides {
+  long long b, h, c;
+  HILS_DI long long of(int bb, int hh, int cc) const { return bb * b + hh * h + cc * c; }
+};
+
 template <typename T, int D, int S, int G>
 __global__ void __launch_bounds__(kThreads) summaries_kernel(Shape s, const T* __restrict__ k,
-                                                             const T* __restrict__ q_lmk, T* __restrict__ k_sum,
-                                                             float* __restrict__ b_sum) {
+                                                             const T* __restrict__ q_lmk, LmkStrides ls,
+                                                             T* __restrict__ k_sum, float* __restrict__ b_sum) {
   __shared__ float ks[S][D + 1];
   __shared__ float qs[G][D];
   __shared__ float lg[G][S];
@@ -37,7 +45,7 @@ __global__ void __launch_bounds__(kThreads) summaries_kernel(Shape s, const T* _
     for (int e = tid; e < S * D; e += kThreads) ks[e / D][e % D] = to_f32(kc[e]);
     for (int e = tid; e < G * D; e += kThreads) {
       const int hg = e / D;
-      qs[hg][e % D] = to_f32(q_lmk[(((long long)b * s.Hq + g * G + hg) * s.C + c) * D + e % D]);
+      qs[hg][e % D] = to_f32(q_lmk[ls.of(b, g * G + hg, c) + e % D]);
     }
     __syncthreads();
     // logits l[h][j] = q'_h . k_j * scale
@@ -81,31 +89,34 @@ __global__ void __launch_bounds__(kThreads) summaries_kernel(Shape s, const T* _
 }
 
 template <typename T, int D, int S, int G>
-cudaError_t go(const Shape& s, const void* k, const void* q_lmk, void* k_sum, float* b_sum, cudaStream_t st) {
+cudaError_t go(const Shape& s, const void* k, const void* q_lmk, const LmkStrides& ls, void* k_sum, float* b_sum,
+               cudaStream_t st) {
   const long long units = (long long)s.B * s.Hkv * s.C;
   if (units == 0) return cudaSuccess;
   const int sms = device_sm_count();
   const long long grid = units < (long long)sms * 8 ? units : (long long)sms * 8;
-  summaries_kernel<T, D, S, G><<<(unsigned)grid, kThreads, 0, st>>>(s, (const T*)k, (const T*)q_lmk, (T*)k_sum,
+  summaries_kernel<T, D, S, G><<<(unsigned)grid, kThreads, 0, st>>>(s, (const T*)k, (const T*)q_lmk, ls, (T*)k_sum,
                                                                      b_sum);
   return cudaGetLastError();
 }
 
 template <typename T, int D, int S>
-cudaError_t go_g(const Shape& s, const void* k, const void* q_lmk, void* k_sum, float* b_sum, cudaStream_t st) {
+cudaError_t go_g(const Shape& s, const void* k, const void* q_lmk, const LmkStrides& ls, void* k_sum, float* b_sum,
+                 cudaStream_t st) {
   switch (s.G) {
-    case 1: return go<T, D, S, 1>(s, k, q_lmk, k_sum, b_sum, st);
-    case 2: return go<T, D, S, 2>(s, k, q_lmk, k_sum, b_sum, st);
-    case 4: return go<T, D, S, 4>(s, k, q_lmk, k_sum, b_sum, st);
-    case 8: return go<T, D, S, 8>(s, k, q_lmk, k_sum, b_sum, st);
+    case 1: return go<T, D, S, 1>(s, k, q_lmk, ls, k_sum, b_sum, st);
+    case 2: return go<T, D, S, 2>(s, k, q_lmk, ls, k_sum, b_sum, st);
+    case 4: return go<T, D, S, 4>(s, k, q_lmk, ls, k_sum, b_sum, st);
+    case 8: return go<T, D, S, 8>(s, k, q_lmk, ls, k_sum, b_sum, st);
   }
   return cudaErrorNotSupported;
 }
 
 template <typename T>
-cudaError_t go_t(const Shape& s, const void* k, const void* q_lmk, void* k_sum, float* b_sum, cudaStream_t st) {
+cudaError_t go_t(const Shape& s, const void* k, const void* q_lmk, const LmkStrides& ls, void* k_sum, float* b_sum,
+                 cudaStream_t st) {
 #define HILS_CASE(DD, SS) \
-  if (s.d == DD && s.S == SS) return go_g<T, DD, SS>(s, k, q_lmk, k_sum, b_sum, st);
+  if (s.d == DD && s.S == SS) return go_g<T, DD, SS>(s, k, q_lmk, ls, k_sum, b_sum, st);
   HILS_CASE(64, 32)
   HILS_CASE(64, 64)
   HILS_CASE(128, 32)
@@ -130,7 +141,7 @@ cudaError_t go_t(const Shape& s, const void* k, const void* q_lmk, void* k_sum, 
 // line-wide loads: gather_mma.cuh; the second read of the tile hits L1.
 template <int G>
 __global__ void __launch_bounds__(256) summaries_mma(Shape s, const __nv_bfloat16* __restrict__ k,
-                                                     const __nv_bfloat16* __restrict__ q_lmk,
+                                                     const __nv_bfloat16* __restrict__ q_lmk, LmkStrides ls,
                                                      __nv_bfloat16* __restrict__ k_sum, float* __restrict__ b_sum) {
   constexpr int D = 128, S = 64;
   const int lane = threadIdx.x & 31;
@@ -144,7 +155,7 @@ __global__ void __launch_bounds__(256) summaries_mma(Shape s, const __nv_bfloat1
     const __nv_bfloat16* kc = k + (((long long)b * s.Hkv + g) * s.N + (long long)c * S) * D;
     // Q'^T as the B operand: column gq = landmark query of head g*G + gq
     uint32_t qf[2][8];
-    load_qcol(gq < G ? q_lmk + (((long long)b * s.Hq + g * G + gq) * s.C + c) * D : nullptr, c4, qf);
+    load_qcol(gq < G ? q_lmk + ls.of(b, g * G + gq, c) : nullptr, c4, qf);
     float sc[4][4];
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt) sc[mt][0] = sc[mt][1] = sc[mt][2] = sc[mt][3] = 0.f;
@@ -215,13 +226,14 @@ __global__ void __launch_bounds__(256) summaries_mma(Shape s, const __nv_bfloat1
 }
 
 template <int G>
-cudaError_t go_mma(const Shape& s, const void* k, const void* q_lmk, void* k_sum, float* b_sum, cudaStream_t st) {
+cudaError_t go_mma(const Shape& s, const void* k, const void* q_lmk, const LmkStrides& ls, void* k_sum, float* b_sum,
+                   cudaStream_t st) {
   const long long units = (long long)s.B * s.Hkv * s.C;
   if (units == 0) return cudaSuccess;
   const long long blocks_needed = (units + 7) / 8;
   const long long cap = (long long)device_sm_count() * 8;
   const unsigned grid = (unsigned)(blocks_needed < cap ? blocks_needed : cap);
-  summaries_mma<G><<<grid, 256, 0, st>>>(s, (const __nv_bfloat16*)k, (const __nv_bfloat16*)q_lmk,
+  summaries_mma<G><<<grid, 256, 0, st>>>(s, (const __nv_bfloat16*)k, (const __nv_bfloat16*)q_lmk, ls,
                                          (__nv_bfloat16*)k_sum, b_sum);
   return cudaGetLastError();
 }
@@ -229,17 +241,20 @@ cudaError_t go_mma(const Shape& s, const void* k, const void* q_lmk, void* k_sum
 }  // namespace
 
 cudaError_t launch_summaries(const Shape& s, const void* k, const void* q_lmk, void* k_sum, float* b_sum,
-                             cudaStream_t st, const DevCtx&) {
-  if (s.dtype == 0) return go_t<float>(s, k, q_lmk, k_sum, b_sum, st);
+                             cudaStream_t st, const DevCtx&, bool shared_lmk) {
+  // per-chunk landmark queries [B, Hq, C, d], or one shared query per head [Hq, d]
+  const LmkStrides ls = shared_lmk ? LmkStrides{0, (long long)s.d, 0}
+                                   : LmkStrides{(long long)s.Hq * s.C * s.d, (long long)s.C * s.d, (long long)s.d};
+  if (s.dtype == 0) return go_t<float>(s, k, q_lmk, ls, k_sum, b_sum, st);
   if (s.d == 128 && s.S == 64) {
     switch (s.G) {
-      case 1: return go_mma<1>(s, k, q_lmk, k_sum, b_sum, st);
-      case 2: return go_mma<2>(s, k, q_lmk, k_sum, b_sum, st);
-      case 4: return go_mma<4>(s, k, q_lmk, k_sum, b_sum, st);
-      case 8: return go_mma<8>(s, k, q_lmk, k_sum, b_sum, st);
+      case 1: return go_mma<1>(s, k, q_lmk, ls, k_sum, b_sum, st);
+      case 2: return go_mma<2>(s, k, q_lmk, ls, k_sum, b_sum, st);
+      case 4: return go_mma<4>(s, k, q_lmk, ls, k_sum, b_sum, st);
+      case 8: return go_mma<8>(s, k, q_lmk, ls, k_sum, b_sum, st);
     }
   }
-  return go_t<__nv_bfloat16>(s, k, q_lmk, k_sum, b_sum, st);
+  return go_t<__nv_bfloat16>(s, k, q_lmk, ls, k_sum, b_sum, st);
 }
 
 }  // namespace hils

@@ -21,6 +21,7 @@ HILS_WS_SCORE_PREFILL, HILS_WS_SCORE_DECODE, HILS_WS_ATTN_DECODE, HILS_WS_PREFIL
 
 EXPORTS = (
     "hils_build_summaries",
+    "hils_build_summaries_shared",
     "hils_score_topk",
     "hils_attn_prefill",
     "hils_attn_decode",
@@ -79,6 +80,7 @@ def load() -> ctypes.CDLL:
         lib = ctypes.CDLL(LIB_PATH)
         P, C = ctypes.c_void_p, ctypes.POINTER(Config)
         lib.hils_build_summaries.argtypes = [C, P, P, P, P, P]
+        lib.hils_build_summaries_shared.argtypes = [C, P, P, P, P, P]
         lib.hils_score_topk.argtypes = [C, P, ctypes.POINTER(QCal), P, P, P, P, P, ctypes.c_size_t, ctypes.c_int32, P]
         lib.hils_attn_prefill.argtypes = [C, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         lib.hils_attn_decode.argtypes = [C, P, P, P, P, P, P, P, ctypes.c_size_t, P]
@@ -93,8 +95,8 @@ def load() -> ctypes.CDLL:
         lib.hils_set_fault_injection.argtypes = [ctypes.c_int32]
         lib.hils_set_fault_injection.restype = None
         lib.hils_version.restype = ctypes.c_char_p
-        for n in ("hils_build_summaries", "hils_score_topk", "hils_attn_prefill", "hils_attn_decode",
-                  "hils_attn_decode_noalloc", "hils_prefill_host", "hils_sync_status"):
+        for n in ("hils_build_summaries", "hils_build_summaries_shared", "hils_score_topk", "hils_attn_prefill",
+                  "hils_attn_decode", "hils_attn_decode_noalloc", "hils_prefill_host", "hils_sync_status"):
             getattr(lib, n).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -137,6 +139,12 @@ def workspace_bytes(cfg: Config, which: int, qcal_rank: int = 0) -> int:
 
 def hils_build_summaries(cfg: Config, k, q_lmk, k_sum, b_sum, stream=None):
     _check(load().hils_build_summaries(ctypes.byref(cfg), _p(k), _p(q_lmk), _p(k_sum), _p(b_sum), _stream(stream)))
+
+
+def hils_build_summaries_shared(cfg: Config, k, q_shared, k_sum, b_sum, stream=None):
+    """Landmark-free summaries: q_shared [Hq, d] is every chunk's landmark query."""
+    _check(load().hils_build_summaries_shared(ctypes.byref(cfg), _p(k), _p(q_shared), _p(k_sum), _p(b_sum),
+                                              _stream(stream)))
 
 
 def hils_score_topk(cfg: Config, q, k_sum, b_sum, idx, s_sel, workspace=None, decode=False, qcal=None, stream=None):
@@ -224,8 +232,12 @@ class Prefill:
         self.ws = alloc_workspace(workspace_bytes(cfg, HILS_WS_SCORE_PREFILL, qcal_rank), device)
         self.ws_attn = alloc_workspace(workspace_bytes(cfg, HILS_WS_ATTN_PREFILL), device)
 
-    def run(self, q, k, v, q_lmk, qcal=None, stream=None):
-        hils_build_summaries(self.cfg, k, q_lmk, self.k_sum, self.b_sum, stream)
+    def run(self, q, k, v, q_lmk, qcal=None, stream=None, shared_lmk=False):
+        """shared_lmk: q_lmk is the landmark-free variant's [Hq, d] shared query."""
+        if shared_lmk:
+            hils_build_summaries_shared(self.cfg, k, q_lmk, self.k_sum, self.b_sum, stream)
+        else:
+            hils_build_summaries(self.cfg, k, q_lmk, self.k_sum, self.b_sum, stream)
         hils_score_topk(self.cfg, q, self.k_sum, self.b_sum, self.idx, self.s_sel, self.ws, False, qcal, stream)
         hils_attn_prefill(self.cfg, q, k, v, self.idx, self.s_sel, self.out, self.ws_attn, stream)
         return self.out

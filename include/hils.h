@@ -104,6 +104,19 @@ hils_status_t hils_build_summaries(const hils_config_t* cfg, const void* k, cons
                                    float* b_sum, void* stream);
 
 /*
+ * The landmark-free variant of the summaries ([Method], last of the practical
+ * design choices: one shared learnable query per layer takes the place of the
+ * per-chunk landmark queries).  Read here as one query per query head,
+ * shared by every chunk of every sequence: q'_{h,c} = q_shared[h] in the
+ * computation of hils_build_summaries.
+ *   k      [B, Hkv, N, d]  (dtype)        q_shared [Hq, d] (dtype)
+ *   k_sum  [B, Hq, C, d]   (dtype, out)   b_sum    [B, Hq, C] (float32, out)
+ * Shapes, errors and kernels are those of hils_build_summaries.
+ */
+hils_status_t hils_build_summaries_shared(const hils_config_t* cfg, const void* k, const void* q_shared,
+                                          void* k_sum, float* b_sum, void* stream);
+
+/*
  * Chunk scoring and top-K selection, [Method] surrogate-score equation and
  * third practical design choice (GQA):
  *   s^_{h,i,c} = q~_{h,i}.k'_{h,c} * scale + b'_{h,c}   for candidates c of i,

@@ -11,6 +11,8 @@ section "方法" (Method):
 
 * :func:`summaries`  -- landmark summaries k'_c (p-weighted key sum) and
   b'_c (entropy of p), the paragraph after the surrogate-score equation;
+  :func:`summaries_shared` -- the landmark-free variant (one shared query
+  per head, the last practical design choice);
 * :func:`qcal`       -- the Q-Cal scoring query q + W_up W_down h (second
   practical design choice);
 * :func:`select`     -- surrogate score s^ = q.k'/sqrt(d) + b', GQA group max,
@@ -137,6 +139,17 @@ def summaries(dm: Dims, k, q_lmk):
     return ks, bs
 
 
+def summaries_shared(dm: Dims, k, q_shared):
+    """The landmark-free variant (Method section, last practical design
+    choice: one shared learnable query per layer instead of per-chunk landmark
+    queries), read as one query per query head [Hq, d] used by every chunk of
+    every sequence: exactly :func:`summaries` with q'_{h,c} = q_shared[h]."""
+    q_shared = _f32(q_shared)
+    assert q_shared.shape == (dm.Hq, dm.d), q_shared.shape
+    q_lmk = np.ascontiguousarray(np.broadcast_to(q_shared[None, :, None, :], (dm.B, dm.Hq, dm.C, dm.d)))
+    return summaries(dm, k, q_lmk)
+
+
 def qcal(dm: Dims, rows, q, h, w_down, w_up):
     """Q-Cal scoring queries [nrows, Hq, d] (float64) for the listed (b, position) rows."""
     lib = _load()
@@ -244,3 +257,124 @@ def union_stats(idx, M_list=(1, 2, 4, 8, 16)):
             ratios.append(len(np.unique(sel)) / K)
         out[M] = float(np.mean(ratios)) if ratios else float("nan")
     return out
+
+
+# ------------------------------------------------------------- backward ---
+# Gradients of the forward pass with the chunk selection held fixed (top-K is
+# a discrete choice).  The fusion weights exp(s^)/Z^ carry the loss into the
+# chunk scores, and from there into k', b' (the landmark summaries), q'_c and
+# the keys, and into the Q-Cal weights (Method section: the factorised w_ij and
+# Z^; the wmrh.cn article's point that the hierarchical softmax lets gradients
+# reach the summaries).  Each function is a plain restatement in the C file.
+
+def _bwd_lib():
+    lib = _load()
+    if not getattr(lib, "_bwd_ready", False):
+        P, dims_p = ctypes.c_void_p, ctypes.POINTER(_Dims)
+        lib.hils_oracle_attend_bwd.argtypes = [dims_p, P, ctypes.c_int64, P, P, P, P, P, P, P, P, P, P]
+        lib.hils_oracle_score_bwd.argtypes = [dims_p, P, ctypes.c_int64, P, P, P, P, P, P, P, P]
+        lib.hils_oracle_summaries_bwd.argtypes = [dims_p, P, P, P, P, P, P]
+        lib.hils_oracle_qcal_bwd.argtypes = [dims_p, ctypes.c_int64, ctypes.c_int64, P, ctypes.c_int64, P, P, P, P,
+                                             P, P, P]
+        for f in (lib.hils_oracle_attend_bwd, lib.hils_oracle_score_bwd, lib.hils_oracle_summaries_bwd,
+                  lib.hils_oracle_qcal_bwd):
+            f.restype = None
+        lib._bwd_ready = True
+    return lib
+
+
+def attend_bwd(dm: Dims, rows, q, k, v, idx, s_sel, dout):
+    """Attention backward for the listed rows: dq [B,Hq,nq,d] (through the
+    attention logits), dk, dv [B,Hkv,N,d] and ds_sel [nrows,Hq,K], the gradient
+    of each chosen chunk's score s^ (float64)."""
+    lib = _bwd_lib()
+    rows = _rows(rows)
+    n = rows.shape[0]
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    idx = np.ascontiguousarray(idx, np.int32).reshape(n, dm.Hkv, dm.K)
+    s_sel = np.ascontiguousarray(s_sel, np.float64).reshape(n, dm.Hq, dm.K)
+    dout = np.ascontiguousarray(dout, np.float64).reshape(n, dm.Hq, dm.d)
+    nq = dm.N if dm.nq is None else dm.nq
+    dq = np.zeros((dm.B, dm.Hq, nq, dm.d))
+    dk = np.zeros((dm.B, dm.Hkv, dm.N, dm.d))
+    dv = np.zeros((dm.B, dm.Hkv, dm.N, dm.d))
+    ds = np.zeros((n, dm.Hq, dm.K))
+    cd = dm.c()
+    lib.hils_oracle_attend_bwd(ctypes.byref(cd), _ptr(rows), n, _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(s_sel),
+                               _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ds))
+    return dq, dk, dv, ds
+
+
+def score_bwd(dm: Dims, rows, q, k_sum, idx, ds_sel, qs=None):
+    """Chunk-score backward: dqs [nrows,Hq,d] (gradient of the scoring query),
+    dk_sum [B,Hq,C,d] and db_sum [B,Hq,C] (float64)."""
+    lib = _bwd_lib()
+    rows = _rows(rows)
+    n = rows.shape[0]
+    q = _f32(q)
+    k_sum = np.ascontiguousarray(k_sum, np.float64)
+    idx = np.ascontiguousarray(idx, np.int32).reshape(n, dm.Hkv, dm.K)
+    ds_sel = np.ascontiguousarray(ds_sel, np.float64).reshape(n, dm.Hq, dm.K)
+    qs = None if qs is None else np.ascontiguousarray(qs, np.float64)
+    dqs = np.zeros((n, dm.Hq, dm.d))
+    dks = np.zeros((dm.B, dm.Hq, dm.C, dm.d))
+    dbs = np.zeros((dm.B, dm.Hq, dm.C))
+    cd = dm.c()
+    lib.hils_oracle_score_bwd(ctypes.byref(cd), _ptr(rows), n, _ptr(qs), _ptr(q), _ptr(k_sum), _ptr(idx),
+                              _ptr(ds_sel), _ptr(dqs), _ptr(dks), _ptr(dbs))
+    return dqs, dks, dbs
+
+
+def summaries_bwd(dm: Dims, k, q_lmk, dk_sum, db_sum):
+    """Summary backward: dk [B,Hkv,N,d] (through the summaries only) and
+    dq_lmk [B,Hq,C,d] (float64)."""
+    lib = _bwd_lib()
+    k, q_lmk = _f32(k), _f32(q_lmk)
+    dk_sum = np.ascontiguousarray(dk_sum, np.float64)
+    db_sum = np.ascontiguousarray(db_sum, np.float64)
+    dk = np.zeros((dm.B, dm.Hkv, dm.N, dm.d))
+    dql = np.zeros((dm.B, dm.Hq, dm.C, dm.d))
+    cd = dm.c()
+    lib.hils_oracle_summaries_bwd(ctypes.byref(cd), _ptr(k), _ptr(q_lmk), _ptr(dk_sum), _ptr(db_sum), _ptr(dk),
+                                  _ptr(dql))
+    return dk, dql
+
+
+def qcal_bwd(dm: Dims, rows, h, w_down, w_up, dqs):
+    """Q-Cal backward: dh [B,nq,Dm], dw_down [r,Dm], dw_up [Hq d, r] (float64)."""
+    lib = _bwd_lib()
+    rows = _rows(rows)
+    h, w_down, w_up = _f32(h), _f32(w_down), _f32(w_up)
+    r, Dm = w_down.shape
+    dqs = np.ascontiguousarray(dqs, np.float64)
+    dh = np.zeros(h.shape)
+    dwd = np.zeros((r, Dm))
+    dwu = np.zeros((dm.Hq * dm.d, r))
+    cd = dm.c()
+    lib.hils_oracle_qcal_bwd(ctypes.byref(cd), Dm, r, _ptr(rows), rows.shape[0], _ptr(h), _ptr(w_down), _ptr(w_up),
+                             _ptr(dqs), _ptr(dh), _ptr(dwd), _ptr(dwu))
+    return dh, dwd, dwu
+
+
+def prefill_bwd(dm: Dims, q, k, v, q_lmk, idx, dout, *, qcal_args=None):
+    """Gradients of sum(out * dout) over every position, for the selection idx
+    [B*N, Hkv, K] (rows in all_rows order) held fixed: a dict with dq, dk, dv,
+    dq_lmk (and dh, dw_down, dw_up with Q-Cal), all float64."""
+    rows = all_rows(dm.B, dm.N)
+    ks, bs = summaries(dm, k, q_lmk)
+    qs = qcal(dm, rows, q, *qcal_args) if qcal_args is not None else None
+    _, _, s_all, _ = select(dm, rows, q, k_sum=ks, b_sum=bs, qs=qs, want_all=True)
+    idx = np.ascontiguousarray(idx, np.int32).reshape(len(rows), dm.Hkv, dm.K)
+    G = dm.Hq // dm.Hkv
+    sel = np.repeat(idx, G, axis=1)
+    s_sel = np.where(sel >= 0, np.take_along_axis(s_all, np.maximum(sel, 0), axis=2), -np.inf)
+    dq, dk, dv, ds = attend_bwd(dm, rows, q, k, v, idx, s_sel, dout)
+    dqs, dks, dbs = score_bwd(dm, rows, q, ks, idx, ds, qs=qs)
+    dk2, dql = summaries_bwd(dm, k, q_lmk, dks, dbs)
+    # the scoring query is q (+ the Q-Cal term): its gradient reaches q either way
+    dq = dq + dqs.reshape(dm.B, dm.N, dm.Hq, dm.d).transpose(0, 2, 1, 3)
+    res = dict(dq=dq, dk=dk + dk2, dv=dv, dq_lmk=dql, ds_sel=ds, dk_sum=dks, db_sum=dbs, s_sel=s_sel)
+    if qcal_args is not None:
+        dh, dwd, dwu = qcal_bwd(dm, rows, *qcal_args, dqs)
+        res.update(dh=dh, dw_down=dwd, dw_up=dwu)
+    return res

@@ -1,6 +1,7 @@
 /*
  * HiLS oracle — a plain, slow, fp64 CPU restatement of Hierarchical Landmark
- * Sparse (HiLS) attention, forward pass.
+ * Sparse (HiLS) attention: the forward pass and, at the end of the file, its
+ * gradients with the chunk selection held fixed.
  *
  * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
  * call this file: only the tests, the smoke check and the CPU-baseline leg of
@@ -347,4 +348,250 @@ void hils_oracle_attend(const hils_oracle_dims *dm, const int64_t *rows, int64_t
     free(ac);
     free(ocs);
   }
+}
+
+/* ------------------------------------------------------------- backward --- */
+/*
+ * Gradients of the forward pass above, with the chunk selection held fixed
+ * (top-K is a discrete choice; gradients reach the chunk scores s^ because they
+ * enter the output through the fusion weights exp(s^)/Z^: hyper.ai summary,
+ * Method section, the factorised token weight w_ij and Z^_i; the wmrh.cn
+ * article's point that the hierarchical softmax lets the language-model loss
+ * train the summaries).  Plain serial loops: the gradient buffers accumulate
+ * across rows, so no row-parallel split.  Every output is accumulated into
+ * (callers zero it).
+ */
+
+/*
+ * Attention backward for the listed rows.  With w_u = e^{A_u}/Z^ for the
+ * window unit and every selected chunk, out = sum_u w_u O_u and D = dout.out:
+ *   window token j:   omega_j = e^{s_ij}/Z^, ds_ij = omega_j (dout.v_j - D),
+ *                     dv_j += omega_j dout;
+ *   chunk c, token j: ds_ij = w_c p_j (dout.v_j - dout.O_c),
+ *                     dv_j += w_c p_j dout,  dA_c = w_c (dout.O_c - D);
+ *   dq_i += scale sum_j ds_ij k_j,  dk_j += scale ds_ij q_i.
+ *   dout [nrows, Hq, d];  dq [B, Hq, nq, d];  dk, dv [B, Hkv, N, d];
+ *   ds_sel [nrows, Hq, K] = dA_c per slot (0 for empty slots).
+ */
+void hils_oracle_attend_bwd(const hils_oracle_dims *dm, const int64_t *rows, int64_t nrows, const float *q,
+                            const float *k, const float *v, const int32_t *idx, const double *s_sel,
+                            const double *dout, double *dq, double *dk, double *dv, double *ds_sel) {
+  const int64_t G = dm->Hq / dm->Hkv, d = dm->d, S = dm->S, K = dm->K;
+  const int64_t span = dm->W > S ? dm->W : S;
+  double *sj = (double *)malloc(sizeof(double) * (size_t)(K * S + span));
+  double *ocs = (double *)malloc(sizeof(double) * (size_t)(K * d));
+  double *ac = (double *)malloc(sizeof(double) * (size_t)K);
+  double *out = (double *)malloc(sizeof(double) * (size_t)d);
+  for (int64_t n = 0; n < nrows; ++n) {
+    const int64_t b = rows[2 * n], i = rows[2 * n + 1], iq = i - dm->q_pos0;
+    for (int64_t h = 0; h < dm->Hq; ++h) {
+      const int64_t grp = h / G;
+      const float *qi = q + ((b * dm->Hq + h) * dm->nq + iq) * d;
+      const float *kb = k + (b * dm->Hkv + grp) * dm->N * d;
+      const float *vb = v + (b * dm->Hkv + grp) * dm->N * d;
+      const double *go = dout + (n * dm->Hq + h) * d;
+      double *gq = dq + ((b * dm->Hq + h) * dm->nq + iq) * d;
+      double *gk = dk + (b * dm->Hkv + grp) * dm->N * d;
+      double *gv = dv + (b * dm->Hkv + grp) * dm->N * d;
+      const int32_t *il = idx + (n * dm->Hkv + grp) * K;
+      /* forward pieces: window logits, chunk logits and outputs, log-masses */
+      const int64_t w0 = window_start(dm, i), nwin = i - w0 + 1;
+      double *sw = sj + K * S;
+      double mw = -INFINITY;
+      for (int64_t j = 0; j < nwin; ++j) {
+        sw[j] = dm->scale * dot_fd(qi, kb + (w0 + j) * d, d);
+        if (sw[j] > mw) mw = sw[j];
+      }
+      double zw = 0.0;
+      for (int64_t j = 0; j < nwin; ++j) zw += exp(sw[j] - mw);
+      const double a_swa = mw + log(zw);
+      double m = a_swa;
+      for (int64_t s = 0; s < K; ++s) {
+        const int32_t c = il[s];
+        if (c < 0) continue;
+        double mc = -INFINITY;
+        for (int64_t j = 0; j < S; ++j) {
+          sj[s * S + j] = dm->scale * dot_fd(qi, kb + (c * S + j) * d, d);
+          if (sj[s * S + j] > mc) mc = sj[s * S + j];
+        }
+        double zc = 0.0;
+        for (int64_t j = 0; j < S; ++j) zc += exp(sj[s * S + j] - mc);
+        for (int64_t e = 0; e < d; ++e) ocs[s * d + e] = 0.0;
+        for (int64_t j = 0; j < S; ++j) {
+          const double p = exp(sj[s * S + j] - mc) / zc;
+          sj[s * S + j] = p; /* keep the intra-chunk softmax */
+          for (int64_t e = 0; e < d; ++e) ocs[s * d + e] += p * (double)vb[(c * S + j) * d + e];
+        }
+        ac[s] = s_sel[(n * dm->Hq + h) * K + s];
+        if (ac[s] > m) m = ac[s];
+      }
+      double zhat = exp(a_swa - m);
+      for (int64_t s = 0; s < K; ++s)
+        if (il[s] >= 0) zhat += exp(ac[s] - m);
+      for (int64_t e = 0; e < d; ++e) out[e] = 0.0;
+      for (int64_t j = 0; j < nwin; ++j) {
+        const double om = exp(sw[j] - m) / zhat;
+        for (int64_t e = 0; e < d; ++e) out[e] += om * (double)vb[(w0 + j) * d + e];
+      }
+      for (int64_t s = 0; s < K; ++s) {
+        if (il[s] < 0) continue;
+        const double wc = exp(ac[s] - m) / zhat;
+        for (int64_t e = 0; e < d; ++e) out[e] += wc * ocs[s * d + e];
+      }
+      double D = 0.0;
+      for (int64_t e = 0; e < d; ++e) D += go[e] * out[e];
+      /* window tokens */
+      for (int64_t j = 0; j < nwin; ++j) {
+        const int64_t t = w0 + j;
+        const double om = exp(sw[j] - m) / zhat;
+        const double gvj = dot_dd(go, vb + t * d, d);
+        const double ds = om * (gvj - D);
+        for (int64_t e = 0; e < d; ++e) {
+          gv[t * d + e] += om * go[e];
+          gq[e] += dm->scale * ds * (double)kb[t * d + e];
+          gk[t * d + e] += dm->scale * ds * (double)qi[e];
+        }
+      }
+      /* selected chunks */
+      for (int64_t s = 0; s < K; ++s) {
+        const int32_t c = il[s];
+        if (c < 0) continue;
+        const double wc = exp(ac[s] - m) / zhat;
+        double go_oc = 0.0;
+        for (int64_t e = 0; e < d; ++e) go_oc += go[e] * ocs[s * d + e];
+        ds_sel[(n * dm->Hq + h) * K + s] += wc * (go_oc - D);
+        for (int64_t j = 0; j < S; ++j) {
+          const int64_t t = c * S + j;
+          const double p = sj[s * S + j];
+          const double gvj = dot_dd(go, vb + t * d, d);
+          const double ds = wc * p * (gvj - go_oc);
+          for (int64_t e = 0; e < d; ++e) {
+            gv[t * d + e] += wc * p * go[e];
+            gq[e] += dm->scale * ds * (double)kb[t * d + e];
+            gk[t * d + e] += dm->scale * ds * (double)qi[e];
+          }
+        }
+      }
+    }
+  }
+  free(sj);
+  free(ocs);
+  free(ac);
+  free(out);
+}
+
+/*
+ * Chunk-score backward: s^_{h,i,c} = qs_{h,i}.k'_{h,c} * scale + b'_{h,c}
+ * ([M], surrogate-score equation) for the chosen chunks, so
+ *   dqs_{h,i} += scale sum_c dA_c k'_{h,c},  dk'_{h,c} += scale dA_c qs_{h,i},
+ *   db'_{h,c} += dA_c.
+ *   qs [nrows, Hq, d] (scoring queries, double), or NULL to read q;
+ *   ds_sel [nrows, Hq, K];  dqs [nrows, Hq, d];  dk_sum [B,Hq,C,d];  db_sum [B,Hq,C].
+ */
+void hils_oracle_score_bwd(const hils_oracle_dims *dm, const int64_t *rows, int64_t nrows, const double *qs,
+                           const float *q, const double *k_sum, const int32_t *idx, const double *ds_sel,
+                           double *dqs, double *dk_sum, double *db_sum) {
+  const int64_t C = n_chunks(dm), G = dm->Hq / dm->Hkv, d = dm->d, K = dm->K;
+  for (int64_t n = 0; n < nrows; ++n) {
+    const int64_t b = rows[2 * n], iq = rows[2 * n + 1] - dm->q_pos0;
+    for (int64_t h = 0; h < dm->Hq; ++h) {
+      const int32_t *il = idx + (n * dm->Hkv + h / G) * K;
+      for (int64_t s = 0; s < K; ++s) {
+        const int32_t c = il[s];
+        if (c < 0) continue;
+        const double g = ds_sel[(n * dm->Hq + h) * K + s];
+        const double *kp = k_sum + ((b * dm->Hq + h) * C + c) * d;
+        double *gkp = dk_sum + ((b * dm->Hq + h) * C + c) * d;
+        for (int64_t e = 0; e < d; ++e) {
+          const double qe = qs ? qs[(n * dm->Hq + h) * d + e] : (double)q[((b * dm->Hq + h) * dm->nq + iq) * d + e];
+          dqs[(n * dm->Hq + h) * d + e] += dm->scale * g * kp[e];
+          gkp[e] += dm->scale * g * qe;
+        }
+        db_sum[(b * dm->Hq + h) * C + c] += g;
+      }
+    }
+  }
+}
+
+/*
+ * Summary backward ([M], the landmark summary: p = softmax(q'.k_j * scale)
+ * over the chunk's keys, k' = sum_j p_j k_j, b' = -sum_j p_j log p_j):
+ *   dp_j = dk'.k_j - db' (log p_j + 1),  dl_j = p_j (dp_j - sum_m p_m dp_m),
+ *   dk_j += p_j dk' + scale dl_j q',     dq' += scale sum_j dl_j k_j.
+ *   dk_sum [B,Hq,C,d], db_sum [B,Hq,C];  dk [B,Hkv,N,d];  dq_lmk [B,Hq,C,d].
+ */
+void hils_oracle_summaries_bwd(const hils_oracle_dims *dm, const float *k, const float *q_lmk,
+                               const double *dk_sum, const double *db_sum, double *dk, double *dq_lmk) {
+  const int64_t C = n_chunks(dm), G = dm->Hq / dm->Hkv, d = dm->d, S = dm->S;
+  double *p = (double *)malloc(sizeof(double) * (size_t)S);
+  double *dl = (double *)malloc(sizeof(double) * (size_t)S);
+  for (int64_t t = 0; t < dm->B * dm->Hq * C; ++t) {
+    const int64_t c = t % C, h = (t / C) % dm->Hq, b = t / (C * dm->Hq);
+    const float *ql = q_lmk + t * d;
+    const float *kc = k + ((b * dm->Hkv + h / G) * dm->N + c * S) * d;
+    double *gkc = dk + ((b * dm->Hkv + h / G) * dm->N + c * S) * d;
+    const double *gks = dk_sum + t * d;
+    const double gb = db_sum[t];
+    double m = -INFINITY;
+    for (int64_t j = 0; j < S; ++j) {
+      p[j] = dm->scale * dot_fd(ql, kc + j * d, d);
+      if (p[j] > m) m = p[j];
+    }
+    double z = 0.0;
+    for (int64_t j = 0; j < S; ++j) z += exp(p[j] - m);
+    const double lz = m + log(z);
+    double pdp = 0.0;
+    for (int64_t j = 0; j < S; ++j) {
+      const double lp = p[j] - lz; /* log p_j */
+      p[j] = exp(lp);
+      dl[j] = dot_dd(gks, kc + j * d, d) - gb * (lp + 1.0); /* dp_j for now */
+      pdp += p[j] * dl[j];
+    }
+    for (int64_t j = 0; j < S; ++j) {
+      dl[j] = p[j] * (dl[j] - pdp);
+      for (int64_t e = 0; e < d; ++e) {
+        gkc[j * d + e] += p[j] * gks[e] + dm->scale * dl[j] * (double)ql[e];
+        dq_lmk[t * d + e] += dm->scale * dl[j] * (double)kc[j * d + e];
+      }
+    }
+  }
+  free(p);
+  free(dl);
+}
+
+/*
+ * Q-Cal backward ([M], second design choice: q~ = q + W_up (W_down h)):
+ *   t = W_down h,  dW_up += dq~ t^T,  dt = W_up^T dq~,  dW_down += dt h^T,
+ *   dh += W_down^T dt  (and dq += dq~, added by the caller).
+ *   rows [nrows,2]; h [B, nq, Dm]; w_down [r, Dm]; w_up [Hq d, r];
+ *   dqs [nrows, Hq, d]; dh [B, nq, Dm]; dw_down [r, Dm]; dw_up [Hq d, r].
+ */
+void hils_oracle_qcal_bwd(const hils_oracle_dims *dm, int64_t Dm, int64_t r, const int64_t *rows, int64_t nrows,
+                          const float *h, const float *w_down, const float *w_up, const double *dqs, double *dh,
+                          double *dw_down, double *dw_up) {
+  const int64_t E = dm->Hq * dm->d;
+  double *t = (double *)malloc(sizeof(double) * (size_t)r);
+  double *dt = (double *)malloc(sizeof(double) * (size_t)r);
+  for (int64_t n = 0; n < nrows; ++n) {
+    const int64_t b = rows[2 * n], iq = rows[2 * n + 1] - dm->q_pos0;
+    const float *hi = h + (b * dm->nq + iq) * Dm;
+    double *ghi = dh + (b * dm->nq + iq) * Dm;
+    const double *g = dqs + n * E;
+    for (int64_t a = 0; a < r; ++a) {
+      t[a] = dot_fd(w_down + a * Dm, hi, Dm);
+      dt[a] = 0.0;
+    }
+    for (int64_t e = 0; e < E; ++e)
+      for (int64_t a = 0; a < r; ++a) {
+        dw_up[e * r + a] += g[e] * t[a];
+        dt[a] += (double)w_up[e * r + a] * g[e];
+      }
+    for (int64_t a = 0; a < r; ++a)
+      for (int64_t mm = 0; mm < Dm; ++mm) {
+        dw_down[a * Dm + mm] += dt[a] * (double)hi[mm];
+        ghi[mm] += (double)w_down[a * Dm + mm] * dt[a];
+      }
+  }
+  free(t);
+  free(dt);
 }

@@ -300,3 +300,40 @@ def test_bad_list_entries_are_dropped_and_reported(chunked):
     ref = oracle.attend(dm, rows, q, k, v, clean[ridx], ssel32[ridx].astype(np.float64))
     got = to_np(out).transpose(0, 2, 1, 3).reshape(w.N, w.Hq, w.d)[ridx]
     assert np.abs(got - ref).max() <= TOL_BF16
+
+
+def test_landmark_free_summaries_and_prefill():
+    """The landmark-free variant (one shared query per head): its summaries
+    equal the per-chunk call given that query tiled over the chunks (bit for
+    bit), match the oracle, and drive an end-to-end prefill that passes the
+    selection and output checks."""
+    w = WORKLOADS["prefill_8k"].scaled(name="lmkfree", N=6144 + 40, Hq=8, Hkv=2, needles_per_head=4)
+    x = prefill_inputs(w)
+    qs = torch.randn((w.Hq, w.d), generator=torch.Generator().manual_seed(11)).to(torch.bfloat16)
+    d = {n: x[n].to(DEV) for n in ("q", "k", "v")}
+    qs_d = qs.to(DEV)
+    cfg = H.config_of(w)
+    ks_a = torch.empty((w.B, w.Hq, w.C, w.d), dtype=torch.bfloat16, device=DEV)
+    bs_a = torch.empty((w.B, w.Hq, w.C), dtype=torch.float32, device=DEV)
+    H.hils_build_summaries_shared(cfg, d["k"], qs_d, ks_a, bs_a)
+    tiled = qs_d[None, :, None, :].expand(w.B, w.Hq, w.C, w.d).contiguous()
+    ks_b, bs_b = torch.empty_like(ks_a), torch.empty_like(bs_a)
+    H.hils_build_summaries(cfg, d["k"], tiled, ks_b, bs_b)
+    H.hils_sync_status()
+    assert torch.equal(ks_a, ks_b) and torch.equal(bs_a, bs_b)
+    dm = _dims(w)
+    q, k, v = (to_np(x[n]) for n in ("q", "k", "v"))
+    ks, bs = oracle.summaries_shared(dm, k, to_np(qs))
+    assert (np.abs(to_np(ks_a) - ks) - np.abs(ks) * 2.0 ** -8).max() <= KSUM_ATOL
+    np.testing.assert_allclose(to_np(bs_a), bs, rtol=0, atol=2e-5)
+    pre = H.Prefill(cfg, DEV)
+    pre.run(d["q"], d["k"], d["v"], qs_d, shared_lmk=True)
+    H.hils_sync_status()
+    rows = sample_rows(w, x["needles"])
+    ridx = np.array([p for _, p in rows])
+    _, _, s_all, g_all = oracle.select(dm, rows, q, k_sum=ks, b_sum=bs, want_all=True)
+    idx_g = to_np(pre.idx).astype(np.int64).transpose(0, 2, 1, 3).reshape(-1, w.Hkv, w.K)[ridx]
+    check_selection(idx_g, g_all, w.K)
+    out_f = oracle.attend(dm, rows, q, k, v, idx_g, forced_s_sel(idx_g, s_all, w.G))
+    got = to_np(pre.out).transpose(0, 2, 1, 3).reshape(-1, w.Hq, w.d)[ridx]
+    assert np.abs(got - out_f).max() <= TOL_BF16

@@ -166,3 +166,18 @@ def test_bad_index_is_skipped_and_reported():
         H.hils_sync_status()
     assert ei.value.status == H.HILS_ERR_INVALID_ARG
     H.hils_sync_status()  # cleared
+
+
+def test_landmark_free_summaries_fp32():
+    """fp32 landmark-free summaries (one shared query per head) against the oracle."""
+    w = WORKLOADS["tiny_f32"]
+    x = prefill_inputs(w)
+    qs = torch.randn((w.Hq, w.d), generator=torch.Generator().manual_seed(3))
+    cfg = H.config_of(w)
+    ks_g = torch.empty((w.B, w.Hq, w.C, w.d), dtype=torch.float32, device=DEV)
+    bs_g = torch.empty((w.B, w.Hq, w.C), dtype=torch.float32, device=DEV)
+    H.hils_build_summaries_shared(cfg, x["k"].to(DEV), qs.to(DEV), ks_g, bs_g)
+    H.hils_sync_status()
+    ks, bs = oracle.summaries_shared(_dims(w), to_np(x["k"]), to_np(qs))
+    np.testing.assert_allclose(to_np(ks_g), ks, rtol=0, atol=TOL_F32)
+    np.testing.assert_allclose(to_np(bs_g), bs, rtol=0, atol=TOL_F32)

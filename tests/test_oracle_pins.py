@@ -371,3 +371,38 @@ def test_union_stats_bounds(oracle_mod):
     idx = np.array([[0, 1], [0, 1], [2, 3], [4, 5]])
     st = oracle_mod.union_stats(idx, (1, 2, 4))
     assert st[1] == 1.0 and st[2] == 1.5 and st[4] == 3.0
+
+
+def test_landmark_free_zero_query_is_mean_pool(oracle_mod):
+    """Landmark-free variant with the shared query 0: every chunk's p is uniform,
+    so b' = log S and k' = the chunk's mean key (the mean-pool case)."""
+    dm, q, k, v, ql = _small()
+    ks, bs = oracle_mod.summaries_shared(dm, k, np.zeros((dm.Hq, dm.d), np.float32))
+    np.testing.assert_allclose(bs, math.log(dm.S), rtol=0, atol=1e-12)
+    kk = k.astype(np.float64).reshape(dm.B, dm.Hkv, dm.C, dm.S, dm.d).mean(3)
+    G = dm.Hq // dm.Hkv
+    for h in range(dm.Hq):
+        np.testing.assert_allclose(ks[:, h], kk[:, h // G], rtol=0, atol=1e-12)
+
+
+def test_landmark_free_same_keys_same_summary(oracle_mod):
+    """One query shared by all chunks: two chunks holding the same keys (in any
+    order) get the same k' and b'; with per-chunk queries they would not."""
+    dm, q, k, v, ql = _small()
+    G = dm.Hq // dm.Hkv
+    k = k.copy()
+    perm = RNG.permutation(dm.S)
+    k[:, :, dm.S:2 * dm.S] = k[:, :, :dm.S][:, :, perm]
+    qs = _rand(dm.Hq, dm.d)
+    ks, bs = oracle_mod.summaries_shared(dm, k, qs)
+    np.testing.assert_allclose(ks[:, :, 1], ks[:, :, 0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(bs[:, :, 1], bs[:, :, 0], rtol=0, atol=1e-12)
+    # the shared query is the landmark query of head h for every chunk: check one
+    # chunk of one head against its definition, the softmax-weighted key sum
+    h, c = 1, 3
+    kc = k[0, h // G, c * dm.S:(c + 1) * dm.S].astype(np.float64)
+    l = kc @ qs[h].astype(np.float64) / math.sqrt(dm.d)
+    p = np.exp(l - l.max())
+    p /= p.sum()
+    np.testing.assert_allclose(ks[0, h, c], p @ kc, rtol=0, atol=1e-12)
+    assert abs(bs[0, h, c] + (p * np.log(p)).sum()) < 1e-12
