@@ -398,6 +398,67 @@ def prefill_roofline(w, pre, ev, pk, pk_kind):
     return roofline, per_kernel
 
 
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # SMs x fp32 lanes x FMA x max clock (74.4)
+
+
+def backward_flops(w):
+    """Algorithmic FLOP of the prefill backward (selection held fixed), per
+    (position, query head): 10 d per attended key (recompute s and dout.v, then
+    dq, dk, dv: five d-long products) + 4 d per chosen chunk (score path), and
+    8 S d per (query head, chunk) for the summary backward."""
+    nw = w.W // w.S
+    tot = 0
+    for i in range(w.N):
+        cur = i // w.S
+        cand = max(0, cur - nw + 1)
+        win = i - max(0, (cur - nw + 1) * w.S) + 1
+        sel = min(w.K, cand)
+        tot += 10 * w.d * (sel * w.S + win) + 4 * w.d * sel
+    return tot * w.B * w.Hq + 8 * w.S * w.d * w.B * w.Hq * w.C
+
+
+def bench_backward(w, dev, stream, args, ws, dist_on):
+    """hils_prefill_bwd after a forward of the same workload: W >= 3 untimed
+    calls, then K calls between CUDA events (max over ranks)."""
+    x = prefill_inputs(w, device=dev)
+    cfg = H.config_of(w)
+    pre = H.Prefill(cfg, dev)
+    with torch.cuda.stream(stream):
+        pre.run(x["q"], x["k"], x["v"], x["q_lmk"], stream=stream)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1)
+    dout = torch.randn(x["q"].shape, generator=gen, device=dev).to(x["q"].dtype)
+    f32 = dict(dtype=torch.float32, device=dev)
+    grads = [torch.empty((w.B, w.Hq, w.N, w.d), **f32), torch.empty((w.B, w.Hkv, w.N, w.d), **f32),
+             torch.empty((w.B, w.Hkv, w.N, w.d), **f32), torch.empty((w.B, w.Hq, w.C, w.d), **f32)]
+    wsb = H.alloc_workspace(H.workspace_bytes(cfg, H.HILS_WS_PREFILL_BWD), dev)
+
+    def step():
+        H.hils_prefill_bwd(cfg, x["q"], x["k"], x["v"], x["q_lmk"], pre.idx, pre.s_sel, pre.k_sum, dout, *grads,
+                           wsb, stream=stream)
+
+    steps = max(2, args.steps // 3)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    H.hils_sync_status(stream)
+    ms = device_time(stream, step, steps, dist_on) / steps
+    H.hils_sync_status(stream)
+    fl = backward_flops(w)
+    ach = fl / (ms / 1e3) / 1e12
+    out = {"workload": w.name, "value": round(whole_job_rate(w.B * w.N, ws, ms), 1), "unit": "tokens/s",
+           "ms_per_call": round(ms, 3), "steps": steps, "warmup": args.warmup,
+           "roofline": {"kernel": "hils_prefill_bwd (bwd_rows_kernel + bwd_keys_kernel + bucketing)", "bound": "alu",
+                        "achieved": round(ach, 2), "peak": round(FP32_ALU_TFLOPS, 1), "unit": "TFLOP/s",
+                        "frac": round(ach / FP32_ALU_TFLOPS, 4), "traffic": None,
+                        "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz",
+                        "algorithmic_flop_per_launch": fl},
+           "gpu_launches": 5 * steps}
+    del x, pre, grads, wsb
+    torch.cuda.empty_cache()
+    return out
+
+
 def extra_prefill(w, dev, stream, args, ws, dist_on, pk, pk_kind):
     """Another prefill workload timed the same way (device-resident inputs,
     W >= 3 warm-up steps, K timed steps between CUDA events, max over ranks),
@@ -432,6 +493,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-qcal", action="store_true", help="skip the 512K Q-Cal prefill reported beside the line")
+    ap.add_argument("--no-bwd", action="store_true", help="skip the prefill backward reported beside the line")
+    ap.add_argument("--bwd-workload", default="prefill_8k", choices=[k for k, v in WORKLOADS.items() if not v.decode])
     ap.add_argument("--seq-len", type=int, default=0, help="override N of the prefill workload (profiling)")
     ap.add_argument("--decode-seq-len", type=int, default=0, help="override L of the decode workload (profiling)")
     args = ap.parse_args()
@@ -505,6 +568,8 @@ def main():
     if not args.no_qcal and args.workload != "prefill_512k_qcal" and not args.seq_len:
         line["prefill_512k_qcal"] = extra_prefill(WORKLOADS["prefill_512k_qcal"], dev, stream, args, ws, dist_on, pk,
                                                   pk_kind)
+    if not args.no_bwd:
+        line["backward"] = bench_backward(WORKLOADS[args.bwd_workload], dev, stream, args, ws, dist_on)
     if rank == 0 and not args.no_cpu:
         v, done, t_s, t_r = cpu_baseline_prefill(w, x)
         line["cpu_baseline"] = {"value": round(v, 2), "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",

@@ -59,7 +59,16 @@ bool aligned16(const void* p) { return p && ((uintptr_t)p & 15u) == 0; }
 
 // The operations whose shape coverage is checked on the host, before any
 // launch: a shape no kernel serves returns HILS_ERR_UNSUPPORTED.
-enum Op { kOpSummaries, kOpScorePrefill, kOpScoreDecode, kOpAttnPrefill, kOpAttnDecode, kOpPrefillHost, kOpNone };
+enum Op {
+  kOpSummaries,
+  kOpScorePrefill,
+  kOpScoreDecode,
+  kOpAttnPrefill,
+  kOpAttnDecode,
+  kOpPrefillHost,
+  kOpPrefillBwd,
+  kOpNone
+};
 
 // Kernel coverage per operation (the dispatchers in the .cu files serve
 // exactly these shapes; anything else would reach no kernel).
@@ -76,6 +85,7 @@ const char* uncovered(const Shape& s, Op op) {
       case kOpSummaries: return summ ? nullptr : "f32 summaries: no kernel for d = 32 with S = 64";
       case kOpScorePrefill: return score ? nullptr : "f32 prefill scoring: no kernel for d = 128 with G = 8";
       case kOpAttnDecode: return dec ? nullptr : "f32 decode attention needs d in {64, 128} and S in {32, 64}";
+      case kOpPrefillBwd: return nullptr;
       case kOpPrefillHost:
         if (!summ) return "f32 summaries: no kernel for d = 32 with S = 64";
         return score ? nullptr : "f32 prefill scoring: no kernel for d = 128 with G = 8";
@@ -287,6 +297,7 @@ size_t hils_workspace_bytes(const hils_config_t* cfg, int32_t which, int32_t qca
                 : which == HILS_WS_ATTN_DECODE  ? kOpAttnDecode
                 : which == HILS_WS_PREFILL_HOST ? kOpPrefillHost
                 : which == HILS_WS_ATTN_PREFILL ? kOpAttnPrefill
+                : which == HILS_WS_PREFILL_BWD  ? kOpPrefillBwd
                                                 : kOpNone;
   if (op == kOpNone) {
     fail(HILS_ERR_INVALID_ARG, "unknown workspace kind %d", which);
@@ -308,6 +319,8 @@ size_t hils_workspace_bytes(const hils_config_t* cfg, int32_t which, int32_t qca
       return host_layout(s, qcal_rank > 0 ? qcal_rank : 0).total;
     case HILS_WS_ATTN_PREFILL:
       return s.dtype == HILS_BF16 ? attn_prefill_tc_workspace(s) : 0;
+    case HILS_WS_PREFILL_BWD:
+      return prefill_bwd_workspace(s);
   }
   return (size_t)-1;
 }
@@ -382,6 +395,27 @@ hils_status_t hils_attn_prefill(const hils_config_t* cfg, const void* q, const v
   } else {
     HILS_LAUNCH(launch_attn_prefill_tc(s, q, k, v, idx, s_sel, out, st, ctx), "attn_prefill_tc");
   }
+  return HILS_OK;
+}
+
+hils_status_t hils_prefill_bwd(const hils_config_t* cfg, const void* q, const void* k, const void* v,
+                               const void* q_lmk, const int32_t* idx, const float* s_sel, const void* k_sum,
+                               const void* dout, float* dq, float* dk, float* dv, float* dq_lmk, float* ds_sel,
+                               void* workspace, size_t ws_bytes, void* stream) {
+  Shape s;
+  HILS_TRY(make_shape(cfg, &s, kOpPrefillBwd));
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_lmk) || !aligned16(idx) || !aligned16(s_sel) ||
+      !aligned16(k_sum) || !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      !aligned16(dq_lmk) || (ds_sel && !aligned16(ds_sel)))
+    return fail(HILS_ERR_INVALID_ARG, "hils_prefill_bwd: NULL or unaligned pointer");
+  const size_t need = prefill_bwd_workspace(s);
+  if (ws_bytes < need || !aligned16(workspace))
+    return fail(HILS_ERR_INVALID_ARG, "hils_prefill_bwd: workspace needs %zu bytes (got %zu)", need, ws_bytes);
+  DevCtx ctx;
+  HILS_TRY(dev_ctx(&ctx));
+  HILS_LAUNCH(launch_prefill_bwd(s, q, k, v, q_lmk, idx, s_sel, k_sum, dout, dq, dk, dv, dq_lmk, ds_sel, workspace,
+                                 (cudaStream_t)stream, ctx),
+              "prefill_bwd");
   return HILS_OK;
 }
 

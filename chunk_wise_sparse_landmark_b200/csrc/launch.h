@@ -72,4 +72,12 @@ cudaError_t launch_attn_decode_static(const Shape& s, const void* q, const void*
                                       const int32_t* idx, const float* s_sel, void* out, cudaStream_t st,
                                       const DevCtx& ctx);
 
+// backward of the prefill (attention, scores, summaries), CUDA-core kernels;
+// workspace of prefill_bwd_workspace(s) bytes; ds_sel may be null
+size_t prefill_bwd_workspace(const Shape& s);
+cudaError_t launch_prefill_bwd(const Shape& s, const void* q, const void* k, const void* v, const void* q_lmk,
+                               const int32_t* idx, const float* s_sel, const void* k_sum, const void* dout, float* dq,
+                               float* dk, float* dv, float* dq_lmk, float* ds_sel, void* ws, cudaStream_t st,
+                               const DevCtx& ctx);
+
 }  // namespace hils

@@ -17,7 +17,8 @@ LIB_PATH = os.path.join(_PKG, "libhils.so")
 
 HILS_OK, HILS_ERR_INVALID_ARG, HILS_ERR_UNSUPPORTED, HILS_ERR_CUDA, HILS_ERR_TIMEOUT = range(5)
 HILS_F32, HILS_BF16 = 0, 1
-HILS_WS_SCORE_PREFILL, HILS_WS_SCORE_DECODE, HILS_WS_ATTN_DECODE, HILS_WS_PREFILL_HOST, HILS_WS_ATTN_PREFILL = range(5)
+(HILS_WS_SCORE_PREFILL, HILS_WS_SCORE_DECODE, HILS_WS_ATTN_DECODE, HILS_WS_PREFILL_HOST, HILS_WS_ATTN_PREFILL,
+ HILS_WS_PREFILL_BWD) = range(6)
 
 EXPORTS = (
     "hils_build_summaries",
@@ -27,6 +28,7 @@ EXPORTS = (
     "hils_attn_decode",
     "hils_attn_decode_noalloc",
     "hils_prefill_host",
+    "hils_prefill_bwd",
     "hils_workspace_bytes",
     "hils_sync_status",
     "hils_last_error",
@@ -86,6 +88,7 @@ def load() -> ctypes.CDLL:
         lib.hils_attn_decode.argtypes = [C, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         lib.hils_attn_decode_noalloc.argtypes = [C, P, P, P, P, P, P, P]
         lib.hils_prefill_host.argtypes = [C, P, P, P, P, ctypes.POINTER(QCal), P, P, ctypes.c_size_t, P]
+        lib.hils_prefill_bwd.argtypes = [C, P, P, P, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         lib.hils_workspace_bytes.argtypes = [C, ctypes.c_int32, ctypes.c_int32]
         lib.hils_workspace_bytes.restype = ctypes.c_size_t
         lib.hils_sync_status.argtypes = [P]
@@ -96,7 +99,8 @@ def load() -> ctypes.CDLL:
         lib.hils_set_fault_injection.restype = None
         lib.hils_version.restype = ctypes.c_char_p
         for n in ("hils_build_summaries", "hils_build_summaries_shared", "hils_score_topk", "hils_attn_prefill",
-                  "hils_attn_decode", "hils_attn_decode_noalloc", "hils_prefill_host", "hils_sync_status"):
+                  "hils_attn_decode", "hils_attn_decode_noalloc", "hils_prefill_host", "hils_prefill_bwd",
+                  "hils_sync_status"):
             getattr(lib, n).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -164,6 +168,16 @@ def hils_attn_prefill(cfg: Config, q, k, v, idx, s_sel, out, workspace=None, str
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(load().hils_attn_prefill(ctypes.byref(cfg), _p(q), _p(k), _p(v), _p(idx), _p(s_sel), _p(out),
                                     _p(workspace), ws_bytes, _stream(stream)))
+
+
+def hils_prefill_bwd(cfg: Config, q, k, v, q_lmk, idx, s_sel, k_sum, dout, dq, dk, dv, dq_lmk, workspace,
+                     ds_sel=None, stream=None):
+    """Gradients of the prefill (float32 outputs dq, dk, dv, dq_lmk and
+    optionally ds_sel), selection held fixed; see include/hils.h."""
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(load().hils_prefill_bwd(ctypes.byref(cfg), _p(q), _p(k), _p(v), _p(q_lmk), _p(idx), _p(s_sel), _p(k_sum),
+                                   _p(dout), _p(dq), _p(dk), _p(dv), _p(dq_lmk), _p(ds_sel), _p(workspace), ws_bytes,
+                                   _stream(stream)))
 
 
 def _ph(t: torch.Tensor):

@@ -253,12 +253,43 @@ hils_status_t hils_prefill_host(const hils_config_t* cfg, const void* h_q, const
                                 const void* h_q_lmk, const hils_qcal_t* qcal, void* h_out, void* workspace,
                                 size_t ws_bytes, void* stream);
 
+/*
+ * Backward of the prefill: gradients of a loss L with respect to q, k, v and
+ * the landmark queries, given dL/dout, with the chunk selection idx held fixed
+ * (top-K is a discrete choice).  [Method], the factorised token weight w_ij
+ * and Z^_i: the loss reaches each chosen chunk's score s^ through its fusion
+ * weight exp(s^)/Z^, and from s^ = q.k'/sqrt(d) + b' the landmark summaries
+ * k', b' and their queries q'_c (the wmrh.cn article on HiLS: the hierarchical
+ * softmax lets the language-model loss train the summaries).  The scoring
+ * query is q (no Q-Cal).
+ *   q [B,Hq,N,d], k, v [B,Hkv,N,d], q_lmk [B,Hq,C,d], k_sum [B,Hq,C,d] (dtype):
+ *     the forward's inputs and its summaries;
+ *   idx [B,Hkv,N,K], s_sel [B,Hq,N,K]: the forward's selection and scores
+ *     (lists in the form of hils_attn_prefill, checked the same way);
+ *   dout [B,Hq,N,d] (dtype): dL/dout.
+ * Outputs, float32, overwritten: dq [B,Hq,N,d] (attention logits and score
+ * path), dk, dv [B,Hkv,N,d] (attention, and for dk the summaries),
+ * dq_lmk [B,Hq,C,d]; ds_sel [B,Hq,N,K] = dL/ds^ per chosen slot (0 elsewhere),
+ * or NULL.  Kernels: CUDA cores, fp32 arithmetic, no floating-point atomics
+ * on global memory.  dq and ds_sel repeat bit for bit; dk, dv and dq_lmk sum
+ * a chunk's rows in the order of its bucket list (filled by atomic arrival),
+ * so repeats agree to fp32 rounding.  workspace: at least
+ * hils_workspace_bytes(cfg, HILS_WS_PREFILL_BWD, 0) bytes.  Shapes: those of
+ * the forward's summaries and attention for the dtype (fp32: d in
+ * {32, 64, 128}; bf16: d = 128, S = 64), any G.
+ */
+hils_status_t hils_prefill_bwd(const hils_config_t* cfg, const void* q, const void* k, const void* v,
+                               const void* q_lmk, const int32_t* idx, const float* s_sel, const void* k_sum,
+                               const void* dout, float* dq, float* dk, float* dv, float* dq_lmk, float* ds_sel,
+                               void* workspace, size_t ws_bytes, void* stream);
+
 enum {
   HILS_WS_SCORE_PREFILL = 0,
   HILS_WS_SCORE_DECODE = 1,
   HILS_WS_ATTN_DECODE = 2,
   HILS_WS_PREFILL_HOST = 3,
-  HILS_WS_ATTN_PREFILL = 4
+  HILS_WS_ATTN_PREFILL = 4,
+  HILS_WS_PREFILL_BWD = 5
 };
 
 /* Bytes of workspace the call `which` needs for this configuration (0 if none);
