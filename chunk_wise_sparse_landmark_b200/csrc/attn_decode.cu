@@ -49,18 +49,23 @@ __global__ void __launch_bounds__(kThreads) attn_decode_partial(Shape s, const T
                                                                 const T* __restrict__ k, const T* __restrict__ v,
                                                                 const int32_t* __restrict__ idx,
                                                                 const float* __restrict__ s_sel,
-                                                                float* __restrict__ ws, int nsplit, DevCtx ctx) {
+                                                                float* __restrict__ ws, int nsplit, DecView dv, DevCtx ctx) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   auto& sm = *reinterpret_cast<DecSmem<T, D, S, G>*>(smem_raw);
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int L = s.N, pos = L - 1, cur = pos / S;
+  int L = dv_len(dv, s, b);
+  const bool len_ok = L >= 1 && L <= s.N;  // invalid: reported, no units (the record stays empty)
+  if (!len_ok) {
+    if (tid == 0) raise_status(ctx, kStatusBadIndex);
+    L = 1;
+  }
+  const int pos = L - 1, cur = pos / S;
   const int ncand = max(0, cur - s.nw + 1);
   const int wc0 = max(0, cur - s.nw + 1);        // first window chunk
   const int nwin = cur - wc0 + 1;                 // window tiles
-  const int nunits = s.K + nwin;
+  const int nunits = len_ok ? s.K + nwin : 0;
   const int32_t* ir = idx + ((long long)b * s.Hkv + g) * s.K;
-  const long long kvbase = ((long long)b * s.Hkv + g) * (long long)L * D;
 
   for (int e = tid; e < G * D; e += kThreads)
     sm.qs[e / D][e % D] = to_f32(q[((long long)b * s.Hq + g * G + e / D) * D + e % D]);
@@ -72,7 +77,7 @@ __global__ void __launch_bounds__(kThreads) attn_decode_partial(Shape s, const T
   __syncthreads();
 
   // this CTA's units: u = split, split + nsplit, ... ; resolve each to a key range
-  auto unit_keys = [&](int u, int& j0, int& nk, bool& sel, int& slot) -> bool {
+  auto unit_keys = [&](int u, long long& off, int& nk, bool& sel, int& slot) -> bool {
     if (u < s.K) {
       const int c = ir[u];
       sel = true;
@@ -81,26 +86,30 @@ __global__ void __launch_bounds__(kThreads) attn_decode_partial(Shape s, const T
         if (c != -1 && tid == 0) raise_status(ctx, kStatusBadIndex);
         return false;
       }
-      j0 = c * S;
+      off = dv_chunk(dv, s, b, g, c);
       nk = S;
-      return true;
+    } else {
+      const int wc = wc0 + (u - s.K);
+      sel = false;
+      slot = -1;
+      off = dv_chunk(dv, s, b, g, wc);
+      nk = min(S, L - wc * S);
     }
-    const int wc = wc0 + (u - s.K);
-    sel = false;
-    slot = -1;
-    j0 = wc * S;
-    nk = min(S, L - j0);
+    if (off < 0) {  // a page outside the pool: reported, never read
+      if (tid == 0) raise_status(ctx, kStatusBadIndex);
+      return false;
+    }
     return true;
   };
   bool inflight[2] = {false, false};  // meaningful in thread 0
-  auto issue = [&](int stage, int j0, int nk) {
+  auto issue = [&](int stage, long long off, int nk) {
     if (ctx.inject == 1) return;  // test hook: no copy, the wait below must run out
     inflight[stage] = true;
     fence_proxy_async_shared();
     const uint32_t bytes = (uint32_t)(nk * D * sizeof(T));
     mbar_arrive_expect_tx(&sm.full[stage], 2 * bytes);
-    tma_load_1d(sm.kt[stage], k + kvbase + (long long)j0 * D, bytes, &sm.full[stage]);
-    tma_load_1d(sm.vt[stage], v + kvbase + (long long)j0 * D, bytes, &sm.full[stage]);
+    tma_load_1d(sm.kt[stage], k + off, bytes, &sm.full[stage]);
+    tma_load_1d(sm.vt[stage], v + off, bytes, &sm.full[stage]);
   };
 
   // running fold per head, thread (h, e) owns num for dims e, e + 128 ... via loop
@@ -119,13 +128,15 @@ __global__ void __launch_bounds__(kThreads) attn_decode_partial(Shape s, const T
   int ulist[16];
   int nu = 0;
   for (int u = split; u < nunits && nu < 16; u += nsplit) {
-    int j0, nk, slot;
+    long long j0;
+    int nk, slot;
     bool sel;
     if (unit_keys(u, j0, nk, sel, slot)) ulist[nu++] = u;
   }
   uint32_t phase[2] = {0u, 0u};
   if (tid == 0 && nu > 0) {
-    int j0, nk, slot;
+    long long j0;
+    int nk, slot;
     bool sel;
     unit_keys(ulist[0], j0, nk, sel, slot);
     issue(0, j0, nk);
@@ -133,11 +144,13 @@ __global__ void __launch_bounds__(kThreads) attn_decode_partial(Shape s, const T
   bool alive = true;  // CTA-wide: every thread sees the same value
   for (int x = 0; x < nu; ++x) {
     const int stage = x & 1;
-    int j0, nk, slot;
+    long long j0;
+    int nk, slot;
     bool sel;
     unit_keys(ulist[x], j0, nk, sel, slot);
     if (tid == 0 && x + 1 < nu) {
-      int j0n, nkn, sln;
+      long long j0n;
+      int nkn, sln;
       bool seln;
       unit_keys(ulist[x + 1], j0n, nkn, seln, sln);
       issue(stage ^ 1, j0n, nkn);
@@ -265,19 +278,24 @@ __global__ void __launch_bounds__(kMmaWarps * 32) attn_decode_mma(Shape s, const
                                                                   const __nv_bfloat16* __restrict__ v,
                                                                   const int32_t* __restrict__ idx,
                                                                   const float* __restrict__ s_sel,
-                                                                  float* __restrict__ ws, int nsplit, DevCtx ctx) {
+                                                                  float* __restrict__ ws, int nsplit, DecView dv, DevCtx ctx) {
   constexpr int D = 128, S = 64;
   __shared__ float red_acc[kMmaWarps][G][D];
   __shared__ float red_m[kMmaWarps][G], red_d[kMmaWarps][G];
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gq = lane >> 2, c4 = lane & 3;
-  const int L = s.N, pos = L - 1, cur = pos / S;
+  int L = dv_len(dv, s, b);
+  const bool len_ok = L >= 1 && L <= s.N;  // invalid: reported, no units (the record stays empty)
+  if (!len_ok) {
+    if (threadIdx.x == 0) raise_status(ctx, kStatusBadIndex);
+    L = 1;
+  }
+  const int pos = L - 1, cur = pos / S;
   const int ncand = max(0, cur - s.nw + 1);
   const int wc0 = max(0, cur - s.nw + 1);
-  const int nunits = s.K + (cur - wc0 + 1);
+  const int nunits = len_ok ? s.K + (cur - wc0 + 1) : 0;
   const int32_t* ir = idx + ((long long)b * s.Hkv + g) * s.K;
-  const long long kvbase = ((long long)b * s.Hkv + g) * (long long)L * D;
   // Q^T as the B operand of S^T: column gq = head gq (zero past G)
   uint32_t qf[2][8];
   load_qcol(gq < G ? q + ((long long)b * s.Hq + g * G + gq) * D : nullptr, c4, qf);
@@ -289,7 +307,8 @@ __global__ void __launch_bounds__(kMmaWarps * 32) attn_decode_mma(Shape s, const
 
   // units of this CTA: u = split + nsplit * t; of this warp: every kMmaWarps-th of those
   for (int u = split + nsplit * warp; u < nunits; u += nsplit * kMmaWarps) {
-    int j0, nk;
+    int nk;
+    long long off;
     bool sel;
     int slot = -1;
     if (u < s.K) {
@@ -300,15 +319,20 @@ __global__ void __launch_bounds__(kMmaWarps * 32) attn_decode_mma(Shape s, const
       }
       sel = true;
       slot = u;
-      j0 = c * S;
+      off = dv_chunk(dv, s, b, g, c);
       nk = S;
     } else {
       sel = false;
-      j0 = (wc0 + (u - s.K)) * S;
-      nk = min(S, L - j0);
+      const int wc = wc0 + (u - s.K);
+      off = dv_chunk(dv, s, b, g, wc);
+      nk = min(S, L - wc * S);
     }
-    const __nv_bfloat16* kc = k + kvbase + (long long)j0 * D;
-    const __nv_bfloat16* vc = v + kvbase + (long long)j0 * D;
+    if (off < 0) {  // a page outside the pool: reported, never read
+      if (lane == 0) raise_status(ctx, kStatusBadIndex);
+      continue;
+    }
+    const __nv_bfloat16* kc = k + off;
+    const __nv_bfloat16* vc = v + off;
     const int kmax = nk - 1;
     float sc[4][4];
 #pragma unroll
@@ -407,10 +431,11 @@ __global__ void __launch_bounds__(kMmaWarps * 32) attn_decode_mma(Shape s, const
 
 template <int G>
 cudaError_t go_mma(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
-                   const float* s_sel, void* out, void* ws, int nsplit, cudaStream_t st, const DevCtx& ctx) {
+                   const float* s_sel, void* out, void* ws, int nsplit, cudaStream_t st, const DevCtx& ctx,
+                   const DecView& dv) {
   attn_decode_mma<G><<<dim3(nsplit, s.Hkv, s.B), kMmaWarps * 32, 0, st>>>(
       s, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, idx, s_sel, (float*)ws, nsplit,
-      ctx);
+      dv, ctx);
   attn_decode_merge<__nv_bfloat16, 128><<<s.B * s.Hq, 128, 0, st>>>(s, (const float*)ws, (__nv_bfloat16*)out,
                                                                      nsplit);
   return cudaGetLastError();
@@ -431,26 +456,26 @@ int pick_nsplit(const Shape& s) {
 
 template <typename T, int D, int S, int G>
 cudaError_t go(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx, const float* s_sel,
-               void* out, void* ws, cudaStream_t st, const DevCtx& ctx) {
+               void* out, void* ws, cudaStream_t st, const DevCtx& ctx, const DecView& dv) {
   const int nsplit = pick_nsplit(s);
   const size_t smem = sizeof(DecSmem<T, D, S, G>);
   auto kern = attn_decode_partial<T, D, S, G>;
   cudaError_t e = ensure_dynamic_smem((const void*)kern, (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<dim3(nsplit, s.Hkv, s.B), kThreads, smem, st>>>(s, (const T*)q, (const T*)k, (const T*)v, idx, s_sel,
-                                                         (float*)ws, nsplit, ctx);
+                                                         (float*)ws, nsplit, dv, ctx);
   attn_decode_merge<T, D><<<s.B * s.Hq, D, 0, st>>>(s, (const float*)ws, (T*)out, nsplit);
   return cudaGetLastError();
 }
 
 template <typename T, int D, int S>
 cudaError_t go_g(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx, const float* s_sel,
-                 void* out, void* ws, cudaStream_t st, const DevCtx& ctx) {
+                 void* out, void* ws, cudaStream_t st, const DevCtx& ctx, const DecView& dv) {
   switch (s.G) {
-    case 1: return go<T, D, S, 1>(s, q, k, v, idx, s_sel, out, ws, st, ctx);
-    case 2: return go<T, D, S, 2>(s, q, k, v, idx, s_sel, out, ws, st, ctx);
-    case 4: return go<T, D, S, 4>(s, q, k, v, idx, s_sel, out, ws, st, ctx);
-    case 8: return go<T, D, S, 8>(s, q, k, v, idx, s_sel, out, ws, st, ctx);
+    case 1: return go<T, D, S, 1>(s, q, k, v, idx, s_sel, out, ws, st, ctx, dv);
+    case 2: return go<T, D, S, 2>(s, q, k, v, idx, s_sel, out, ws, st, ctx, dv);
+    case 4: return go<T, D, S, 4>(s, q, k, v, idx, s_sel, out, ws, st, ctx, dv);
+    case 8: return go<T, D, S, 8>(s, q, k, v, idx, s_sel, out, ws, st, ctx, dv);
   }
   return cudaErrorNotSupported;
 }
@@ -469,19 +494,20 @@ size_t decode_attn_workspace(const Shape& s) {
 }
 
 cudaError_t launch_attn_decode(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
-                               const float* s_sel, void* out, void* ws, cudaStream_t st, const DevCtx& ctx) {
+                               const float* s_sel, void* out, void* ws, cudaStream_t st, const DevCtx& ctx,
+                               const DecView& dv) {
   if (s.dtype == 0) {
-    if (s.d == 64 && s.S == 32) return go_g<float, 64, 32>(s, q, k, v, idx, s_sel, out, ws, st, ctx);
-    if (s.d == 64 && s.S == 64) return go_g<float, 64, 64>(s, q, k, v, idx, s_sel, out, ws, st, ctx);
-    if (s.d == 128 && s.S == 64) return go_g<float, 128, 64>(s, q, k, v, idx, s_sel, out, ws, st, ctx);
-    if (s.d == 128 && s.S == 32) return go_g<float, 128, 32>(s, q, k, v, idx, s_sel, out, ws, st, ctx);
+    if (s.d == 64 && s.S == 32) return go_g<float, 64, 32>(s, q, k, v, idx, s_sel, out, ws, st, ctx, dv);
+    if (s.d == 64 && s.S == 64) return go_g<float, 64, 64>(s, q, k, v, idx, s_sel, out, ws, st, ctx, dv);
+    if (s.d == 128 && s.S == 64) return go_g<float, 128, 64>(s, q, k, v, idx, s_sel, out, ws, st, ctx, dv);
+    if (s.d == 128 && s.S == 32) return go_g<float, 128, 32>(s, q, k, v, idx, s_sel, out, ws, st, ctx, dv);
   } else if (s.d == 128 && s.S == 64) {
     const int nsplit = pick_nsplit(s);
     switch (s.G) {
-      case 1: return go_mma<1>(s, q, k, v, idx, s_sel, out, ws, nsplit, st, ctx);
-      case 2: return go_mma<2>(s, q, k, v, idx, s_sel, out, ws, nsplit, st, ctx);
-      case 4: return go_mma<4>(s, q, k, v, idx, s_sel, out, ws, nsplit, st, ctx);
-      case 8: return go_mma<8>(s, q, k, v, idx, s_sel, out, ws, nsplit, st, ctx);
+      case 1: return go_mma<1>(s, q, k, v, idx, s_sel, out, ws, nsplit, st, ctx, dv);
+      case 2: return go_mma<2>(s, q, k, v, idx, s_sel, out, ws, nsplit, st, ctx, dv);
+      case 4: return go_mma<4>(s, q, k, v, idx, s_sel, out, ws, nsplit, st, ctx, dv);
+      case 8: return go_mma<8>(s, q, k, v, idx, s_sel, out, ws, nsplit, st, ctx, dv);
     }
   }
   return cudaErrorNotSupported;
@@ -512,7 +538,7 @@ cudaError_t launch_attn_decode_static(const Shape& s, const void* q, const void*
     }
     ws = addr[dev];
   }
-  return launch_attn_decode(s, q, k, v, idx, s_sel, out, ws, st, ctx);
+  return launch_attn_decode(s, q, k, v, idx, s_sel, out, ws, st, ctx, DecView{});
 }
 
 }  // namespace hils

@@ -581,6 +581,95 @@ hils_status_t hils_attn_decode_noalloc(const hils_config_t* cfg, const void* q, 
   return HILS_OK;
 }
 
+// host checks of a paged-cache description; its device arrays are checked by
+// the kernels (lengths in [1, N], pages inside the pool)
+static hils_status_t paged_view(const Shape& s, const hils_paged_t* pg, DecView* dv) {
+  if (!pg) return fail(HILS_ERR_INVALID_ARG, "paged cache description is NULL");
+  if (!pg->seq_lens || ((uintptr_t)pg->seq_lens & 3u) || !pg->block_table || ((uintptr_t)pg->block_table & 3u))
+    return fail(HILS_ERR_INVALID_ARG, "paged cache: NULL or unaligned seq_lens / block_table");
+  const int need = (s.N + s.S - 1) / s.S;
+  if (pg->max_pages < need)
+    return fail(HILS_ERR_INVALID_ARG, "paged cache: max_pages %d < ceil(seq_len / S) = %d", pg->max_pages, need);
+  if (pg->num_pages < 1) return fail(HILS_ERR_INVALID_ARG, "paged cache: num_pages %d < 1", pg->num_pages);
+  dv->seq_lens = pg->seq_lens;
+  dv->pages = pg->block_table;
+  dv->max_pages = pg->max_pages;
+  dv->num_pages = pg->num_pages;
+  return HILS_OK;
+}
+
+hils_status_t hils_decode_append(const hils_config_t* cfg, const hils_paged_t* paged, const void* k_new,
+                                 const void* v_new, const void* q_lmk_new, void* k_pool, void* v_pool, void* k_sum,
+                                 float* b_sum, void* stream) {
+  Shape s;
+  HILS_TRY(make_shape(cfg, &s, kOpSummaries));
+  DecView dv;
+  HILS_TRY(paged_view(s, paged, &dv));
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(q_lmk_new) || !aligned16(k_pool) || !aligned16(v_pool) ||
+      !aligned16(k_sum) || !aligned16(b_sum))
+    return fail(HILS_ERR_INVALID_ARG, "hils_decode_append: NULL or unaligned pointer");
+  DevCtx ctx;
+  HILS_TRY(dev_ctx(&ctx));
+  cudaStream_t st = (cudaStream_t)stream;
+  HILS_LAUNCH(launch_decode_append(s, k_new, v_new, k_pool, v_pool, dv, st, ctx), "decode_append");
+  HILS_LAUNCH(launch_summaries_paged(s, k_pool, q_lmk_new, k_sum, b_sum, dv, true, st, ctx), "summaries_paged");
+  return HILS_OK;
+}
+
+hils_status_t hils_build_summaries_paged(const hils_config_t* cfg, const hils_paged_t* paged, const void* k_pool,
+                                         const void* q_lmk, void* k_sum, float* b_sum, void* stream) {
+  Shape s;
+  HILS_TRY(make_shape(cfg, &s, kOpSummaries));
+  DecView dv;
+  HILS_TRY(paged_view(s, paged, &dv));
+  if (!aligned16(k_pool) || !aligned16(q_lmk) || !aligned16(k_sum) || !aligned16(b_sum))
+    return fail(HILS_ERR_INVALID_ARG, "hils_build_summaries_paged: NULL or unaligned pointer");
+  DevCtx ctx;
+  HILS_TRY(dev_ctx(&ctx));
+  HILS_LAUNCH(launch_summaries_paged(s, k_pool, q_lmk, k_sum, b_sum, dv, false, (cudaStream_t)stream, ctx),
+              "summaries_paged");
+  return HILS_OK;
+}
+
+hils_status_t hils_score_topk_paged(const hils_config_t* cfg, const void* q, const hils_paged_t* paged,
+                                    const void* k_sum, const float* b_sum, int32_t* idx, float* s_sel,
+                                    void* workspace, size_t ws_bytes, void* stream) {
+  Shape s;
+  HILS_TRY(make_shape(cfg, &s, kOpScoreDecode));
+  DecView dv;
+  HILS_TRY(paged_view(s, paged, &dv));
+  if (!aligned16(q) || !aligned16(k_sum) || !aligned16(b_sum) || !aligned16(idx) || !aligned16(s_sel))
+    return fail(HILS_ERR_INVALID_ARG, "hils_score_topk_paged: NULL or unaligned pointer");
+  const size_t need = decode_score_workspace(s);
+  if (ws_bytes < need || !aligned16(workspace))
+    return fail(HILS_ERR_INVALID_ARG, "hils_score_topk_paged: workspace needs %zu bytes (got %zu)", need, ws_bytes);
+  DevCtx ctx;
+  HILS_TRY(dev_ctx(&ctx));
+  HILS_LAUNCH(launch_score_topk_decode(s, q, k_sum, b_sum, idx, s_sel, workspace, (cudaStream_t)stream, ctx, dv),
+              "score_topk_paged");
+  return HILS_OK;
+}
+
+hils_status_t hils_attn_decode_paged(const hils_config_t* cfg, const void* q, const void* k_pool, const void* v_pool,
+                                     const hils_paged_t* paged, const int32_t* idx, const float* s_sel, void* out,
+                                     void* workspace, size_t ws_bytes, void* stream) {
+  Shape s;
+  HILS_TRY(make_shape(cfg, &s, kOpAttnDecode));
+  DecView dv;
+  HILS_TRY(paged_view(s, paged, &dv));
+  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(idx) || !aligned16(s_sel) ||
+      !aligned16(out))
+    return fail(HILS_ERR_INVALID_ARG, "hils_attn_decode_paged: NULL or unaligned pointer");
+  const size_t need = decode_attn_workspace(s);
+  if (ws_bytes < need || !aligned16(workspace))
+    return fail(HILS_ERR_INVALID_ARG, "hils_attn_decode_paged: workspace needs %zu bytes (got %zu)", need, ws_bytes);
+  DevCtx ctx;
+  HILS_TRY(dev_ctx(&ctx));
+  HILS_LAUNCH(launch_attn_decode(s, q, k_pool, v_pool, idx, s_sel, out, workspace, (cudaStream_t)stream, ctx, dv),
+              "attn_decode_paged");
+  return HILS_OK;
+}
+
 hils_status_t hils_sync_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");

@@ -142,7 +142,7 @@ cudaError_t go_prefill(const Shape& s, const void* q, const void* k_sum, const f
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(256) decode_scores(Shape s, const T* __restrict__ q, const T* __restrict__ k_sum,
                                                      const float* __restrict__ b_sum, float* __restrict__ s_all,
-                                                     float* __restrict__ g_all, int ncand) {
+                                                     float* __restrict__ g_all, int ncand_max, DecView dv) {
   // lane layout: LPR lanes per (chunk, head) row (16 for d = 128: 8 elements each)
   constexpr int LPR = D / 8 >= 32 ? 32 : D / 8;  // lanes per row
   constexpr int EPL = D / LPR;                    // elements per lane
@@ -152,6 +152,9 @@ __global__ void __launch_bounds__(256) decode_scores(Shape s, const T* __restric
   constexpr int U = (sizeof(T) == 2 && EPL == 8) ? (G >= 8 ? 2 : 16 / G) : 1;
   __shared__ float qs[G][D];
   const int g = blockIdx.y, b = blockIdx.z;
+  // candidates of this sequence's token at L - 1 (an out-of-range L has none)
+  const int L = dv_len(dv, s, b);
+  const int ncand = (L >= 1 && L <= s.N) ? min(ncand_max, max(0, (L - 1) / s.S - s.nw + 1)) : 0;
   for (int e = threadIdx.x; e < G * D; e += blockDim.x)
     qs[e / D][e % D] = to_f32(q[((long long)b * s.Hq + g * G + e / D) * D + e % D]);
   __syncthreads();
@@ -225,7 +228,8 @@ constexpr int kSelThreads = 1024;
 template <int G>
 __global__ void __launch_bounds__(kSelThreads) decode_select(Shape s, const float* __restrict__ s_all,
                                                              const float* __restrict__ g_all, int32_t* __restrict__ idx,
-                                                             float* __restrict__ s_sel, int ncand) {
+                                                             float* __restrict__ s_sel, int ncand_max, DecView dv,
+                                                             DevCtx ctx) {
   __shared__ unsigned hist[256];
   __shared__ unsigned prefix_sh, need_sh;
   __shared__ int sel[64];
@@ -233,6 +237,9 @@ __global__ void __launch_bounds__(kSelThreads) decode_select(Shape s, const floa
   __shared__ unsigned scan[kSelThreads];
   const int g = blockIdx.x % s.Hkv, b = blockIdx.x / s.Hkv;
   const int tid = threadIdx.x;
+  const int L = dv_len(dv, s, b);
+  if ((L < 1 || L > s.N) && tid == 0) raise_status(ctx, kStatusBadIndex);
+  const int ncand = (L >= 1 && L <= s.N) ? min(ncand_max, max(0, (L - 1) / s.S - s.nw + 1)) : 0;
   const float* gr = g_all + ((long long)b * s.Hkv + g) * s.C;
   const int K = s.K;
   if (tid == 0) nsel_sh = 0;
@@ -382,7 +389,7 @@ __global__ void __launch_bounds__(kSelThreads) decode_select(Shape s, const floa
 
 template <typename T, int D, int G>
 cudaError_t go_decode(const Shape& s, const void* q, const void* k_sum, const float* b_sum, int32_t* idx,
-                      float* s_sel, void* ws, cudaStream_t st) {
+                      float* s_sel, void* ws, cudaStream_t st, const DevCtx& ctx, const DecView& dv) {
   const int cur = (s.N - 1) / s.S;
   const int ncand = max(0, cur - s.nw + 1);
   float* s_all = (float*)ws;
@@ -396,20 +403,20 @@ cudaError_t go_decode(const Shape& s, const void* q, const void* k_sum, const fl
     const int want = (sms * 8 + s.B * s.Hkv - 1) / (s.B * s.Hkv);
     if (gx > want) gx = want;
     decode_scores<T, D, G><<<dim3(gx, s.Hkv, s.B), 256, 0, st>>>(s, (const T*)q, (const T*)k_sum, b_sum, s_all,
-                                                                  g_all, ncand);
+                                                                  g_all, ncand, dv);
   }
-  decode_select<G><<<s.B * s.Hkv, kSelThreads, 0, st>>>(s, s_all, g_all, idx, s_sel, ncand);
+  decode_select<G><<<s.B * s.Hkv, kSelThreads, 0, st>>>(s, s_all, g_all, idx, s_sel, ncand, dv, ctx);
   return cudaGetLastError();
 }
 
 template <typename T, int D>
 cudaError_t go_decode_g(const Shape& s, const void* q, const void* k_sum, const float* b_sum, int32_t* idx,
-                        float* s_sel, void* ws, cudaStream_t st) {
+                        float* s_sel, void* ws, cudaStream_t st, const DevCtx& ctx, const DecView& dv) {
   switch (s.G) {
-    case 1: return go_decode<T, D, 1>(s, q, k_sum, b_sum, idx, s_sel, ws, st);
-    case 2: return go_decode<T, D, 2>(s, q, k_sum, b_sum, idx, s_sel, ws, st);
-    case 4: return go_decode<T, D, 4>(s, q, k_sum, b_sum, idx, s_sel, ws, st);
-    case 8: return go_decode<T, D, 8>(s, q, k_sum, b_sum, idx, s_sel, ws, st);
+    case 1: return go_decode<T, D, 1>(s, q, k_sum, b_sum, idx, s_sel, ws, st, ctx, dv);
+    case 2: return go_decode<T, D, 2>(s, q, k_sum, b_sum, idx, s_sel, ws, st, ctx, dv);
+    case 4: return go_decode<T, D, 4>(s, q, k_sum, b_sum, idx, s_sel, ws, st, ctx, dv);
+    case 8: return go_decode<T, D, 8>(s, q, k_sum, b_sum, idx, s_sel, ws, st, ctx, dv);
   }
   return cudaErrorNotSupported;
 }
@@ -432,13 +439,14 @@ size_t decode_score_workspace(const Shape& s) {
 }
 
 cudaError_t launch_score_topk_decode(const Shape& s, const void* q, const void* k_sum, const float* b_sum,
-                                     int32_t* idx, float* s_sel, void* ws, cudaStream_t st, const DevCtx&) {
+                                     int32_t* idx, float* s_sel, void* ws, cudaStream_t st, const DevCtx& ctx,
+                                     const DecView& dv) {
   if (s.dtype == 0) {
-    if (s.d == 32) return go_decode_g<float, 32>(s, q, k_sum, b_sum, idx, s_sel, ws, st);
-    if (s.d == 64) return go_decode_g<float, 64>(s, q, k_sum, b_sum, idx, s_sel, ws, st);
-    if (s.d == 128) return go_decode_g<float, 128>(s, q, k_sum, b_sum, idx, s_sel, ws, st);
+    if (s.d == 32) return go_decode_g<float, 32>(s, q, k_sum, b_sum, idx, s_sel, ws, st, ctx, dv);
+    if (s.d == 64) return go_decode_g<float, 64>(s, q, k_sum, b_sum, idx, s_sel, ws, st, ctx, dv);
+    if (s.d == 128) return go_decode_g<float, 128>(s, q, k_sum, b_sum, idx, s_sel, ws, st, ctx, dv);
   } else {
-    if (s.d == 128) return go_decode_g<__nv_bfloat16, 128>(s, q, k_sum, b_sum, idx, s_sel, ws, st);
+    if (s.d == 128) return go_decode_g<__nv_bfloat16, 128>(s, q, k_sum, b_sum, idx, s_sel, ws, st, ctx, dv);
   }
   return cudaErrorNotSupported;
 }

@@ -28,20 +28,51 @@ struct LmkStrides {
   HILS_DI long long of(int bb, int hh, int cc) const { return bb * b + hh * h + cc * c; }
 };
 
+// Which chunks a launch summarises.  kAllChunks: every complete chunk of a
+// contiguous cache [B, Hkv, N, d].  kPagedAll: every complete chunk of each
+// sequence of a paged cache (units over max_pages, those past the sequence's
+// length skipped).  kPagedLast: the chunk that the last token of each sequence
+// completed, if it completed one (length % S == 0), with its landmark query
+// given per sequence (chunk stride 0 in LmkStrides).
+enum SummUnits { kAllChunks = 0, kPagedAll = 1, kPagedLast = 2 };
+
 template <typename T, int D, int S, int G>
 __global__ void __launch_bounds__(kThreads) summaries_kernel(Shape s, const T* __restrict__ k,
                                                              const T* __restrict__ q_lmk, LmkStrides ls,
-                                                             T* __restrict__ k_sum, float* __restrict__ b_sum) {
+                                                             T* __restrict__ k_sum, float* __restrict__ b_sum,
+                                                             DecView dv, int mode, DevCtx ctx) {
   __shared__ float ks[S][D + 1];
   __shared__ float qs[G][D];
   __shared__ float lg[G][S];
   const int tid = threadIdx.x;
-  const long long units = (long long)s.B * s.Hkv * s.C;
+  const int per = mode == kAllChunks ? s.C : mode == kPagedAll ? dv.max_pages : 1;
+  const long long units = (long long)s.B * s.Hkv * per;
   for (long long u = blockIdx.x; u < units; u += gridDim.x) {
-    const int c = (int)(u % s.C);
-    const int g = (int)((u / s.C) % s.Hkv);
-    const int b = (int)(u / ((long long)s.C * s.Hkv));
-    const T* kc = k + (((long long)b * s.Hkv + g) * s.N + (long long)c * S) * D;
+    int c = (int)(u % per);
+    const int g = (int)((u / per) % s.Hkv);
+    const int b = (int)(u / ((long long)per * s.Hkv));
+    long long koff;
+    if (mode == kAllChunks) {
+      koff = (((long long)b * s.Hkv + g) * s.N + (long long)c * S) * D;
+    } else {
+      const int L = dv_len(dv, s, b);
+      if (L < 1 || L > s.N) {
+        if (tid == 0 && g == 0 && c == 0) raise_status(ctx, kStatusBadIndex);
+        continue;
+      }
+      if (mode == kPagedLast) {
+        if (L % S) continue;  // the last token completed no chunk
+        c = L / S - 1;
+      } else if (c >= L / S) {
+        continue;  // not a complete chunk of this sequence
+      }
+      koff = dv_chunk(dv, s, b, g, c);
+      if (koff < 0) {  // a page outside the pool: reported, never read
+        if (tid == 0) raise_status(ctx, kStatusBadIndex);
+        continue;
+      }
+    }
+    const T* kc = k + koff;
     for (int e = tid; e < S * D; e += kThreads) ks[e / D][e % D] = to_f32(kc[e]);
     for (int e = tid; e < G * D; e += kThreads) {
       const int hg = e / D;
@@ -90,33 +121,34 @@ __global__ void __launch_bounds__(kThreads) summaries_kernel(Shape s, const T* _
 
 template <typename T, int D, int S, int G>
 cudaError_t go(const Shape& s, const void* k, const void* q_lmk, const LmkStrides& ls, void* k_sum, float* b_sum,
-               cudaStream_t st) {
-  const long long units = (long long)s.B * s.Hkv * s.C;
+               cudaStream_t st, const DevCtx& ctx, const DecView& dv = DecView{}, int mode = kAllChunks) {
+  const int per = mode == kAllChunks ? s.C : mode == kPagedAll ? dv.max_pages : 1;
+  const long long units = (long long)s.B * s.Hkv * per;
   if (units == 0) return cudaSuccess;
   const int sms = device_sm_count();
   const long long grid = units < (long long)sms * 8 ? units : (long long)sms * 8;
   summaries_kernel<T, D, S, G><<<(unsigned)grid, kThreads, 0, st>>>(s, (const T*)k, (const T*)q_lmk, ls, (T*)k_sum,
-                                                                     b_sum);
+                                                                     b_sum, dv, mode, ctx);
   return cudaGetLastError();
 }
 
 template <typename T, int D, int S>
 cudaError_t go_g(const Shape& s, const void* k, const void* q_lmk, const LmkStrides& ls, void* k_sum, float* b_sum,
-                 cudaStream_t st) {
+                 cudaStream_t st, const DevCtx& ctx, const DecView& dv, int mode) {
   switch (s.G) {
-    case 1: return go<T, D, S, 1>(s, k, q_lmk, ls, k_sum, b_sum, st);
-    case 2: return go<T, D, S, 2>(s, k, q_lmk, ls, k_sum, b_sum, st);
-    case 4: return go<T, D, S, 4>(s, k, q_lmk, ls, k_sum, b_sum, st);
-    case 8: return go<T, D, S, 8>(s, k, q_lmk, ls, k_sum, b_sum, st);
+    case 1: return go<T, D, S, 1>(s, k, q_lmk, ls, k_sum, b_sum, st, ctx, dv, mode);
+    case 2: return go<T, D, S, 2>(s, k, q_lmk, ls, k_sum, b_sum, st, ctx, dv, mode);
+    case 4: return go<T, D, S, 4>(s, k, q_lmk, ls, k_sum, b_sum, st, ctx, dv, mode);
+    case 8: return go<T, D, S, 8>(s, k, q_lmk, ls, k_sum, b_sum, st, ctx, dv, mode);
   }
   return cudaErrorNotSupported;
 }
 
 template <typename T>
 cudaError_t go_t(const Shape& s, const void* k, const void* q_lmk, const LmkStrides& ls, void* k_sum, float* b_sum,
-                 cudaStream_t st) {
+                 cudaStream_t st, const DevCtx& ctx, const DecView& dv = DecView{}, int mode = kAllChunks) {
 #define HILS_CASE(DD, SS) \
-  if (s.d == DD && s.S == SS) return go_g<T, DD, SS>(s, k, q_lmk, ls, k_sum, b_sum, st);
+  if (s.d == DD && s.S == SS) return go_g<T, DD, SS>(s, k, q_lmk, ls, k_sum, b_sum, st, ctx, dv, mode);
   HILS_CASE(64, 32)
   HILS_CASE(64, 64)
   HILS_CASE(128, 32)
@@ -241,11 +273,11 @@ cudaError_t go_mma(const Shape& s, const void* k, const void* q_lmk, const LmkSt
 }  // namespace
 
 cudaError_t launch_summaries(const Shape& s, const void* k, const void* q_lmk, void* k_sum, float* b_sum,
-                             cudaStream_t st, const DevCtx&, bool shared_lmk) {
+                             cudaStream_t st, const DevCtx& ctx, bool shared_lmk) {
   // per-chunk landmark queries [B, Hq, C, d], or one shared query per head [Hq, d]
   const LmkStrides ls = shared_lmk ? LmkStrides{0, (long long)s.d, 0}
                                    : LmkStrides{(long long)s.Hq * s.C * s.d, (long long)s.C * s.d, (long long)s.d};
-  if (s.dtype == 0) return go_t<float>(s, k, q_lmk, ls, k_sum, b_sum, st);
+  if (s.dtype == 0) return go_t<float>(s, k, q_lmk, ls, k_sum, b_sum, st, ctx);
   if (s.d == 128 && s.S == 64) {
     switch (s.G) {
       case 1: return go_mma<1>(s, k, q_lmk, ls, k_sum, b_sum, st);
@@ -254,7 +286,17 @@ cudaError_t launch_summaries(const Shape& s, const void* k, const void* q_lmk, v
       case 8: return go_mma<8>(s, k, q_lmk, ls, k_sum, b_sum, st);
     }
   }
-  return go_t<__nv_bfloat16>(s, k, q_lmk, ls, k_sum, b_sum, st);
+  return go_t<__nv_bfloat16>(s, k, q_lmk, ls, k_sum, b_sum, st, ctx);
+}
+
+cudaError_t launch_summaries_paged(const Shape& s, const void* k_pool, const void* q_lmk, void* k_sum, float* b_sum,
+                                   const DecView& dv, bool last_only, cudaStream_t st, const DevCtx& ctx) {
+  // every chunk: q_lmk [B, Hq, C, d]; the chunk the last token completed: q_lmk [B, Hq, d]
+  const LmkStrides ls = last_only ? LmkStrides{(long long)s.Hq * s.d, (long long)s.d, 0}
+                                  : LmkStrides{(long long)s.Hq * s.C * s.d, (long long)s.C * s.d, (long long)s.d};
+  const int mode = last_only ? kPagedLast : kPagedAll;
+  if (s.dtype == 0) return go_t<float>(s, k_pool, q_lmk, ls, k_sum, b_sum, st, ctx, dv, mode);
+  return go_t<__nv_bfloat16>(s, k_pool, q_lmk, ls, k_sum, b_sum, st, ctx, dv, mode);
 }
 
 }  // namespace hils

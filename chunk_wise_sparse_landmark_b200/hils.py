@@ -29,6 +29,10 @@ EXPORTS = (
     "hils_attn_decode_noalloc",
     "hils_prefill_host",
     "hils_prefill_bwd",
+    "hils_decode_append",
+    "hils_build_summaries_paged",
+    "hils_score_topk_paged",
+    "hils_attn_decode_paged",
     "hils_workspace_bytes",
     "hils_sync_status",
     "hils_last_error",
@@ -70,6 +74,16 @@ class QCal(ctypes.Structure):
     ]
 
 
+class Paged(ctypes.Structure):
+    """A paged, chunk-aligned decode cache (include/hils.h, hils_paged_t)."""
+    _fields_ = [
+        ("seq_lens", ctypes.c_void_p),
+        ("block_table", ctypes.c_void_p),
+        ("max_pages", ctypes.c_int32),
+        ("num_pages", ctypes.c_int32),
+    ]
+
+
 _lib = None
 
 
@@ -89,6 +103,11 @@ def load() -> ctypes.CDLL:
         lib.hils_attn_decode_noalloc.argtypes = [C, P, P, P, P, P, P, P]
         lib.hils_prefill_host.argtypes = [C, P, P, P, P, ctypes.POINTER(QCal), P, P, ctypes.c_size_t, P]
         lib.hils_prefill_bwd.argtypes = [C, P, P, P, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+        PG = ctypes.POINTER(Paged)
+        lib.hils_decode_append.argtypes = [C, PG, P, P, P, P, P, P, P, P]
+        lib.hils_build_summaries_paged.argtypes = [C, PG, P, P, P, P, P]
+        lib.hils_score_topk_paged.argtypes = [C, P, PG, P, P, P, P, P, ctypes.c_size_t, P]
+        lib.hils_attn_decode_paged.argtypes = [C, P, P, P, PG, P, P, P, P, ctypes.c_size_t, P]
         lib.hils_workspace_bytes.argtypes = [C, ctypes.c_int32, ctypes.c_int32]
         lib.hils_workspace_bytes.restype = ctypes.c_size_t
         lib.hils_sync_status.argtypes = [P]
@@ -100,7 +119,8 @@ def load() -> ctypes.CDLL:
         lib.hils_version.restype = ctypes.c_char_p
         for n in ("hils_build_summaries", "hils_build_summaries_shared", "hils_score_topk", "hils_attn_prefill",
                   "hils_attn_decode", "hils_attn_decode_noalloc", "hils_prefill_host", "hils_prefill_bwd",
-                  "hils_sync_status"):
+                  "hils_decode_append", "hils_build_summaries_paged", "hils_score_topk_paged",
+                  "hils_attn_decode_paged", "hils_sync_status"):
             getattr(lib, n).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -178,6 +198,34 @@ def hils_prefill_bwd(cfg: Config, q, k, v, q_lmk, idx, s_sel, k_sum, dout, dq, d
     _check(load().hils_prefill_bwd(ctypes.byref(cfg), _p(q), _p(k), _p(v), _p(q_lmk), _p(idx), _p(s_sel), _p(k_sum),
                                    _p(dout), _p(dq), _p(dk), _p(dv), _p(dq_lmk), _p(ds_sel), _p(workspace), ws_bytes,
                                    _stream(stream)))
+
+
+def paged(seq_lens, block_table, num_pages: int) -> Paged:
+    """seq_lens [B] and block_table [B, max_pages] are int32 CUDA tensors."""
+    assert seq_lens.dtype == torch.int32 and block_table.dtype == torch.int32
+    return Paged(_p(seq_lens).value, _p(block_table).value, block_table.shape[1], num_pages)
+
+
+def hils_decode_append(cfg: Config, pg: Paged, k_new, v_new, q_lmk_new, k_pool, v_pool, k_sum, b_sum, stream=None):
+    _check(load().hils_decode_append(ctypes.byref(cfg), ctypes.byref(pg), _p(k_new), _p(v_new), _p(q_lmk_new),
+                                     _p(k_pool), _p(v_pool), _p(k_sum), _p(b_sum), _stream(stream)))
+
+
+def hils_build_summaries_paged(cfg: Config, pg: Paged, k_pool, q_lmk, k_sum, b_sum, stream=None):
+    _check(load().hils_build_summaries_paged(ctypes.byref(cfg), ctypes.byref(pg), _p(k_pool), _p(q_lmk), _p(k_sum),
+                                             _p(b_sum), _stream(stream)))
+
+
+def hils_score_topk_paged(cfg: Config, q, pg: Paged, k_sum, b_sum, idx, s_sel, workspace, stream=None):
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(load().hils_score_topk_paged(ctypes.byref(cfg), _p(q), ctypes.byref(pg), _p(k_sum), _p(b_sum), _p(idx),
+                                        _p(s_sel), _p(workspace), ws_bytes, _stream(stream)))
+
+
+def hils_attn_decode_paged(cfg: Config, q, k_pool, v_pool, pg: Paged, idx, s_sel, out, workspace, stream=None):
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(load().hils_attn_decode_paged(ctypes.byref(cfg), _p(q), _p(k_pool), _p(v_pool), ctypes.byref(pg), _p(idx),
+                                         _p(s_sel), _p(out), _p(workspace), ws_bytes, _stream(stream)))
 
 
 def _ph(t: torch.Tensor):

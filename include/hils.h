@@ -3,7 +3,8 @@
  * Sparse (HiLS) attention on NVIDIA B200 (sm_100a).
  *
  * Source of the method: the hyper.ai summary of arXiv 2607.02980
- * (HiLS-Attention), section "方法" (Method); cited below as [Method].
+ * (HiLS-Attention), section "方法" (Method); cited below as [Method];
+ * section "实验" (Experiments) of the same page is cited as [Exp].
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -217,6 +218,60 @@ hils_status_t hils_attn_decode(const hils_config_t* cfg, const void* q, const vo
 hils_status_t hils_attn_decode_noalloc(const hils_config_t* cfg, const void* q, const void* k_cache,
                                        const void* v_cache, const int32_t* idx, const float* s_sel, void* out,
                                        void* stream);
+
+/*
+ * Decode across steps on a paged, chunk-aligned KV cache, for sequences of
+ * different lengths.  [Exp]: decode latency grows sublinearly with context
+ * because a step touches only the token's K chunks and its window; so a cache
+ * that grows by one token per step needs only the new token's key and value
+ * written into place and, when that token completes a chunk, the summary of
+ * that one chunk (no rebuild of the cache's summaries).
+ *
+ * The cache is a pool of one-chunk pages, k_pool / v_pool [num_pages, Hkv, S, d]
+ * (dtype): chunk c of sequence b lives in page block_table[b * max_pages + c],
+ * so one chunk of one KV head is one contiguous S x d tile.  cfg->seq_len is
+ * the capacity L_max (it sets C = L_max / S, the chunk dimension of k_sum and
+ * b_sum); sequence b has length seq_lens[b] in [1, L_max], its new token at
+ * position seq_lens[b] - 1.  All arrays are device memory owned by the caller.
+ * Checked on the device: a length outside [1, L_max] or a page outside
+ * [0, num_pages) is skipped and reported (HILS_ERR_INVALID_ARG from
+ * hils_sync_status()); never dereferenced.
+ */
+typedef struct {
+  const int32_t* seq_lens;    /* [B] cache length of each sequence, new token included */
+  const int32_t* block_table; /* [B, max_pages] pool page of chunk c of sequence b */
+  int32_t max_pages;          /* >= ceil(cfg->seq_len / S) */
+  int32_t num_pages;          /* pages in the pool */
+} hils_paged_t;
+
+/* Append one token per sequence: k_new, v_new [B, Hkv, d] go to position
+ * seq_lens[b] - 1 of their pages (seq_lens already counts them).  If that
+ * position ends a chunk (seq_lens[b] % S == 0), the chunk's summary is built
+ * with its landmark query q_lmk_new[b] ([B, Hq, d]) into
+ * k_sum [B, Hq, C, d] and b_sum [B, Hq, C] at chunk seq_lens[b] / S - 1
+ * (the computation of hils_build_summaries for that chunk). */
+hils_status_t hils_decode_append(const hils_config_t* cfg, const hils_paged_t* paged, const void* k_new,
+                                 const void* v_new, const void* q_lmk_new, void* k_pool, void* v_pool, void* k_sum,
+                                 float* b_sum, void* stream);
+
+/* Summaries of every complete chunk of each sequence of a paged cache
+ * (q_lmk [B, Hq, C, d]; chunks past a sequence's length are left untouched),
+ * e.g. after a prefill written into the pool. */
+hils_status_t hils_build_summaries_paged(const hils_config_t* cfg, const hils_paged_t* paged, const void* k_pool,
+                                         const void* q_lmk, void* k_sum, float* b_sum, void* stream);
+
+/* hils_score_topk (decode = 1) for sequences of the given lengths: the
+ * candidates of sequence b are its complete chunks before the window of
+ * position seq_lens[b] - 1.  Workspace: HILS_WS_SCORE_DECODE. */
+hils_status_t hils_score_topk_paged(const hils_config_t* cfg, const void* q, const hils_paged_t* paged,
+                                    const void* k_sum, const float* b_sum, int32_t* idx, float* s_sel,
+                                    void* workspace, size_t ws_bytes, void* stream);
+
+/* hils_attn_decode on the paged cache, each sequence at its own length.
+ * Workspace: HILS_WS_ATTN_DECODE. */
+hils_status_t hils_attn_decode_paged(const hils_config_t* cfg, const void* q, const void* k_pool, const void* v_pool,
+                                     const hils_paged_t* paged, const int32_t* idx, const float* s_sel, void* out,
+                                     void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * The whole prefill path from host memory: copies the inputs to the device,
