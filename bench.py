@@ -459,6 +459,84 @@ def bench_backward(w, dev, stream, args, ws, dist_on):
     return out
 
 
+def bench_decode_offload(dev, stream, args, ws, dist_on):
+    """Decode attention with the KV cache in page-locked host memory (the
+    summaries stay on the device): the kernel reads the token's K chunks and
+    window over the host link.  Workload: the decode workload's shapes at 4
+    sequences of 128K (2 x 1 GiB of pinned host cache)."""
+    w = WORKLOADS["decode_512k"].scaled(name="decode_offload_4x128k", B=4, N=131072)
+    x = decode_inputs(w, device=dev)
+    cfg = H.config_of(w)
+    dec = H.Decode(cfg, dev)
+    with torch.cuda.stream(stream):
+        dec.summarize(x["k"], x["q_lmk"], stream)
+        dec.step(x["q"], x["k"], x["v"], stream)
+    H.hils_sync_status(stream)
+    kh, vh = x["k"].cpu().pin_memory(), x["v"].cpu().pin_memory()
+    del x["k"], x["v"]
+    kp, vp = H.hils_host_device_pointer(kh), H.hils_host_device_pointer(vh)
+
+    def step():
+        H.hils_attn_decode(cfg, x["q"], kp, vp, dec.idx, dec.s_sel, dec.out, dec.ws_attn, stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    H.hils_sync_status(stream)
+    n = args.steps * 5
+    ms = device_time(stream, step, n, dist_on) / n
+    H.hils_sync_status(stream)
+    _, gb, _ = decode_bytes(w)
+    out = {"workload": w.name, "attn_decode_ms": round(ms, 4), "link_gbs": round(gb / (ms / 1e3) / 1e9, 1),
+           "bytes_per_step": gb, "cache_bytes_on_host": 2 * kh.numel() * kh.element_size(),
+           "note": "KV cache in pinned host memory; only the selected chunks and the window cross the link",
+           "gpu_launches": 2 * n}
+    del kh, vh, dec, x
+    torch.cuda.empty_cache()
+    return out
+
+
+def dense_comparator(dev, stream, reps=2):
+    """Dense causal attention of the same shapes on this GPU, for context only:
+    the pages quote HiLS against full attention (13.5x prefill and 15.7x decode
+    at 512K, hardware not stated).  This is a library kernel (torch's scaled
+    dot-product attention, GQA, bf16), not part of the path; it times one
+    attention call per shape, L2 not flushed (inputs far larger than L2)."""
+    import torch.nn.functional as F
+
+    res = {}
+    shapes = {"prefill_128k": (1, 32, 8, 131072), "prefill_512k": (1, 32, 8, 524288)}
+    for name, (B, Hq, Hkv, N) in shapes.items():
+        g = torch.Generator(device=dev)
+        g.manual_seed(9)
+        q = torch.randn((B, Hq, N, 128), generator=g, device=dev, dtype=torch.bfloat16)
+        k = torch.randn((B, Hkv, N, 128), generator=g, device=dev, dtype=torch.bfloat16)
+        v = torch.randn((B, Hkv, N, 128), generator=g, device=dev, dtype=torch.bfloat16)
+        with torch.cuda.stream(stream):
+            F.scaled_dot_product_attention(q, k, v, is_causal=True, enable_gqa=True)
+        ms = device_time(stream, lambda: F.scaled_dot_product_attention(q, k, v, is_causal=True, enable_gqa=True),
+                         reps, False) / reps
+        flop = 4 * 128 * B * Hq * N * (N + 1) / 2
+        res[name] = {"ms": round(ms, 3), "tflops": round(flop / (ms / 1e3) / 1e12, 1)}
+        del q, k, v
+    # decode: one query per sequence over a 512K cache, 16 sequences
+    B, Hq, Hkv, L = 16, 32, 8, 524288
+    g = torch.Generator(device=dev)
+    g.manual_seed(10)
+    q = torch.randn((B, Hq, 1, 128), generator=g, device=dev, dtype=torch.bfloat16)
+    k = torch.randn((B, Hkv, L, 128), generator=g, device=dev, dtype=torch.bfloat16)
+    v = torch.randn((B, Hkv, L, 128), generator=g, device=dev, dtype=torch.bfloat16)
+    with torch.cuda.stream(stream):
+        F.scaled_dot_product_attention(q, k, v, enable_gqa=True)
+    ms = device_time(stream, lambda: F.scaled_dot_product_attention(q, k, v, enable_gqa=True), reps * 5, False) / (
+        reps * 5)
+    res["decode_512k"] = {"ms": round(ms, 3), "gbs": round(2 * k.numel() * 2 / (ms / 1e3) / 1e9, 1)}
+    del q, k, v
+    torch.cuda.empty_cache()
+    res["kernel"] = "torch scaled_dot_product_attention (library, bf16, GQA), context only"
+    return res
+
+
 def extra_prefill(w, dev, stream, args, ws, dist_on, pk, pk_kind):
     """Another prefill workload timed the same way (device-resident inputs,
     W >= 3 warm-up steps, K timed steps between CUDA events, max over ranks),
@@ -494,6 +572,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-qcal", action="store_true", help="skip the 512K Q-Cal prefill reported beside the line")
     ap.add_argument("--no-bwd", action="store_true", help="skip the prefill backward reported beside the line")
+    ap.add_argument("--no-dense", action="store_true",
+                    help="skip timing dense attention of the same shapes (library kernel, context only)")
     ap.add_argument("--bwd-workload", default="prefill_8k", choices=[k for k, v in WORKLOADS.items() if not v.decode])
     ap.add_argument("--seq-len", type=int, default=0, help="override N of the prefill workload (profiling)")
     ap.add_argument("--decode-seq-len", type=int, default=0, help="override L of the decode workload (profiling)")
@@ -565,11 +645,27 @@ def main():
                                    / (summ_ms / 1e3) / 1e9, 1),
             "gpu_launches": 4 * args.steps * 5}
         del xd, dec
+        try:
+            line["decode"]["offload"] = bench_decode_offload(dev, stream, args, ws, dist_on)
+        except Exception as ex:  # host memory can run short on a box; report rather than stop
+            line["decode"]["offload"] = {"unavailable": f"{type(ex).__name__}: {str(ex)[:200]}"}
     if not args.no_qcal and args.workload != "prefill_512k_qcal" and not args.seq_len:
         line["prefill_512k_qcal"] = extra_prefill(WORKLOADS["prefill_512k_qcal"], dev, stream, args, ws, dist_on, pk,
                                                   pk_kind)
     if not args.no_bwd:
         line["backward"] = bench_backward(WORKLOADS[args.bwd_workload], dev, stream, args, ws, dist_on)
+    if not args.no_dense:
+        try:
+            dc = dense_comparator(dev, stream)
+        except Exception as ex:  # the library comparator is context: its failure must not stop the bench
+            dc = {"unavailable": f"{type(ex).__name__}: {str(ex)[:200]}"}
+        if "prefill_512k_qcal" in line and "prefill_512k" in dc:
+            dc["prefill_512k_ratio"] = round(dc["prefill_512k"]["ms"] / line["prefill_512k_qcal"]["ms_per_step"], 2)
+        if not args.seq_len and args.workload == "prefill_128k" and "prefill_128k" in dc:
+            dc["prefill_128k_ratio"] = round(dc["prefill_128k"]["ms"] / line["ms_per_step"], 2)
+        if "decode" in line and "decode_512k" in dc:
+            dc["decode_512k_ratio"] = round(dc["decode_512k"]["ms"] / line["decode"]["ms_per_step"], 2)
+        line["dense_context"] = dc
     if rank == 0 and not args.no_cpu:
         v, done, t_s, t_r = cpu_baseline_prefill(w, x)
         line["cpu_baseline"] = {"value": round(v, 2), "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",

@@ -57,6 +57,16 @@ hils_status_t dev_ctx(DevCtx* ctx) {
 
 bool aligned16(const void* p) { return p && ((uintptr_t)p & 15u) == 0; }
 
+// page-locked host memory (a host-resident decode cache)
+bool host_resident(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return a.type == cudaMemoryTypeHost;
+}
+
 // The operations whose shape coverage is checked on the host, before any
 // launch: a shape no kernel serves returns HILS_ERR_UNSUPPORTED.
 enum Op {
@@ -553,6 +563,9 @@ hils_status_t hils_attn_decode(const hils_config_t* cfg, const void* q, const vo
   const size_t need = decode_attn_workspace(s);
   if (ws_bytes < need || !aligned16(workspace))
     return fail(HILS_ERR_INVALID_ARG, "hils_attn_decode: workspace needs %zu bytes (got %zu)", need, ws_bytes);
+  if (s.dtype == HILS_F32 && (host_resident(k_cache) || host_resident(v_cache)))
+    return fail(HILS_ERR_UNSUPPORTED, "hils_attn_decode: a host-resident cache needs bf16 (the fp32 kernel copies "
+                                      "tiles with the bulk-copy engine)");
   DevCtx ctx;
   HILS_TRY(dev_ctx(&ctx));
   HILS_LAUNCH(launch_attn_decode(s, q, k_cache, v_cache, idx, s_sel, out, workspace, (cudaStream_t)stream, ctx),
@@ -663,10 +676,25 @@ hils_status_t hils_attn_decode_paged(const hils_config_t* cfg, const void* q, co
   const size_t need = decode_attn_workspace(s);
   if (ws_bytes < need || !aligned16(workspace))
     return fail(HILS_ERR_INVALID_ARG, "hils_attn_decode_paged: workspace needs %zu bytes (got %zu)", need, ws_bytes);
+  if (s.dtype == HILS_F32 && (host_resident(k_pool) || host_resident(v_pool)))
+    return fail(HILS_ERR_UNSUPPORTED, "hils_attn_decode_paged: a host-resident pool needs bf16");
   DevCtx ctx;
   HILS_TRY(dev_ctx(&ctx));
   HILS_LAUNCH(launch_attn_decode(s, q, k_pool, v_pool, idx, s_sel, out, workspace, (cudaStream_t)stream, ctx, dv),
               "attn_decode_paged");
+  return HILS_OK;
+}
+
+hils_status_t hils_host_device_pointer(const void* host, void** device_ptr) {
+  if (!host || !device_ptr) return fail(HILS_ERR_INVALID_ARG, "hils_host_device_pointer: NULL argument");
+  void* p = nullptr;
+  const cudaError_t e = cudaHostGetDevicePointer(&p, const_cast<void*>(host), 0);
+  if (e != cudaSuccess) {
+    cudaGetLastError();  // clear the error state so that later calls do not report it
+    return fail(HILS_ERR_INVALID_ARG, "hils_host_device_pointer: not page-locked mapped host memory (%s)",
+                cudaGetErrorString(e));
+  }
+  *device_ptr = p;
   return HILS_OK;
 }
 

@@ -33,6 +33,7 @@ EXPORTS = (
     "hils_build_summaries_paged",
     "hils_score_topk_paged",
     "hils_attn_decode_paged",
+    "hils_host_device_pointer",
     "hils_workspace_bytes",
     "hils_sync_status",
     "hils_last_error",
@@ -103,6 +104,8 @@ def load() -> ctypes.CDLL:
         lib.hils_attn_decode_noalloc.argtypes = [C, P, P, P, P, P, P, P]
         lib.hils_prefill_host.argtypes = [C, P, P, P, P, ctypes.POINTER(QCal), P, P, ctypes.c_size_t, P]
         lib.hils_prefill_bwd.argtypes = [C, P, P, P, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+        lib.hils_host_device_pointer.argtypes = [P, ctypes.POINTER(ctypes.c_void_p)]
+        lib.hils_host_device_pointer.restype = ctypes.c_int
         PG = ctypes.POINTER(Paged)
         lib.hils_decode_append.argtypes = [C, PG, P, P, P, P, P, P, P, P]
         lib.hils_build_summaries_paged.argtypes = [C, PG, P, P, P, P, P]
@@ -245,10 +248,24 @@ def hils_prefill_host(cfg: Config, q, k, v, q_lmk, out, workspace, qcal=None, st
                                     _p(workspace), ws_bytes, _stream(stream)))
 
 
+def _pc(t):
+    """A CUDA tensor, or a device address (int) such as hils_host_device_pointer's."""
+    return ctypes.c_void_p(t) if isinstance(t, int) else _p(t)
+
+
 def hils_attn_decode(cfg: Config, q, k_cache, v_cache, idx, s_sel, out, workspace, stream=None):
+    """k_cache / v_cache: CUDA tensors, or device addresses of pinned host memory."""
     ws_bytes = workspace.numel() * workspace.element_size()
-    _check(load().hils_attn_decode(ctypes.byref(cfg), _p(q), _p(k_cache), _p(v_cache), _p(idx), _p(s_sel), _p(out),
+    _check(load().hils_attn_decode(ctypes.byref(cfg), _p(q), _pc(k_cache), _pc(v_cache), _p(idx), _p(s_sel), _p(out),
                                    _p(workspace), ws_bytes, _stream(stream)))
+
+
+def hils_host_device_pointer(t: torch.Tensor) -> int:
+    """Device address of a pinned host tensor (for a host-resident decode cache)."""
+    assert not t.is_cuda and t.is_pinned() and t.is_contiguous()
+    out = ctypes.c_void_p()
+    _check(load().hils_host_device_pointer(ctypes.c_void_p(t.data_ptr()), ctypes.byref(out)))
+    return out.value
 
 
 def hils_attn_decode_noalloc(cfg: Config, q, k_cache, v_cache, idx, s_sel, out, stream=None):

@@ -274,6 +274,18 @@ hils_status_t hils_attn_decode_paged(const hils_config_t* cfg, const void* q, co
                                      void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Device address of page-locked (pinned), mapped host memory, for keeping the
+ * decode KV cache in host memory (the wmrh.cn article on HiLS: chunk-sparse
+ * attention lets the unselected chunks of the cache stay off the GPU).  Passed
+ * as k_cache / v_cache to hils_attn_decode (or as the pools of
+ * hils_attn_decode_paged), the decode attention reads only the token's K
+ * chunks and its window, i.e. (K S + W) Hkv d 2 elements per sequence, over
+ * the host link; the summaries stay in device memory.  Returns
+ * HILS_ERR_INVALID_ARG (and launches nothing) if `host` is not such memory.
+ */
+hils_status_t hils_host_device_pointer(const void* host, void** device_ptr);
+
+/*
  * The whole prefill path from host memory: copies the inputs to the device,
  * builds the summaries, scores and selects (hils_build_summaries,
  * hils_score_topk) and attends (hils_attn_prefill), then copies the output
