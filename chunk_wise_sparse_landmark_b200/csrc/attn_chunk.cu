@@ -349,11 +349,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ---------------------------------------------------------- epilogue ----
     // Partial record of (position, slot k): [head][128] bf16; in a head's row,
     // element 64 h2 + 8 r + 4 a + t holds d = 64 h2 + 32 a + r + 8 t (h2, a =
-    // 0..1, r = 0..7, t = 0..3).  Each 64-column half of the TMEM row is one
-    // contiguous 128-byte run written with 32-byte stores (measured: records
-    // written as 16-byte halves of sectors from separate passes cost ~13 ms of
-    // the 128K attention), and the 16 bytes at 64 h2 + 8 r are what one thread
-    // of the window pass's MMA fragments consumes.  Item metadata is fetched ahead.
+    // 0..1, r = 0..7, t = 0..3); the 16 bytes at 64 h2 + 8 r are what one
+    // thread of the window pass's MMA fragments consumes.  Each 64-column half
+    // of the TMEM row is one contiguous 128-byte run written with 32-byte
+    // stores (measured: records written as 16-byte halves of sectors from
+    // separate passes cost ~13 ms of the 128K attention; staging the rows in
+    // shared memory so that each warp store covers a whole 512-byte run, and
+    // bulk copies of 1 KB records from shared memory, were both slower, 41 and
+    // 32 ms against 30 ms).  Item metadata is fetched ahead.
     const int qw = warp & 3, row = 32 * qw + lane, jr = row >> 2, h = row & 3;
     const uint32_t lrow = (uint32_t)(32 * qw) << 16;
     Item m0 = item_of(0), m1 = item_of(1);
@@ -423,16 +426,34 @@ HILS_DI void list_of(const Shape& s, const int32_t* __restrict__ idx, int t0, in
   if (report && bad && lane == 0) raise_status(*report, kStatusBadIndex);
 }
 
+// Both passes run one block per (KV group bg, block of PB positions) and count
+// into a shared histogram over the C chunks first, so that global atomics are
+// one per (block, non-empty bucket) instead of one per pair (measured: ~0.25 ms
+// per 32K-position tile with a global atomic per pair).
+constexpr int PB = 1024;  // positions per bucketing block
+
+HILS_DI void count_block(const Shape& s, const int32_t* __restrict__ idx, int t0, int np, int* hist,
+                         const DevCtx* report) {
+  const int bg = blockIdx.x / ((np + PB - 1) / PB), pb = blockIdx.x % ((np + PB - 1) / PB);
+  const int p_end = min(np, (pb + 1) * PB), wpb = blockDim.x >> 5;
+  for (int c = threadIdx.x; c < s.C; c += blockDim.x) hist[c] = 0;
+  __syncthreads();
+  for (int pl = pb * PB + (threadIdx.x >> 5); pl < p_end; pl += wpb) {
+    int bgx, plx, a, b;
+    list_of(s, idx, t0, np, (long long)bg * np + pl, bgx, plx, a, b, report);
+    if (a >= 0) atomicAdd(hist + a, 1);
+    if (b >= 0) atomicAdd(hist + b, 1);
+  }
+  __syncthreads();
+}
+
 __global__ void bucket_count_kernel(Shape s, const int32_t* __restrict__ idx, int t0, int np, int* __restrict__ cnt,
                                     DevCtx ctx) {
-  const long long lists = (long long)s.B * s.Hkv * np;
-  const long long wpb = blockDim.x >> 5;
-  for (long long r = blockIdx.x * wpb + (threadIdx.x >> 5); r < lists; r += (long long)gridDim.x * wpb) {
-    int bg, pl, a, b;
-    list_of(s, idx, t0, np, r, bg, pl, a, b, &ctx);
-    if (a >= 0) atomicAdd(cnt + bg * s.C + a, 1);
-    if (b >= 0) atomicAdd(cnt + bg * s.C + b, 1);
-  }
+  extern __shared__ int hist[];
+  count_block(s, idx, t0, np, hist, &ctx);
+  const int bg = blockIdx.x / ((np + PB - 1) / PB);
+  for (int c = threadIdx.x; c < s.C; c += blockDim.x)
+    if (hist[c]) atomicAdd(cnt + bg * s.C + c, hist[c]);
 }
 
 // One block: exclusive scans of the bucket counts (pair offsets) and of their
@@ -495,18 +516,24 @@ __global__ void __launch_bounds__(1024) bucket_scan_kernel(int U, int* __restric
 __global__ void bucket_scatter_kernel(Shape s, const int32_t* __restrict__ idx, int t0, int np,
                                       const int* __restrict__ off, const int* __restrict__ ioff, int* __restrict__ cur,
                                       int* __restrict__ ent, int4* __restrict__ items) {
-  const long long lists = (long long)s.B * s.Hkv * np;
-  const long long wpb = blockDim.x >> 5;
+  extern __shared__ int hist[];
+  count_block(s, idx, t0, np, hist, nullptr);  // the count pass reported bad entries
+  const int bg = blockIdx.x / ((np + PB - 1) / PB), pb = blockIdx.x % ((np + PB - 1) / PB);
+  const int p_end = min(np, (pb + 1) * PB), wpb = blockDim.x >> 5;
   const int lane = threadIdx.x & 31;
-  for (long long r = blockIdx.x * wpb + (threadIdx.x >> 5); r < lists; r += (long long)gridDim.x * wpb) {
-    int bg, pl, a, b;
-    list_of(s, idx, t0, np, r, bg, pl, a, b, nullptr);  // the count pass reported bad entries
+  // this block's range of every bucket: one global atomic per non-empty bucket
+  for (int c = threadIdx.x; c < s.C; c += blockDim.x)
+    if (hist[c]) hist[c] = atomicAdd(cur + bg * s.C + c, hist[c]);
+  __syncthreads();
+  for (int pl = pb * PB + (threadIdx.x >> 5); pl < p_end; pl += wpb) {
+    int bgx, plx, a, b;
+    list_of(s, idx, t0, np, (long long)bg * np + pl, bgx, plx, a, b, nullptr);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int c = h ? b : a;
       if (c < 0) continue;
       const int u = bg * s.C + c;
-      const int slot = atomicAdd(cur + u, 1);
+      const int slot = atomicAdd(hist + c, 1);  // shared cursor
       ent[slot] = (pl << 6) | (lane + 32 * h);
       const int rel = slot - __ldg(off + u);
       if (rel % PPI == 0)
@@ -592,11 +619,11 @@ cudaError_t launch_attn_prefill_chunked(const Shape& s, const void* q, const voi
     if (U > 0) {
       e = cudaMemsetAsync(cnt, 0, (size_t)U * 4, st);
       if (e != cudaSuccess) return e;
-      const long long lists = (long long)s.B * s.Hkv * np;
-      const int grid = (int)std::min<long long>((lists + 7) / 8, (long long)sms * 16);
-      bucket_count_kernel<<<grid, 256, 0, st>>>(s, idx, t0, np, cnt, ctx);
+      const int grid = s.B * s.Hkv * ((np + PB - 1) / PB);
+      const size_t hsmem = (size_t)s.C * sizeof(int);  // C <= 8192: at most 32 KB
+      bucket_count_kernel<<<grid, 512, hsmem, st>>>(s, idx, t0, np, cnt, ctx);
       bucket_scan_kernel<<<1, 1024, 0, st>>>(U, cnt, off, ioff);
-      bucket_scatter_kernel<<<grid, 256, 0, st>>>(s, idx, t0, np, off, ioff, cnt, ent, items);
+      bucket_scatter_kernel<<<grid, 512, hsmem, st>>>(s, idx, t0, np, off, ioff, cnt, ent, items);
       attn_chunk_kernel<<<sms, THREADS, kSmemBytes, st>>>(s, tmk, tmv, (const __nv_bfloat16*)q, ioff, items, ent, t0,
                                                           w.PT, part, ctx);
       e = cudaGetLastError();
