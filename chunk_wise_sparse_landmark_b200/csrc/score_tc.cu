@@ -11,7 +11,7 @@
 // One CTA = 128 positions (the MMA's M) of one (sequence, KV group).  The
 // four heads' query tiles are written once into tensor memory (256 columns)
 // and serve as the A operand of every MMA; k' tiles of 64 chunks x 128 for the
-// four heads (64 KB) stream through a 3-stage TMA ring (128-byte swizzle,
+// four heads (64 KB) stream through a 2-stage TMA ring (128-byte swizzle,
 // chunks past C read as zero) into one 4 x 64-column fp32 accumulator.  A
 // thread that issues tcgen05.mma gets one instruction through every ~130
 // cycles whatever its N, so each head has its own issuing warp (warps 0..3,
@@ -22,7 +22,9 @@
 // Selection is exact and deterministic.  Pass 1 streams every tile; each
 // epilogue thread keeps the multiset of the KT >= K largest group scores of
 // its half, sorted in registers, updated by branch-free insertion of the few
-// candidates above its current KT-th value.  After the last tile the row's
+// candidates above its current KT-th value, or, while a tile brings many of
+// them (a row's first tiles), by sorting the tile's 32 candidates with a
+// bitonic network and merging the two sorted lists.  After the last tile the row's
 // threshold tau (its K-th largest score) is the minimum over j < K of
 // max(a_j, b_{K-1-j}) for the two halves' sorted lists a, b, and A = the
 // number of scores above tau.  Pass 2 recomputes the same tiles (same
@@ -39,7 +41,7 @@ constexpr int D = 128, G = 4;
 constexpr int MQ = 128;   // positions per CTA (MMA M, TMEM lanes)
 constexpr int TCH = 64;   // chunks per tile (MMA N)
 constexpr int HALF = TCH / 2;
-constexpr int NST = 3;    // k' ring stages
+constexpr int NST = 2;    // k' ring stages (measured: 3 stages were 0.5 ms slower at 128K)
 constexpr int KMAX = 64;
 constexpr int NMMA = G;   // MMA-issuing warps, one per head
 constexpr int EPI = 256;  // epilogue threads
@@ -81,6 +83,47 @@ HILS_DI void insert_desc(float (&a)[KT], float x) {
 #pragma unroll
   for (int j = KT - 1; j > 0; --j) a[j] = fmaxf(fminf(a[j - 1], x), a[j]);
   a[0] = fmaxf(a[0], x);
+}
+
+// sort 32 values descending in registers (bitonic network, 240 compare-exchanges)
+HILS_DI void sort32_desc(float (&a)[32]) {
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1)
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1)
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int l = i ^ j;
+        if (l > i) {
+          const float x = a[i], y = a[l];
+          const bool desc = (i & k) == 0;
+          a[i] = desc ? fmaxf(x, y) : fminf(x, y);
+          a[l] = desc ? fminf(x, y) : fmaxf(x, y);
+        }
+      }
+}
+
+// top (the KT largest so far, descending) <- the KT largest of top and b (32
+// values, descending): the elementwise max of top and b reversed is bitonic and
+// holds those KT values; a bitonic merge sorts it descending
+template <int KT>
+HILS_DI void merge_top(float (&top)[KT], const float (&b)[32]) {
+#pragma unroll
+  for (int i = 0; i < KT; ++i) {
+    const int bi = KT - 1 - i;
+    top[i] = fmaxf(top[i], bi < 32 ? b[bi] : -INFINITY);
+  }
+#pragma unroll
+  for (int j = KT >> 1; j > 0; j >>= 1)
+#pragma unroll
+    for (int i = 0; i < KT; ++i) {
+      const int l = i ^ j;
+      if (l > i) {
+        const float x = top[i], y = top[l];
+        top[i] = fmaxf(x, y);
+        top[l] = fminf(x, y);
+      }
+    }
 }
 
 // v[j] for a runtime j in [0, 32), by a tree of selects (no local memory)
@@ -285,9 +328,24 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.dempty);
-        // candidates above the current KT-th value, staged, then inserted
+        // candidates above the current KT-th value: when any lane of the warp
+        // has many (the first tiles of a row), the tile is sorted and merged
+        // into the list (~670 operations); otherwise each is staged and
+        // inserted (~63 operations each)
+        const float thr0 = top[KT - 1];
+        int nab = 0;
+#pragma unroll
+        for (int j = 0; j < HALF; ++j) nab += (c0 + j < ncand && gv[j] > thr0) ? 1 : 0;
+        const bool bulk = __any_sync(0xffffffffu, nab >= 12);
+        if (bulk) {
+#pragma unroll
+          for (int j = 0; j < HALF; ++j) gv[j] = (c0 + j < ncand && gv[j] > thr0) ? gv[j] : -INFINITY;
+          sort32_desc(gv);
+          merge_top<KT>(top, gv);
+        }
 #pragma unroll
         for (int rd = 0; rd < HALF / STG; ++rd) {
+          if (bulk) break;  // warp-uniform
           const float thr = top[KT - 1];
           int ns = 0;
 #pragma unroll
@@ -368,6 +426,9 @@ __global__ void __launch_bounds__(THREADS, 1)
               }
             }
           }
+          // (measured: writing each head's 32 scores to a per-thread column of
+          // shared memory and reading the chosen ones by index was slower,
+          // 10.8 against 8.6 ms at 128K, than this select tree per chosen chunk)
 #pragma unroll
           for (int hh = 0; hh < G; ++hh) {
             uint32_t v[HALF];
