@@ -15,11 +15,9 @@
 //   P = softmax over the 64 keys of each row, bf16, written back into TMEM
 //   O (128 rows x 128 d)    = P (128 x 64) . V_c (64 x d)     tcgen05, fp32 in TMEM
 //
-// O is stored in bf16 as the item's block of partial records (one row per
-// (position, slot k of its selection list, head), item-major, launch.h), and
-// the window pass (attn_ring.cu) adds the window's exact softmax terms and
-// fuses the partials with the exp(s^) weights; the scatter writes where each
-// (position, slot) pair's rows landed.
+// O is stored as one 1 KB bf16 record per (position, slot k of its selection
+// list; heads innermost) -- the "partial" -- and the window pass (attn_ring.cu) adds the window's
+// exact softmax terms and fuses the partials with the exp(s^) weights.
 //
 // Why chunk-major: on the pages' i.i.d.-like workloads adjacent positions
 // share almost none of their selected chunks, so a position-major kernel
@@ -47,8 +45,8 @@
 //   warps 10-13 softmax: TMEM S row -> max, exp2 -> normalised bf16 P row,
 //               written back into the first half of the row's S columns; the
 //               second MMA reads P from TMEM (no shared-memory traffic)
-//   warps 14-17 epilogue: TMEM O row -> bf16 partial record row (16-byte
-//               pieces, one 512-byte run per warp store)
+//   warps 14-17 epilogue: TMEM O row -> bf16 partial record (a position's
+//               4 head rows are adjacent lanes: 128-byte lines per store)
 // 18 warps: the register file is split across the four sub-partitions, so
 // 96 registers per thread is the most that fits.
 //
@@ -66,7 +64,6 @@
 // Every wait is bounded (status word + early return), see common.cuh.
 #include <algorithm>
 
-#include "gather_mma.cuh"
 #include "launch.h"
 #include "tmap.h"
 
@@ -97,9 +94,16 @@ struct __align__(1024) SmemC {
 constexpr size_t kSmemBytes = sizeof(SmemC) + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
-// 16-byte global store
-HILS_DI void stg16(void* p, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
-  asm volatile("st.global.v4.b32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
+HILS_DI void ldg32(const void* p, uint32_t (&w)[8]) {
+  asm volatile("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+               : "l"(p));
+}
+// 32-byte global store (address 32-byte aligned)
+HILS_DI void stg32(void* p, const uint32_t (&w)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+               "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
 }
 // 32 lanes x 16 consecutive 32-bit columns <- 16 registers per thread
 HILS_DI void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
@@ -131,7 +135,7 @@ struct Item {
 __global__ void __launch_bounds__(THREADS, 1)
     attn_chunk_kernel(Shape s, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                       const __nv_bfloat16* __restrict__ q, const int* __restrict__ ioff,
-                      const int4* __restrict__ items, const int* __restrict__ ent, int t0,
+                      const int4* __restrict__ items, const int* __restrict__ ent, int t0, int PT,
                       __nv_bfloat16* __restrict__ part, DevCtx ctx) {
   extern __shared__ unsigned char smem_raw[];
   SmemC& sm = *reinterpret_cast<SmemC*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -344,25 +348,32 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     // ---------------------------------------------------------- epilogue ----
-    // Records are item-major (launch.h): this item's 128 rows x 16 pieces of
-    // 16 bytes, piece-major, so each warp store covers 32 consecutive rows, a
-    // 512-byte run.  Piece pc = 8 h2 + r of a row holds, at element 4 a + t,
-    // d = 64 h2 + 32 a + r + 8 t (h2, a = 0..1, r = 0..7, t = 0..3): the 8
-    // values one thread of the window pass's MMA fragments consumes.
-    // Measured at 128K before this layout: with one row per lane each warp
-    // store touched 32 rows (32 cache lines); 16-byte halves of sectors from
-    // separate passes cost ~13 ms of the attention, contiguous 128-byte runs
-    // per row half ~7 ms; staging in shared memory for 512-byte runs (41 ms,
-    // with spills) and bulk copies of 1 KB records (32 ms) were slower.
-    const int qw = warp & 3, row = 32 * qw + lane, jr = row >> 2;
+    // Partial record of (position, slot k): 1 KB of bf16, [unit u][head][32 B]
+    // with u = 4 h2 + r / 2 (8 units of 128 bytes, heads innermost).  Unit
+    // u's 32 bytes of a head hold pieces r and r + 1 of the head's 64-column
+    // half h2 (r even); in piece r, element 4 a + t holds d = 64 h2 + 32 a +
+    // r + 8 t (a = 0..1, t = 0..3): the 8 values one thread of the window
+    // pass's MMA fragments consumes.  The 4 head rows of a position are 4
+    // adjacent lanes, so each warp store writes 8 whole 128-byte lines.
+    // Measured at 128K: head-major records (each warp store touching 32
+    // lines) cost ~7 ms of the attention; item-major blocks of 128 rows (one
+    // 512-byte run per store) were as fast to write but left the window pass
+    // reading 64-byte pieces 2 KB apart (17.5 ms against 13 ms); staging in
+    // shared memory for 512-byte runs (41 ms, with spills) and bulk copies of
+    // 1 KB records (32 ms) were slower.  Item metadata is fetched ahead.
+    const int qw = warp & 3, row = 32 * qw + lane, jr = row >> 2, h = row & 3;
     const uint32_t lrow = (uint32_t)(32 * qw) << 16;
-    Item nx = item_of(0);
+    Item m0 = item_of(0), m1 = item_of(1);
+    int e0 = jr < m0.n ? __ldg(ent + m0.s0 + jr) : 0;
     for (int it = 0; it < nmine; ++it) {
       const int st = it % NST;
-      const Item im = nx;
-      nx = item_of(it + 1);
+      const Item im = m0;
+      const int e = e0;
+      e0 = jr < m1.n ? __ldg(ent + m1.s0 + jr) : 0;
+      m0 = m1;
+      m1 = item_of(it + 2);
       const bool valid = jr < im.n;
-      __nv_bfloat16* dst = part + (long long)(bid + it * nb) * (kItemRows * D) + row * 8;
+      __nv_bfloat16* dst = part + (((long long)im.bg * PT + (e >> 6)) * s.K + (e & 63)) * (G * D) + h * 16;
       const bool ok = mbar_wait(&sm.ofull[st], (it / NST) & 1, ctx);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
@@ -374,12 +385,17 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_wait_ld();
         if (valid) {
 #pragma unroll
-          for (int r = 0; r < 8; ++r)
-            stg16(dst + (8 * pr + r) * (kItemRows * 8),
-                  pack_bf16x2(__uint_as_float(v0[r]), __uint_as_float(v0[r + 8])),
-                  pack_bf16x2(__uint_as_float(v0[r + 16]), __uint_as_float(v0[r + 24])),
-                  pack_bf16x2(__uint_as_float(v1[r]), __uint_as_float(v1[r + 8])),
-                  pack_bf16x2(__uint_as_float(v1[r + 16]), __uint_as_float(v1[r + 24])));
+          for (int r = 0; r < 8; r += 2) {
+            uint32_t o[8];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              o[4 * u + 0] = pack_bf16x2(__uint_as_float(v0[r + u]), __uint_as_float(v0[r + u + 8]));
+              o[4 * u + 1] = pack_bf16x2(__uint_as_float(v0[r + u + 16]), __uint_as_float(v0[r + u + 24]));
+              o[4 * u + 2] = pack_bf16x2(__uint_as_float(v1[r + u]), __uint_as_float(v1[r + u + 8]));
+              o[4 * u + 3] = pack_bf16x2(__uint_as_float(v1[r + u + 16]), __uint_as_float(v1[r + u + 24]));
+            }
+            stg32(dst + (4 * pr + r / 2) * (G * 16), o);
+          }
         }
       }
       tc_fence_before();
@@ -503,7 +519,7 @@ __global__ void __launch_bounds__(1024) bucket_scan_kernel(int U, int* __restric
 
 __global__ void bucket_scatter_kernel(Shape s, const int32_t* __restrict__ idx, int t0, int np,
                                       const int* __restrict__ off, const int* __restrict__ ioff, int* __restrict__ cur,
-                                      int* __restrict__ ent, int4* __restrict__ items, int* __restrict__ loc, int PT) {
+                                      int* __restrict__ ent, int4* __restrict__ items) {
   extern __shared__ int hist[];
   count_block(s, idx, t0, np, hist, nullptr);  // the count pass reported bad entries
   const int bg = blockIdx.x / ((np + PB - 1) / PB), pb = blockIdx.x % ((np + PB - 1) / PB);
@@ -524,9 +540,8 @@ __global__ void bucket_scatter_kernel(Shape s, const int32_t* __restrict__ idx, 
       const int slot = atomicAdd(hist + c, 1);  // shared cursor
       ent[slot] = (pl << 6) | (lane + 32 * h);
       const int rel = slot - __ldg(off + u);
-      const int i0 = __ldg(ioff + u);
-      if (rel % PPI == 0) items[i0 + rel / PPI] = make_int4(u, slot, min(PPI, __ldg(off + u + 1) - slot), 0);
-      loc[((long long)bg * PT + pl) * s.K + lane + 32 * h] = i0 * PPI + rel;  // item * 32 + position in item
+      if (rel % PPI == 0)
+        items[__ldg(ioff + u) + rel / PPI] = make_int4(u, slot, min(PPI, __ldg(off + u + 1) - slot), 0);
     }
   }
 }
@@ -535,7 +550,7 @@ size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // workspace pieces, in order
 struct ChunkWs {
-  size_t cnt, off, ioff, ent, items, loc, part, total;
+  size_t cnt, off, ioff, ent, items, part, total;
   int PT;
 };
 
@@ -565,8 +580,7 @@ ChunkWs chunk_ws(const Shape& s) {
   w.ioff = take((U + 1) * 4);
   w.ent = take(pairs * 4);
   w.items = take((pairs / PPI + U + 1) * 16);
-  w.loc = take(pairs * 4);
-  w.part = take((pairs / PPI + U + 1) * (size_t)kItemRows * D * 2);  // one record block per item
+  w.part = take(pairs * G * D * 2);
   w.total = o;
   return w;
 }
@@ -589,7 +603,6 @@ cudaError_t launch_attn_prefill_chunked(const Shape& s, const void* q, const voi
   int* ioff = (int*)(W + w.ioff);
   int* ent = (int*)(W + w.ent);
   int4* items = (int4*)(W + w.items);
-  int* loc = (int*)(W + w.loc);
   __nv_bfloat16* part = (__nv_bfloat16*)(W + w.part);
   const int U = s.B * s.Hkv * s.C;
 
@@ -614,14 +627,13 @@ cudaError_t launch_attn_prefill_chunked(const Shape& s, const void* q, const voi
       const size_t hsmem = (size_t)s.C * sizeof(int);  // C <= 8192: at most 32 KB
       bucket_count_kernel<<<grid, 512, hsmem, st>>>(s, idx, t0, np, cnt, ctx);
       bucket_scan_kernel<<<1, 1024, 0, st>>>(U, cnt, off, ioff);
-      bucket_scatter_kernel<<<grid, 512, hsmem, st>>>(s, idx, t0, np, off, ioff, cnt, ent, items, loc, w.PT);
+      bucket_scatter_kernel<<<grid, 512, hsmem, st>>>(s, idx, t0, np, off, ioff, cnt, ent, items);
       attn_chunk_kernel<<<sms, THREADS, kSmemBytes, st>>>(s, tmk, tmv, (const __nv_bfloat16*)q, ioff, items, ent, t0,
-                                                          part, ctx);
+                                                          w.PT, part, ctx);
       e = cudaGetLastError();
       if (e != cudaSuccess) return e;
     }
-    e = launch_attn_window_merge(s, q, k, v, idx, s_sel, out, U > 0 ? part : nullptr, U > 0 ? loc : nullptr, t0,
-                                 t0 + np, w.PT, st, ctx);
+    e = launch_attn_window_merge(s, q, k, v, idx, s_sel, out, U > 0 ? part : nullptr, t0, t0 + np, w.PT, st, ctx);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

@@ -55,7 +55,6 @@
 // rescaled) when a window logit exceeds it.  out = acc / den.
 #include <climits>
 
-#include "gather_mma.cuh"
 #include "launch.h"
 #include "tmap.h"
 
@@ -132,8 +131,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     attn_ring_kernel(Shape s, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                      const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ idx,
                      const float* __restrict__ s_sel, __nv_bfloat16* __restrict__ out,
-                     const __nv_bfloat16* __restrict__ part, const int* __restrict__ loc, int t0, int t1,
-                     int PT, DevCtx ctx) {
+                     const __nv_bfloat16* __restrict__ part, int t0, int t1, int PT, DevCtx ctx) {
   extern __shared__ unsigned char smem_raw[];
   SmemR& sm = *reinterpret_cast<SmemR*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -499,45 +497,34 @@ __global__ void __launch_bounds__(THREADS, 2)
     }
 
     // ---- selected chunks from their partial records O_c (attn_chunk.cu):
-    // acc += e^{s^ - m} O_c, den += e^{s^ - m}.  The pair's rows sit in item
-    // gr / 32 at rows 4 (gr % 32) + h (gr from loc).  Piece pc = 8 hh + gq of
-    // a head row holds this thread's values d = 64 hh + 32 a + gq + 8 t at
-    // element 4 a + t (hh, a = 0..1, t = 0..3), i.e. d = 16 mt + gq (+ 8) for
-    // mt = 4 hh + 2 a + t/2; rows my_h and my_h + 1 are adjacent, so one
-    // 32-byte load brings both.  MSL slots are loaded at a time (predicated,
-    // no branch) so that their HBM round trips overlap.
+    // acc += e^{s^ - m} O_c, den += e^{s^ - m}.  A record is [unit][head][32 B]
+    // (attn_chunk.cu); piece (hh, gq) of a head, 16 bytes in unit 4 hh + gq/2
+    // at half gq % 2, holds this thread's values d = 64 hh + 32 a + gq + 8 t
+    // at element 4 a + t (a = 0..1, t = 0..3), i.e. d = 16 mt + gq (+ 8) for
+    // mt = 4 hh + 2 a + t/2.  MSL slots are loaded at a time (predicated, no branch)
+    // so that their HBM round trips overlap.
     if (PART && ok) {
-      const int* lr = loc + ((long long)bg * PT + (my_pos - t0)) * K;
+      const __nv_bfloat16* rec =
+          part + (((long long)bg * PT + (my_pos - t0)) * K) * (G * D) + (gq >> 1) * (G * 16) + (gq & 1) * 8;
       for (int x0 = 0; x0 < K; x0 += MSL) {
-        uint32_t w[MSL][2][8];
+        uint4 w[MSL][2][2];
         float wg[MSL][2];
-        int gr[MSL];
 #pragma unroll
         for (int j = 0; j < MSL; ++j) {
           const int x = x0 + j;
           const int ca = entry(m0a, m0b, x), cb = entry(m1a, m1b, x);
           const bool v = my_valid && (my_q == 0 ? ca : cb) >= 0;
-          gr[j] = v ? __ldg(lr + x) : -1;
-        }
-#pragma unroll
-        for (int j = 0; j < MSL; ++j) {
-          const int x = x0 + j;
-          const bool v = gr[j] >= 0;
-          const __nv_bfloat16* rx =
-              part + (long long)(gr[j] >> 5) * (kItemRows * D) + ((gr[j] & 31) * G + my_h) * 8 + gq * (kItemRows * 8);
+          const __nv_bfloat16* rx = rec + (long long)x * (G * D);
 #pragma unroll
           for (int r = 0; r < 2; ++r) {
             float sv = -INFINITY;
             if (v) sv = __ldg(ss0 + r * sstride + x);
             wg[j][r] = sv;
-          }
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            if (v) {
-              ldg32(rx + hh * (8 * kItemRows * 8), w[j][hh]);
-            } else {
-#pragma unroll
-              for (int y = 0; y < 8; ++y) w[j][hh][y] = 0u;
+            for (int hh = 0; hh < 2; ++hh) {
+              uint4 u = make_uint4(0u, 0u, 0u, 0u);
+              if (v) u = __ldg(reinterpret_cast<const uint4*>(rx + hh * (4 * G * 16) + (my_h + r) * 16));
+              w[j][r][hh] = u;
             }
           }
         }
@@ -549,10 +536,11 @@ __global__ void __launch_bounds__(THREADS, 2)
             den[r] += wgt;
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
+              const uint32_t ww[4] = {w[j][r][hh].x, w[j][r][hh].y, w[j][r][hh].z, w[j][r][hh].w};
 #pragma unroll
               for (int q2 = 0; q2 < 4; ++q2) {  // a = q2 / 2, t pair = q2 % 2
                 const int mt = 4 * hh + q2;
-                const float2 f = bf16x2_to_f32x2(w[j][hh][4 * r + q2]);
+                const float2 f = bf16x2_to_f32x2(ww[q2]);
                 acc[mt][r] = fmaf(wgt, f.x, acc[mt][r]);
                 acc[mt][2 + r] = fmaf(wgt, f.y, acc[mt][2 + r]);
               }
@@ -584,8 +572,8 @@ constexpr size_t kSmemBytes = sizeof(SmemR) + 1024;
 }  // namespace
 
 cudaError_t launch_attn_window_merge(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
-                                     const float* s_sel, void* out, const void* part, const int* loc, int t0, int t1,
-                                     int PT, cudaStream_t st, const DevCtx& ctx) {
+                                     const float* s_sel, void* out, const void* part, int t0, int t1, int PT,
+                                     cudaStream_t st, const DevCtx& ctx) {
   if (s.d != D || s.S != S || s.G != G || s.K > KMAX || s.C > MAXC || s.nw > 32) return cudaErrorNotSupported;
   if (t0 % 2 || t1 <= t0) return cudaErrorInvalidValue;
   CUtensorMap tmk, tmv;
@@ -596,19 +584,18 @@ cudaError_t launch_attn_window_merge(const Shape& s, const void* q, const void* 
   if (e != cudaSuccess) return e;
   e = make_tmap_bf16(&tmv, v, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
-  if ((part == nullptr) != (loc == nullptr)) return cudaErrorInvalidValue;
   auto kern = part ? attn_ring_kernel<true> : attn_ring_kernel<false>;
   e = ensure_dynamic_smem((const void*)kern, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid((t1 - t0 + BP - 1) / BP, s.Hkv, s.B);
   kern<<<grid, THREADS, kSmemBytes, st>>>(s, tmk, tmv, (const __nv_bfloat16*)q, idx, s_sel, (__nv_bfloat16*)out,
-                                          (const __nv_bfloat16*)part, loc, t0, t1, PT, ctx);
+                                          (const __nv_bfloat16*)part, t0, t1, PT, ctx);
   return cudaGetLastError();
 }
 
 cudaError_t launch_attn_prefill_tc(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
                                    const float* s_sel, void* out, cudaStream_t st, const DevCtx& ctx) {
-  return launch_attn_window_merge(s, q, k, v, idx, s_sel, out, nullptr, nullptr, 0, s.N, 0, st, ctx);
+  return launch_attn_window_merge(s, q, k, v, idx, s_sel, out, nullptr, 0, s.N, 0, st, ctx);
 }
 
 }  // namespace hils

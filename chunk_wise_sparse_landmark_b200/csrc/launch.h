@@ -81,20 +81,12 @@ cudaError_t launch_attn_prefill_simt(const Shape& s, const void* q, const void* 
 // chunk union (no workspace)
 cudaError_t launch_attn_prefill_tc(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
                                    const float* s_sel, void* out, cudaStream_t st, const DevCtx& ctx);
-// Partial records of the chunk-major prefill: one block of kItemRows rows per
-// item (32 positions x 4 heads, row = 4 j + h), laid out [16-byte piece
-// (kRecPieces)][row] in bf16, so that one warp store covers 32 consecutive
-// rows.  loc[(bg * PT + p_local) * K + slot] = item * 32 + j locates the pair.
-constexpr int kItemRows = 128;
-constexpr int kRecPieces = 16;
-
-// the window pass over positions [t0, t1); with `part` and `loc` (partial
-// records of the selected chunks and their locations, tile of PT positions)
-// it attends the window only and fuses the records, without them it also
-// streams the selected chunks
+// the window pass over positions [t0, t1); with `part` (partial records of the
+// selected chunks, tile of PT positions) it attends the window only and fuses
+// the records, without it it also streams the selected chunks
 cudaError_t launch_attn_window_merge(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
-                                     const float* s_sel, void* out, const void* part, const int* loc, int t0, int t1,
-                                     int PT, cudaStream_t st, const DevCtx& ctx);
+                                     const float* s_sel, void* out, const void* part, int t0, int t1, int PT,
+                                     cudaStream_t st, const DevCtx& ctx);
 // bf16 prefill attention, chunk-major selected chunks (tcgen05) + window pass,
 // by position tiles; workspace of attn_prefill_tc_workspace(s) bytes
 size_t attn_prefill_tc_workspace(const Shape& s);
