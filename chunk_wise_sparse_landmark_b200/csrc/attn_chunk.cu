@@ -134,9 +134,8 @@ struct Item {
 
 __global__ void __launch_bounds__(THREADS, 1)
     attn_chunk_kernel(Shape s, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
-                      const __nv_bfloat16* __restrict__ q, const int* __restrict__ ioff,
-                      const int4* __restrict__ items, const int* __restrict__ ent, int t0, int PT,
-                      __nv_bfloat16* __restrict__ part, DevCtx ctx) {
+                      const int* __restrict__ ioff, const int4* __restrict__ items, const int* __restrict__ ent,
+                      int PT, const __nv_bfloat16* __restrict__ qg, __nv_bfloat16* __restrict__ part, DevCtx ctx) {
   extern __shared__ unsigned char smem_raw[];
   SmemC& sm = *reinterpret_cast<SmemC*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -264,7 +263,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     // -------------------------------------------------------- query rows ----
     // Group wg (warps 2-5 or 6-9) takes items wg, wg + 2, ...; thread = TMEM
     // lane = row r = 4 j + h: head h of the item's position j (rows past the
-    // item's count are zero).  The 256-byte row is loaded before the stage is
+    // item's count are zero).  The rows come from the tile's regrouped copy,
+    // where a position's 4 heads sit side by side in 32-byte pieces, so each
+    // warp load reads 8 whole 128-byte lines (from q itself, 4 head planes
+    // apart, it touched 32).  The 256-byte row is loaded before the stage is
     // known to be free, so the loads of one item overlap the wait for it.
     // Item metadata: records two items ahead, entries one item ahead.
     const int wg = (warp - 2) >> 2, qw = warp & 3, row = 32 * qw + lane, jr = row >> 2, h = row & 3;
@@ -274,14 +276,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int it = wg; it < nmine; it += 2) {
       const int sq = it % NQS, li = it / NQS;
       const bool valid = jr < m0.n;
-      const int b = m0.bg / s.Hkv, g = m0.bg - b * s.Hkv;
-      const __nv_bfloat16* src = q + ((long long)(b * s.Hq + g * G + h) * s.N + t0 + (e0 >> 6)) * D;
+      // regrouped rows (regroup_q_kernel): piece x of head h at (4 x + h) * 16
+      const __nv_bfloat16* src = qg + ((long long)m0.bg * PT + (e0 >> 6)) * (G * D) + h * 16;
       uint32_t w[64];
 #pragma unroll
       for (int x = 0; x < 8; ++x) {
         uint32_t t8[8];
         if (valid) {
-          ldg32(src + 16 * x, t8);
+          ldg32(src + 64 * x, t8);
         } else {
 #pragma unroll
           for (int y = 0; y < 8; ++y) t8[y] = 0u;
@@ -408,6 +410,22 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+// The query rows of positions [t0, t0 + np), regrouped per KV group as
+// qg[bg][p - t0][x][h][16 elements] (bg stride PT positions): 32-byte piece x
+// of the G = 4 heads side by side (1 KB per position).  One warp per (bg, position): lane 4 x + h
+// reads piece x of head h and the warp writes the position's 1 KB at once.
+__global__ void __launch_bounds__(256) regroup_q_kernel(Shape s, const __nv_bfloat16* __restrict__ q, int t0, int np,
+                                                        int PT, __nv_bfloat16* __restrict__ qg) {
+  const int lane = threadIdx.x & 31;
+  const long long w = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (w >= (long long)s.B * s.Hkv * np) return;
+  const int bg = (int)(w / np), pl = (int)(w - (long long)bg * np);
+  const int b = bg / s.Hkv, g = bg - b * s.Hkv, x = lane >> 2, h = lane & 3;
+  uint32_t t8[8];
+  ldg32(q + ((long long)(b * s.Hq + g * G + h) * s.N + t0 + pl) * D + 16 * x, t8);
+  stg32(qg + ((long long)bg * PT + pl) * (G * D) + lane * 16, t8);
 }
 
 // ------------------------------------------------------------ bucketing ----
@@ -550,7 +568,7 @@ size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // workspace pieces, in order
 struct ChunkWs {
-  size_t cnt, off, ioff, ent, items, part, total;
+  size_t cnt, off, ioff, ent, items, qg, part, total;
   int PT;
 };
 
@@ -580,6 +598,7 @@ ChunkWs chunk_ws(const Shape& s) {
   w.ioff = take((U + 1) * 4);
   w.ent = take(pairs * 4);
   w.items = take((pairs / PPI + U + 1) * 16);
+  w.qg = take((size_t)s.B * s.Hkv * w.PT * G * D * 2);
   w.part = take(pairs * G * D * 2);
   w.total = o;
   return w;
@@ -603,6 +622,7 @@ cudaError_t launch_attn_prefill_chunked(const Shape& s, const void* q, const voi
   int* ioff = (int*)(W + w.ioff);
   int* ent = (int*)(W + w.ent);
   int4* items = (int4*)(W + w.items);
+  __nv_bfloat16* qg = (__nv_bfloat16*)(W + w.qg);
   __nv_bfloat16* part = (__nv_bfloat16*)(W + w.part);
   const int U = s.B * s.Hkv * s.C;
 
@@ -628,8 +648,9 @@ cudaError_t launch_attn_prefill_chunked(const Shape& s, const void* q, const voi
       bucket_count_kernel<<<grid, 512, hsmem, st>>>(s, idx, t0, np, cnt, ctx);
       bucket_scan_kernel<<<1, 1024, 0, st>>>(U, cnt, off, ioff);
       bucket_scatter_kernel<<<grid, 512, hsmem, st>>>(s, idx, t0, np, off, ioff, cnt, ent, items);
-      attn_chunk_kernel<<<sms, THREADS, kSmemBytes, st>>>(s, tmk, tmv, (const __nv_bfloat16*)q, ioff, items, ent, t0,
-                                                          w.PT, part, ctx);
+      const long long nrows = (long long)s.B * s.Hkv * np;
+      regroup_q_kernel<<<(unsigned)((nrows + 7) / 8), 256, 0, st>>>(s, (const __nv_bfloat16*)q, t0, np, w.PT, qg);
+      attn_chunk_kernel<<<sms, THREADS, kSmemBytes, st>>>(s, tmk, tmv, ioff, items, ent, w.PT, qg, part, ctx);
       e = cudaGetLastError();
       if (e != cudaSuccess) return e;
     }
