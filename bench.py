@@ -138,9 +138,10 @@ def attention_stats(w, idx):
       (2 d S + 2 S d) FLOP of algorithmic selected-chunk work.
     * items: per position tile and bucket (sequence, group, chunk), ceil(n/32)
       items of 128 query rows; each executes 128 rows x 4 d S FLOP on tcgen05.
-    * window: each warp of the window pass covers 2 positions x 4 heads (8
-      rows) against every window chunk of its position pair (64 keys each,
-      causal keys masked inside the current chunk), 8 x 4 d S FLOP per chunk.
+    * window: an item of the window kernel is 32 aligned positions x 4 heads
+      (128 rows) of one group against every window chunk of its block (64
+      keys each, causal keys masked inside the current chunk); two passes,
+      S then S and P V: 128 x 6 d S FLOP per chunk.
     * union_over_k_m4: mean size of the union of the chunk sets of M = 4
       adjacent positions divided by K (rows with full lists), the reuse measure
       of grouping adjacent queries.
@@ -160,11 +161,11 @@ def attention_stats(w, idx):
         cnt = torch.bincount(u.long(), minlength=B * Hkv * C)
         items += int(((cnt + 31) // 32).sum().item())
     win_chunks = 0
-    for p0 in range(0, N, 2):
+    for p0 in range(0, N, 32):
         cur = p0 // S
         win_chunks += cur - max(0, cur - nw + 1) + 1
     exec_chunk = items * 128 * 4 * d * S
-    exec_win = B * Hkv * win_chunks * 8 * 4 * d * S
+    exec_win = B * Hkv * win_chunks * 128 * 6 * d * S
     M = 4
     nb = N // M
     blk = idx[:, :, : nb * M].reshape(B, Hkv, nb, M * K)
@@ -365,9 +366,9 @@ def cpu_baseline_prefill(w, x, budget_s=15.0, rows=None, seed=0):
 
 def prefill_launches(w) -> int:
     """Kernels one prefill step launches: summaries, [Q-Cal,] scoring, and per
-    attention position tile bucket count, scan, scatter, the chunk-major pass
-    and the window pass."""
-    return 2 + (1 if w.d_model else 0) + 5 * attn_tiles(w)
+    attention position tile bucket count, scan, scatter, the query regroup,
+    the chunk-major pass, the window pass and the fusion."""
+    return 2 + (1 if w.d_model else 0) + 7 * attn_tiles(w)
 
 
 def prefill_roofline(w, pre, ev, pk, pk_kind):
@@ -380,11 +381,11 @@ def prefill_roofline(w, pre, ev, pk, pk_kind):
     peak_tf = pk["bf16_tflops_sustained"]
     ach = attn_f / (t_attn / 1e3) / 1e12
     st = attention_stats(w, pre.idx)
-    roofline = {"kernel": f"hils_attn_prefill (attn_chunk_kernel + attn_ring_kernel<1> + bucketing, "
-                          f"{attn_tiles(w)} position tiles)",
+    roofline = {"kernel": f"hils_attn_prefill (attn_chunk_kernel + attn_window_kernel + attn_fuse_kernel + "
+                          f"bucketing, {attn_tiles(w)} position tiles)",
                 "bound": "tensor", "achieved": round(ach, 2),
                 "peak": peak_tf, "unit": "TFLOP/s", "frac": round(ach / peak_tf, 4),
-                "traffic": traffic_for(["attn_chunk.cu", "attn_ring.cu", "common.cuh"], "hils_attn_prefill", w.name),
+                "traffic": traffic_for(["attn_chunk.cu", "attn_window.cu", "common.cuh"], "hils_attn_prefill", w.name),
                 "peak_source": f"{pk_kind} bf16_tflops_sustained",
                 "algorithmic_flop_per_launch": attn_f,
                 "executed_flop_per_launch": st["executed_flop_per_launch"],
@@ -682,18 +683,19 @@ def main():
 def attn_tiles(w) -> int:
     """Position tiles of the chunk-major attention (hils.h, hils_attn_prefill):
     the fewest tiles whose 1 KB partial records (one per position, KV group and
-    selected chunk) fit about 8 GiB each.  Each tile launches five kernels:
-    bucket count, scan and scatter, the chunk-major pass, the window pass."""
+    selected chunk) fit about 8 GiB each.  Each tile launches seven kernels:
+    bucket count, scan and scatter, the query regroup, the chunk-major pass,
+    the window pass and the fusion."""
     per_pos = w.B * w.Hkv * w.K * w.G * w.d * 2
     cap = max(1, (8 << 30) // per_pos)
     return (w.N + cap - 1) // cap
 
 
 def attn_tile_positions(w) -> int:
-    """Positions per tile: N split evenly over the tiles, rounded up to 14."""
+    """Positions per tile: N split evenly over the tiles, rounded up to 64."""
     nt = attn_tiles(w)
     pt = -(-w.N // nt)
-    return -(-pt // 14) * 14
+    return -(-pt // 64) * 64
 
 
 def run_config(w, ws):

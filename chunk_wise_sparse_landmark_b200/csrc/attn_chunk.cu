@@ -16,8 +16,9 @@
 //   O (128 rows x 128 d)    = P (128 x 64) . V_c (64 x d)     tcgen05, fp32 in TMEM
 //
 // O is stored as one 1 KB bf16 record per (position, slot k of its selection
-// list; heads innermost) -- the "partial" -- and the window pass (attn_ring.cu) adds the window's
-// exact softmax terms and fuses the partials with the exp(s^) weights.
+// list; heads innermost) -- the "partial" -- and attn_window.cu attends the
+// window with its exact softmax terms and fuses the partials with the exp(s^)
+// weights.
 //
 // Why chunk-major: on the pages' i.i.d.-like workloads adjacent positions
 // share almost none of their selected chunks, so a position-major kernel
@@ -25,7 +26,7 @@
 // reads it back for 8 query rows.  Grouped by chunk, a tile serves ~100+ rows
 // and the work becomes dense tensor-core tiles; the price is the gathered
 // query rows (1 KB per pair, mostly L2 hits) and the partial records (1 KB per
-// pair written here, read once by the window pass).
+// pair written here, read once by the fusion kernel).
 //
 // Host-side bucketing (three small kernels per position tile): count the pairs
 // per (sequence, KV group, chunk) bucket, scan the counts into bucket offsets
@@ -105,29 +106,6 @@ HILS_DI void stg32(void* p, const uint32_t (&w)[8]) {
                "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
                : "memory");
 }
-// 32 lanes x 16 consecutive 32-bit columns <- 16 registers per thread
-HILS_DI void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
-          taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
-      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
-}
-// Shared-memory descriptor of an MN-major operand with the 128-byte swizzle:
-// 64 MN-elements per 128-byte row, rows of consecutive K 128 B apart in
-// 8-row (1024 B) atoms; `lbo` = bytes between 64-element MN blocks, `sbo` =
-// bytes between 8-row K groups.
-HILS_DI uint64_t sdesc_mn_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-  uint64_t d = 0;
-  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
-  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-  d |= (uint64_t)1u << 46;  // descriptor version (sm_100)
-  d |= (uint64_t)2u << 61;  // 128-byte swizzle
-  return d;
-}
-
 struct Item {
   int bg, c, s0, n;
 };
@@ -354,13 +332,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     // with u = 4 h2 + r / 2 (8 units of 128 bytes, heads innermost).  Unit
     // u's 32 bytes of a head hold pieces r and r + 1 of the head's 64-column
     // half h2 (r even); in piece r, element 4 a + t holds d = 64 h2 + 32 a +
-    // r + 8 t (a = 0..1, t = 0..3): the 8 values one thread of the window
-    // pass's MMA fragments consumes.  The 4 head rows of a position are 4
+    // r + 8 t (a = 0..1, t = 0..3): the values d = r (mod 8) of one half, the
+    // unit of one fusion-kernel lane.  The 4 head rows of a position are 4
     // adjacent lanes, so each warp store writes 8 whole 128-byte lines.
     // Measured at 128K: head-major records (each warp store touching 32
     // lines) cost ~7 ms of the attention; item-major blocks of 128 rows (one
-    // 512-byte run per store) were as fast to write but left the window pass
-    // reading 64-byte pieces 2 KB apart (17.5 ms against 13 ms); staging in
+    // 512-byte run per store) were as fast to write but left the record reader
+    // with 64-byte pieces 2 KB apart (17.5 ms against 13 ms); staging in
     // shared memory for 512-byte runs (41 ms, with spills) and bulk copies of
     // 1 KB records (32 ms) were slower.  Item metadata is fetched ahead.
     const int qw = warp & 3, row = 32 * qw + lane, jr = row >> 2, h = row & 3;
@@ -432,7 +410,7 @@ __global__ void __launch_bounds__(256) regroup_q_kernel(Shape s, const __nv_bflo
 // The lists of a position tile [t0, t0 + np): list r = bg * np + pl holds the
 // K entries of position t0 + pl in KV group bg.  One warp reads one list
 // (lane j: entries j and j + 32) and keeps the entries that have the list
-// form (accept_list_warp, common.cuh); the window pass applies the same rule
+// form (accept_list_warp, common.cuh); the fusion kernel applies the same rule
 // before it fuses the records, so both agree on every pair.
 HILS_DI void list_of(const Shape& s, const int32_t* __restrict__ idx, int t0, int np, long long r, int& bg, int& pl,
                      int& a, int& b, const DevCtx* report) {
@@ -568,15 +546,15 @@ size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // workspace pieces, in order
 struct ChunkWs {
-  size_t cnt, off, ioff, ent, items, qg, part, total;
+  size_t cnt, off, ioff, ent, items, qg, wst, part, total;
   int PT;
 };
 
 // Positions per tile: the fewest tiles whose partial records fit about
-// kPartBudget bytes each, of equal size rounded up to a multiple of the window
-// pass's block (14 positions).
+// kPartBudget bytes each, of equal size rounded up to a multiple of a chunk
+// (the window pass's 32-position blocks then never straddle a tile).
 constexpr size_t kPartBudget = size_t(8) << 30;
-constexpr int kRingBlock = 14;
+constexpr int kTileAlign = 64;
 
 ChunkWs chunk_ws(const Shape& s) {
   ChunkWs w{};
@@ -584,7 +562,7 @@ ChunkWs chunk_ws(const Shape& s) {
   const long long cap = std::max<long long>(1, (long long)(kPartBudget / per_pos));
   const long long ntiles = (s.N + cap - 1) / cap;
   const long long pt = (s.N + ntiles - 1) / ntiles;
-  w.PT = (int)((pt + kRingBlock - 1) / kRingBlock * kRingBlock);
+  w.PT = (int)((pt + kTileAlign - 1) / kTileAlign * kTileAlign);
   const size_t U = (size_t)s.B * s.Hkv * s.C;
   const size_t pairs = (size_t)s.B * s.Hkv * w.PT * s.K;
   size_t o = 0;
@@ -599,6 +577,7 @@ ChunkWs chunk_ws(const Shape& s) {
   w.ent = take(pairs * 4);
   w.items = take((pairs / PPI + U + 1) * 16);
   w.qg = take((size_t)s.B * s.Hkv * w.PT * G * D * 2);
+  w.wst = take(window_state_bytes(s, w.PT));
   w.part = take(pairs * G * D * 2);
   w.total = o;
   return w;
@@ -624,6 +603,7 @@ cudaError_t launch_attn_prefill_chunked(const Shape& s, const void* q, const voi
   int4* items = (int4*)(W + w.items);
   __nv_bfloat16* qg = (__nv_bfloat16*)(W + w.qg);
   __nv_bfloat16* part = (__nv_bfloat16*)(W + w.part);
+  void* wst = W + w.wst;
   const int U = s.B * s.Hkv * s.C;
 
   CUtensorMap tmk, tmv;
@@ -654,7 +634,7 @@ cudaError_t launch_attn_prefill_chunked(const Shape& s, const void* q, const voi
       e = cudaGetLastError();
       if (e != cudaSuccess) return e;
     }
-    e = launch_attn_window_merge(s, q, k, v, idx, s_sel, out, U > 0 ? part : nullptr, t0, t0 + np, w.PT, st, ctx);
+    e = launch_attn_window_fused(s, q, k, v, idx, s_sel, out, part, wst, t0, np, w.PT, st, ctx);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

@@ -126,19 +126,18 @@ struct Walk {
   int slot0 = 0, slot1 = 0;  // positions in the two lists (s^ lookup)
 };
 
-template <bool PART>
 __global__ void __launch_bounds__(THREADS, 2)
     attn_ring_kernel(Shape s, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                      const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ idx,
                      const float* __restrict__ s_sel, __nv_bfloat16* __restrict__ out,
-                     const __nv_bfloat16* __restrict__ part, int t0, int t1, int PT, DevCtx ctx) {
+                     DevCtx ctx) {
   extern __shared__ unsigned char smem_raw[];
   SmemR& sm = *reinterpret_cast<SmemR*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = blockIdx.y, b = blockIdx.z;
   const int bg = b * s.Hkv + g;
-  const int i0 = t0 + blockIdx.x * BP;
-  const int nend = min(s.N, t1);  // this launch's positions: [t0, nend)
+  const int i0 = blockIdx.x * BP;
+  const int nend = s.N;
   const int K = s.K;
   // stream: selected chunks below lo (bitmap, ascending), then every chunk lo..hi
   const int lo = max(0, i0 / S - s.nw + 1);    // first window chunk of the block
@@ -184,10 +183,6 @@ __global__ void __launch_bounds__(THREADS, 2)
     accept_list_warp(l1a, l1b, K, ncand, bad1);
     if ((bad0 || bad1) && lane == 0) raise_status(ctx, kStatusBadIndex);
   }
-  // with partial records the selected chunks were attended elsewhere: the
-  // lists are kept for the fusion at the end and the stream is the window only
-  const int m0a = l0a, m0b = l0b, m1a = l1a, m1b = l1b;
-  if (PART) l0a = l0b = l1a = l1b = -1;
   if (warp < CW) {
     if (l0a >= 0 && l0a < lo) atomicOr(&sm.bits[l0a >> 5], 1u << (l0a & 31));
     if (l0b >= 0 && l0b < lo) atomicOr(&sm.bits[l0b >> 5], 1u << (l0b & 31));
@@ -496,59 +491,6 @@ __global__ void __launch_bounds__(THREADS, 2)
       if (lane == 0) mbar_arrive(&sm.empty[vit % NSI]);
     }
 
-    // ---- selected chunks from their partial records O_c (attn_chunk.cu):
-    // acc += e^{s^ - m} O_c, den += e^{s^ - m}.  A record is [unit][head][32 B]
-    // (attn_chunk.cu); piece (hh, gq) of a head, 16 bytes in unit 4 hh + gq/2
-    // at half gq % 2, holds this thread's values d = 64 hh + 32 a + gq + 8 t
-    // at element 4 a + t (a = 0..1, t = 0..3), i.e. d = 16 mt + gq (+ 8) for
-    // mt = 4 hh + 2 a + t/2.  MSL slots are loaded at a time (predicated, no branch)
-    // so that their HBM round trips overlap.
-    if (PART && ok) {
-      const __nv_bfloat16* rec =
-          part + (((long long)bg * PT + (my_pos - t0)) * K) * (G * D) + (gq >> 1) * (G * 16) + (gq & 1) * 8;
-      for (int x0 = 0; x0 < K; x0 += MSL) {
-        uint4 w[MSL][2][2];
-        float wg[MSL][2];
-#pragma unroll
-        for (int j = 0; j < MSL; ++j) {
-          const int x = x0 + j;
-          const int ca = entry(m0a, m0b, x), cb = entry(m1a, m1b, x);
-          const bool v = my_valid && (my_q == 0 ? ca : cb) >= 0;
-          const __nv_bfloat16* rx = rec + (long long)x * (G * D);
-#pragma unroll
-          for (int r = 0; r < 2; ++r) {
-            float sv = -INFINITY;
-            if (v) sv = __ldg(ss0 + r * sstride + x);
-            wg[j][r] = sv;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              uint4 u = make_uint4(0u, 0u, 0u, 0u);
-              if (v) u = __ldg(reinterpret_cast<const uint4*>(rx + hh * (4 * G * 16) + (my_h + r) * 16));
-              w[j][r][hh] = u;
-            }
-          }
-        }
-#pragma unroll
-        for (int j = 0; j < MSL; ++j)
-#pragma unroll
-          for (int r = 0; r < 2; ++r) {
-            const float wgt = exp2f(wg[j][r] * kLog2e - m2[r]);  // 0 for skipped slots
-            den[r] += wgt;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              const uint32_t ww[4] = {w[j][r][hh].x, w[j][r][hh].y, w[j][r][hh].z, w[j][r][hh].w};
-#pragma unroll
-              for (int q2 = 0; q2 < 4; ++q2) {  // a = q2 / 2, t pair = q2 % 2
-                const int mt = 4 * hh + q2;
-                const float2 f = bf16x2_to_f32x2(ww[q2]);
-                acc[mt][r] = fmaf(wgt, f.x, acc[mt][r]);
-                acc[mt][2 + r] = fmaf(wgt, f.y, acc[mt][2 + r]);
-              }
-            }
-          }
-      }
-    }
-
     // ---- epilogue: thread holds d = 16 mt + gq (acc[mt][0/1]) and 16 mt + gq + 8
     // (acc[mt][2/3]) of its rows 2c4, 2c4+1 (position my_pos, heads my_h, my_h + 1);
     // the 8 lanes of a quad column write 16 consecutive bytes per store
@@ -571,11 +513,9 @@ constexpr size_t kSmemBytes = sizeof(SmemR) + 1024;
 
 }  // namespace
 
-cudaError_t launch_attn_window_merge(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
-                                     const float* s_sel, void* out, const void* part, int t0, int t1, int PT,
-                                     cudaStream_t st, const DevCtx& ctx) {
+cudaError_t launch_attn_prefill_tc(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
+                                   const float* s_sel, void* out, cudaStream_t st, const DevCtx& ctx) {
   if (s.d != D || s.S != S || s.G != G || s.K > KMAX || s.C > MAXC || s.nw > 32) return cudaErrorNotSupported;
-  if (t0 % 2 || t1 <= t0) return cudaErrorInvalidValue;
   CUtensorMap tmk, tmv;
   const uint64_t dims[3] = {(uint64_t)D, (uint64_t)s.N, (uint64_t)s.B * s.Hkv};
   const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)s.N * D * 2};
@@ -584,18 +524,12 @@ cudaError_t launch_attn_window_merge(const Shape& s, const void* q, const void* 
   if (e != cudaSuccess) return e;
   e = make_tmap_bf16(&tmv, v, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
-  auto kern = part ? attn_ring_kernel<true> : attn_ring_kernel<false>;
-  e = ensure_dynamic_smem((const void*)kern, (int)kSmemBytes);
+  e = ensure_dynamic_smem((const void*)attn_ring_kernel, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid((t1 - t0 + BP - 1) / BP, s.Hkv, s.B);
-  kern<<<grid, THREADS, kSmemBytes, st>>>(s, tmk, tmv, (const __nv_bfloat16*)q, idx, s_sel, (__nv_bfloat16*)out,
-                                          (const __nv_bfloat16*)part, t0, t1, PT, ctx);
+  dim3 grid((s.N + BP - 1) / BP, s.Hkv, s.B);
+  attn_ring_kernel<<<grid, THREADS, kSmemBytes, st>>>(s, tmk, tmv, (const __nv_bfloat16*)q, idx, s_sel,
+                                                      (__nv_bfloat16*)out, ctx);
   return cudaGetLastError();
-}
-
-cudaError_t launch_attn_prefill_tc(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
-                                   const float* s_sel, void* out, cudaStream_t st, const DevCtx& ctx) {
-  return launch_attn_window_merge(s, q, k, v, idx, s_sel, out, nullptr, 0, s.N, 0, st, ctx);
 }
 
 }  // namespace hils

@@ -81,14 +81,17 @@ cudaError_t launch_attn_prefill_simt(const Shape& s, const void* q, const void* 
 // chunk union (no workspace)
 cudaError_t launch_attn_prefill_tc(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
                                    const float* s_sel, void* out, cudaStream_t st, const DevCtx& ctx);
-// the window pass over positions [t0, t1); with `part` (partial records of the
-// selected chunks, tile of PT positions) it attends the window only and fuses
-// the records, without it it also streams the selected chunks
-cudaError_t launch_attn_window_merge(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
-                                     const float* s_sel, void* out, const void* part, int t0, int t1, int PT,
-                                     cudaStream_t st, const DevCtx& ctx);
-// bf16 prefill attention, chunk-major selected chunks (tcgen05) + window pass,
-// by position tiles; workspace of attn_prefill_tc_workspace(s) bytes
+// window attention (tcgen05, two passes over the window chunks) of positions
+// [t0, t0 + np) of a tile of PT positions (t0 a multiple of 32) into the
+// window state (window_state_bytes(s, PT)), then the fusion with the partial
+// records `part` of the selected chunks into out
+size_t window_state_bytes(const Shape& s, int PT);
+cudaError_t launch_attn_window_fused(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
+                                     const float* s_sel, void* out, const void* part, void* wstate, int t0, int np,
+                                     int PT, cudaStream_t st, const DevCtx& ctx);
+// bf16 prefill attention, chunk-major selected chunks (tcgen05) + window
+// attention and fusion (attn_window.cu), by position tiles; workspace of
+// attn_prefill_tc_workspace(s) bytes
 size_t attn_prefill_tc_workspace(const Shape& s);
 cudaError_t launch_attn_prefill_chunked(const Shape& s, const void* q, const void* k, const void* v,
                                         const int32_t* idx, const float* s_sel, void* out, void* ws,

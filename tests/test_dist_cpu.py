@@ -64,7 +64,7 @@ def test_attention_tiles_and_traffic_lookup():
     assert bench.attn_tiles(WORKLOADS["prefill_128k"]) == 4
     assert bench.attn_tiles(WORKLOADS["prefill_512k_qcal"]) == 32
     assert bench.attn_tiles(WORKLOADS["prefill_8k"]) == 1
-    files = ["attn_chunk.cu", "attn_ring.cu"]
+    files = ["attn_chunk.cu", "attn_window.cu", "common.cuh"]
     t = bench.traffic_for(files, "hils_attn_prefill", "prefill_128k")
     assert t is None or t > 0
     assert bench.traffic_for(["attn_chunk.cu"], "hils_attn_prefill", "prefill_128k") is None  # other sources
