@@ -186,8 +186,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           tma_load_3d(sm.v[sk][1], &tmv, 64, im.c * S, im.bg, &sm.kvfull[sk]);
         }
       }
-      // copies still in flight (only after a timeout) land before the CTA exits
-      if (!ok && ctx.inject != 1)
+      // the copies issued last land before the CTA exits, whichever role gave
+      // up first (their phases completed long ago on the normal path)
+      if (ctx.inject != 1)
         for (int j = max(0, it - NKV); j < it; ++j) mbar_wait(&sm.kvfull[j % NKV], (j / NKV) & 1, ctx);
     }
     __syncwarp();

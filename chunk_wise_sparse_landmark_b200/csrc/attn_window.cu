@@ -126,7 +126,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // for each w (the MMA warp's order), V_{n-1} last
     if (lane == 0) {
       bool ok = true;
-      int kt = 0;  // K/V tiles issued
+      int kt = 0, nq = 0;  // K/V tiles and query tiles issued
       if (nmine > 0) {
         prefetch_tmap(&tmq);
         prefetch_tmap(&tmk);
@@ -153,6 +153,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int h = 0; h < G; ++h)
           for (int hf = 0; hf < 2; ++hf)
             tma_load_3d(sm.q[qb][hf] + h * QHEAD, &tmq, 64 * hf, im.p0, b * s.Hq + g * G + h, &sm.qfull[qb]);
+        ++nq;
         for (int w = 0; w < im.n && ok; ++w) ok = tile(false, im.wc0 + w, im.bg);
         if (ok) ok = tile(false, im.wc0, im.bg);
         for (int w = 0; w < im.n && ok; ++w) {
@@ -160,9 +161,10 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (ok) ok = tile(true, im.wc0 + w, im.bg);
         }
       }
-      // copies still in flight (only after a timeout) land before the CTA exits
-      if (!ok)
-        for (int j = std::max(0, kt - NKV); j < kt; ++j) mbar_wait(&sm.kvfull[j % NKV], (j / NKV) & 1, ctx);
+      // the copies issued last land before the CTA exits, whichever role gave
+      // up first (their phases completed long ago on the normal path)
+      for (int j = std::max(0, kt - NKV); j < kt; ++j) mbar_wait(&sm.kvfull[j % NKV], (j / NKV) & 1, ctx);
+      for (int j = std::max(0, nq - 2); j < nq; ++j) mbar_wait(&sm.qfull[j & 1], (j >> 1) & 1, ctx);
     }
     __syncwarp();
   } else if (warp == 1) {
