@@ -135,9 +135,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       auto tile = [&](bool isv, int c, int bg) -> bool {
         const int x = kt % NKV;
         if (kt >= NKV && !mbar_wait(&sm.kvempty[x], ((kt / NKV) - 1) & 1, ctx)) return false;
-        mbar_arrive_expect_tx(&sm.kvfull[x], 2 * BOX);
-        tma_load_3d(sm.kv[x][0], isv ? &tmv : &tmk, 0, c * S, bg, &sm.kvfull[x]);
-        tma_load_3d(sm.kv[x][1], isv ? &tmv : &tmk, 64, c * S, bg, &sm.kvfull[x]);
+        if (ctx.inject != 1) {  // host fault injection: no copy, the consumers' waits run out
+          mbar_arrive_expect_tx(&sm.kvfull[x], 2 * BOX);
+          tma_load_3d(sm.kv[x][0], isv ? &tmv : &tmk, 0, c * S, bg, &sm.kvfull[x]);
+          tma_load_3d(sm.kv[x][1], isv ? &tmv : &tmk, 64, c * S, bg, &sm.kvfull[x]);
+        }
         ++kt;
         return true;
       };
@@ -149,11 +151,13 @@ __global__ void __launch_bounds__(THREADS, 1)
           break;
         }
         const int b = im.bg / s.Hkv, g = im.bg - b * s.Hkv;
-        mbar_arrive_expect_tx(&sm.qfull[qb], 2 * QHALF);
-        for (int h = 0; h < G; ++h)
-          for (int hf = 0; hf < 2; ++hf)
-            tma_load_3d(sm.q[qb][hf] + h * QHEAD, &tmq, 64 * hf, im.p0, b * s.Hq + g * G + h, &sm.qfull[qb]);
-        ++nq;
+        if (ctx.inject != 1) {
+          mbar_arrive_expect_tx(&sm.qfull[qb], 2 * QHALF);
+          for (int h = 0; h < G; ++h)
+            for (int hf = 0; hf < 2; ++hf)
+              tma_load_3d(sm.q[qb][hf] + h * QHEAD, &tmq, 64 * hf, im.p0, b * s.Hq + g * G + h, &sm.qfull[qb]);
+          ++nq;
+        }
         for (int w = 0; w < im.n && ok; ++w) ok = tile(false, im.wc0 + w, im.bg);
         if (ok) ok = tile(false, im.wc0, im.bg);
         for (int w = 0; w < im.n && ok; ++w) {
@@ -163,7 +167,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       // the copies issued last land before the CTA exits, whichever role gave
       // up first (their phases completed long ago on the normal path)
-      for (int j = std::max(0, kt - NKV); j < kt; ++j) mbar_wait(&sm.kvfull[j % NKV], (j / NKV) & 1, ctx);
+      if (ctx.inject != 1)
+        for (int j = std::max(0, kt - NKV); j < kt; ++j) mbar_wait(&sm.kvfull[j % NKV], (j / NKV) & 1, ctx);
       for (int j = std::max(0, nq - 2); j < nq; ++j) mbar_wait(&sm.qfull[j & 1], (j >> 1) & 1, ctx);
     }
     __syncwarp();
