@@ -139,9 +139,9 @@ def attention_stats(w, idx):
     * items: per position tile and bucket (sequence, group, chunk), ceil(n/32)
       items of 128 query rows; each executes 128 rows x 4 d S FLOP on tcgen05.
     * window: an item of the window kernel is 32 aligned positions x 4 heads
-      (128 rows) of one group against every window chunk of its block (64
-      keys each, causal keys masked inside the current chunk); two passes,
-      S then S and P V: 128 x 6 d S FLOP per chunk.
+      (128 rows) of one group against its block's window chunks, taken two at
+      a time (an odd count padded with one chunk whose keys are all masked);
+      two passes, S then S and P V: 128 x 6 d S FLOP per chunk taken.
     * union_over_k_m4: mean size of the union of the chunk sets of M = 4
       adjacent positions divided by K (rows with full lists), the reuse measure
       of grouping adjacent queries.
@@ -163,7 +163,7 @@ def attention_stats(w, idx):
     win_chunks = 0
     for p0 in range(0, N, 32):
         cur = p0 // S
-        win_chunks += cur - max(0, cur - nw + 1) + 1
+        win_chunks += 2 * ((cur - max(0, cur - nw + 1) + 2) // 2)
     exec_chunk = items * 128 * 4 * d * S
     exec_win = B * Hkv * win_chunks * 128 * 6 * d * S
     M = 4
