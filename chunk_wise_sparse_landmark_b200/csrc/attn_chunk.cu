@@ -64,6 +64,7 @@
 //     one 256-byte bulk copy per row) did not complete, and are not used.
 // Every wait is bounded (status word + early return), see common.cuh.
 #include <algorithm>
+#include <mutex>
 
 #include "launch.h"
 #include "tmap.h"
@@ -545,6 +546,25 @@ __global__ void bucket_scatter_kernel(Shape s, const int32_t* __restrict__ idx, 
 
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// A side stream and its events per device, made on first use.  g_side_mu is
+// held for a whole call's enqueue, so concurrent calls never record an event
+// that another call is about to wait on.
+struct Side {
+  cudaStream_t st = nullptr;
+  cudaEvent_t start = nullptr, next = nullptr, win = nullptr;
+};
+Side g_side[64];
+std::mutex g_side_mu;
+
+cudaError_t side_init(Side& sd) {
+  cudaError_t e = cudaSuccess;
+  if (!sd.st) e = cudaStreamCreateWithFlags(&sd.st, cudaStreamNonBlocking);
+  if (e == cudaSuccess && !sd.start) e = cudaEventCreateWithFlags(&sd.start, cudaEventDisableTiming);
+  if (e == cudaSuccess && !sd.next) e = cudaEventCreateWithFlags(&sd.next, cudaEventDisableTiming);
+  if (e == cudaSuccess && !sd.win) e = cudaEventCreateWithFlags(&sd.win, cudaEventDisableTiming);
+  return e;
+}
+
 // workspace pieces, in order
 struct ChunkWs {
   size_t cnt, off, ioff, ent, items, qg, wst, part, total;
@@ -578,7 +598,7 @@ ChunkWs chunk_ws(const Shape& s) {
   w.ent = take(pairs * 4);
   w.items = take((pairs / PPI + U + 1) * 16);
   w.qg = take((size_t)s.B * s.Hkv * w.PT * G * D * 2);
-  w.wst = take(window_state_bytes(s, w.PT));
+  w.wst = take(2 * window_state_bytes(s, w.PT));  // two tiles' window states
   w.part = take(pairs * G * D * 2);
   w.total = o;
   return w;
@@ -604,7 +624,6 @@ cudaError_t launch_attn_prefill_chunked(const Shape& s, const void* q, const voi
   int4* items = (int4*)(W + w.items);
   __nv_bfloat16* qg = (__nv_bfloat16*)(W + w.qg);
   __nv_bfloat16* part = (__nv_bfloat16*)(W + w.part);
-  void* wst = W + w.wst;
   const int U = s.B * s.Hkv * s.C;
 
   CUtensorMap tmk, tmv;
@@ -619,6 +638,31 @@ cudaError_t launch_attn_prefill_chunked(const Shape& s, const void* q, const voi
   if (e != cudaSuccess) return e;
   const int sms = device_sm_count();
 
+  // The window kernel of tile t + 1 runs on a side stream beside the fusion of
+  // tile t (an HBM-bound kernel with room beside it on every SM); the chunk
+  // kernel, which fills the SMs, runs alone.  Order per tile on `st`:
+  // bucketing, regroup, [wait window(t)] chunk(t), [window(t + 1) starts on the
+  // side stream], fusion(t).  The window state is double-buffered by tile.
+  WindowMaps wm;
+  e = make_window_maps(s, q, k, v, &wm);
+  if (e != cudaSuccess) return e;
+  const size_t wsb = window_state_bytes(s, w.PT);
+  auto wstate = [&](int t0) -> void* { return W + w.wst + ((t0 / w.PT) & 1) * wsb; };
+  int dev = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_side_mu);  // one call's records and waits at a time
+  Side& sd = g_side[dev];
+  e = side_init(sd);
+  if (e != cudaSuccess) return e;
+  // the side stream starts after the work already on `st` (inputs, workspace)
+  e = cudaEventRecord(sd.start, st);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(sd.st, sd.start, 0);
+  if (e == cudaSuccess) e = launch_attn_window(s, wm, wstate(0), 0, std::min(w.PT, s.N), w.PT, sd.st, ctx);
+  if (e == cudaSuccess) e = cudaEventRecord(sd.win, sd.st);
+  if (e != cudaSuccess) return e;
+
   for (int t0 = 0; t0 < s.N; t0 += w.PT) {
     const int np = std::min(w.PT, s.N - t0);
     if (U > 0) {
@@ -631,11 +675,25 @@ cudaError_t launch_attn_prefill_chunked(const Shape& s, const void* q, const voi
       bucket_scatter_kernel<<<grid, 512, hsmem, st>>>(s, idx, t0, np, off, ioff, cnt, ent, items);
       const long long nrows = (long long)s.B * s.Hkv * np;
       regroup_q_kernel<<<(unsigned)((nrows + 7) / 8), 256, 0, st>>>(s, (const __nv_bfloat16*)q, t0, np, w.PT, qg);
+    }
+    e = cudaStreamWaitEvent(st, sd.win, 0);  // window(t) done
+    if (e != cudaSuccess) return e;
+    if (U > 0) {
       attn_chunk_kernel<<<sms, THREADS, kSmemBytes, st>>>(s, tmk, tmv, ioff, items, ent, w.PT, qg, part, ctx);
       e = cudaGetLastError();
       if (e != cudaSuccess) return e;
     }
-    e = launch_attn_window_fused(s, q, k, v, idx, s_sel, out, part, wst, t0, np, w.PT, st, ctx);
+    if (t0 + w.PT < s.N) {
+      // window(t + 1) overwrites the state that fusion(t - 1), earlier on `st`, read
+      e = cudaEventRecord(sd.next, st);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(sd.st, sd.next, 0);
+      const int t1 = t0 + w.PT;
+      if (e == cudaSuccess)
+        e = launch_attn_window(s, wm, wstate(t1), t1, std::min(w.PT, s.N - t1), w.PT, sd.st, ctx);
+      if (e == cudaSuccess) e = cudaEventRecord(sd.win, sd.st);
+      if (e != cudaSuccess) return e;
+    }
+    e = launch_attn_fuse(s, idx, s_sel, part, wstate(t0), out, t0, np, w.PT, st);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

@@ -484,34 +484,44 @@ __global__ void __launch_bounds__(FW * 32) attn_fuse_kernel(Shape s, const int32
 
 size_t window_state_bytes(const Shape& s, int PT) { return (size_t)s.B * s.Hkv * PT * G * (8 * 16 + 2) * 4; }
 
-cudaError_t launch_attn_window_fused(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
-                                     const float* s_sel, void* out, const void* part, void* wstate, int t0, int np,
-                                     int PT, cudaStream_t st, const DevCtx& ctx) {
+cudaError_t make_window_maps(const Shape& s, const void* q, const void* k, const void* v, WindowMaps* m) {
   if (s.d != D || s.S != S || s.G != G || s.K > KMAX || s.nw < 1) return cudaErrorNotSupported;
-  if (t0 % BPOS || np < 1 || np > PT || !part || !wstate) return cudaErrorInvalidValue;
-  CUtensorMap tmq, tmk, tmv;
   const uint64_t qdims[3] = {(uint64_t)D, (uint64_t)s.N, (uint64_t)s.B * s.Hq};
   const uint64_t kdims[3] = {(uint64_t)D, (uint64_t)s.N, (uint64_t)s.B * s.Hkv};
   const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)s.N * D * 2};
   const uint32_t qbox[3] = {64, (uint32_t)BPOS, 1};
   const uint32_t kbox[3] = {64, (uint32_t)TK, 1};
-  cudaError_t e = make_tmap_bf16(&tmq, q, 3, qdims, strides, qbox, CU_TENSOR_MAP_SWIZZLE_128B);
+  cudaError_t e = make_tmap_bf16(&m->q, q, 3, qdims, strides, qbox, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
-  e = make_tmap_bf16(&tmk, k, 3, kdims, strides, kbox, CU_TENSOR_MAP_SWIZZLE_128B);
+  e = make_tmap_bf16(&m->k, k, 3, kdims, strides, kbox, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
-  e = make_tmap_bf16(&tmv, v, 3, kdims, strides, kbox, CU_TENSOR_MAP_SWIZZLE_128B);
+  return make_tmap_bf16(&m->v, v, 3, kdims, strides, kbox, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// window state: accumulators [B Hkv][PT][8][G][16], then (m', l) [B Hkv][PT][G][2]
+static float* window_md(const Shape& s, void* wstate, int PT) {
+  return (float*)wstate + (size_t)s.B * s.Hkv * PT * 8 * G * 16;
+}
+
+cudaError_t launch_attn_window(const Shape& s, const WindowMaps& m, void* wstate, int t0, int np, int PT,
+                               cudaStream_t st, const DevCtx& ctx) {
+  if (t0 % BPOS || np < 1 || np > PT || !wstate) return cudaErrorInvalidValue;
+  cudaError_t e = ensure_dynamic_smem((const void*)attn_window_kernel, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  e = ensure_dynamic_smem((const void*)attn_window_kernel, (int)kSmemBytes);
-  if (e != cudaSuccess) return e;
-  // window state: accumulators [B Hkv][PT][8][G][16], then (m', l) [B Hkv][PT][G][2]
-  float* wacc = (float*)wstate;
-  float* wmd = wacc + (size_t)s.B * s.Hkv * PT * 8 * G * 16;
   const int nitems = s.B * s.Hkv * ((np + BPOS - 1) / BPOS);
   const int grid = std::min(nitems, device_sm_count());
-  attn_window_kernel<<<grid, THREADS, kSmemBytes, st>>>(s, tmq, tmk, tmv, t0, np, PT, wacc, wmd, ctx);
+  attn_window_kernel<<<grid, THREADS, kSmemBytes, st>>>(s, m.q, m.k, m.v, t0, np, PT, (float*)wstate,
+                                                        window_md(s, wstate, PT), ctx);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_fuse(const Shape& s, const int32_t* idx, const float* s_sel, const void* part,
+                             const void* wstate, void* out, int t0, int np, int PT, cudaStream_t st) {
+  if (np < 1 || np > PT || !part || !wstate) return cudaErrorInvalidValue;
   const long long rows = (long long)s.B * s.Hkv * np;
   attn_fuse_kernel<<<(unsigned)((rows + FW - 1) / FW), FW * 32, 0, st>>>(
-      s, idx, s_sel, (const __nv_bfloat16*)part, wacc, wmd, (__nv_bfloat16*)out, t0, np, PT);
+      s, idx, s_sel, (const __nv_bfloat16*)part, (const float*)wstate, window_md(s, (void*)wstate, PT),
+      (__nv_bfloat16*)out, t0, np, PT);
   return cudaGetLastError();
 }
 

@@ -8,6 +8,7 @@
 #include <stdint.h>
 
 #include "common.cuh"
+#include "tmap.h"
 
 namespace hils {
 
@@ -81,14 +82,20 @@ cudaError_t launch_attn_prefill_simt(const Shape& s, const void* q, const void* 
 // chunk union (no workspace)
 cudaError_t launch_attn_prefill_tc(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
                                    const float* s_sel, void* out, cudaStream_t st, const DevCtx& ctx);
-// window attention (tcgen05, two passes over the window chunks) of positions
-// [t0, t0 + np) of a tile of PT positions (t0 a multiple of 32) into the
-// window state (window_state_bytes(s, PT)), then the fusion with the partial
-// records `part` of the selected chunks into out
+// window attention (tcgen05, two passes over the window chunks, attn_window.cu)
+// of positions [t0, t0 + np) of a tile of PT positions (t0 a multiple of 32)
+// into a window state of window_state_bytes(s, PT); then the fusion of that
+// state with the partial records `part` of the selected chunks into out.  The
+// tensor maps of q, k, v are made once per call.
+struct WindowMaps {
+  CUtensorMap q, k, v;
+};
 size_t window_state_bytes(const Shape& s, int PT);
-cudaError_t launch_attn_window_fused(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
-                                     const float* s_sel, void* out, const void* part, void* wstate, int t0, int np,
-                                     int PT, cudaStream_t st, const DevCtx& ctx);
+cudaError_t make_window_maps(const Shape& s, const void* q, const void* k, const void* v, WindowMaps* m);
+cudaError_t launch_attn_window(const Shape& s, const WindowMaps& m, void* wstate, int t0, int np, int PT,
+                               cudaStream_t st, const DevCtx& ctx);
+cudaError_t launch_attn_fuse(const Shape& s, const int32_t* idx, const float* s_sel, const void* part,
+                             const void* wstate, void* out, int t0, int np, int PT, cudaStream_t st);
 // bf16 prefill attention, chunk-major selected chunks (tcgen05) + window
 // attention and fusion (attn_window.cu), by position tiles; workspace of
 // attn_prefill_tc_workspace(s) bytes

@@ -78,9 +78,9 @@ def test_attn_prefill_workspace_size():
     (U + 1 ints each, U = B Hkv C buckets), the pairs of one position tile
     (ints), the item table (int4: bucket, first pair, count; at most
     pairs / 32 + U + 1 items), the tile's query rows regrouped per KV group
-    (1 KB per position and group), the window pass's fp32 state (4 heads x
-    (128 accumulators + reference exponent + sum) per position and group) and
-    one 1 KB bf16 partial record per pair; the fewest equal tiles whose
+    (1 KB per position and group), the window pass's fp32 state for two
+    tiles (4 heads x (128 accumulators + reference exponent + sum) per
+    position and group) and one 1 KB bf16 partial record per pair; the fewest equal tiles whose
     records fit about 8 GiB, rounded up to a multiple of 64 positions."""
     up = lambda n: (n + 255) // 256 * 256
     B, N, Hq, Hkv, K = 1, 131072, 32, 8, 32
@@ -92,14 +92,14 @@ def test_attn_prefill_workspace_size():
     assert (ntiles, PT) == (4, 32768)
     U, pairs = B * Hkv * (N // 64), B * Hkv * PT * K
     want = (3 * up((U + 1) * 4) + up(pairs * 4) + up((pairs // 32 + U + 1) * 16) + up(pairs // K * 1024)
-            + up(pairs // K * 2080) + up(pairs * 1024))
+            + up(2 * (pairs // K) * 2080) + up(pairs * 1024))
     assert H.workspace_bytes(cfg, H.HILS_WS_ATTN_PREFILL) == want
     # short sequences: one tile of N rounded up to 64 positions
     small = H.make_config(2, 1000, 8, 2, 128, 64, 128, 8, "bf16")
     PT, U = 1024, 2 * 2 * (1000 // 64)
     pairs = 2 * 2 * PT * 8
     want = (3 * up((U + 1) * 4) + up(pairs * 4) + up((pairs // 32 + U + 1) * 16) + up(pairs // 8 * 1024)
-            + up(pairs // 8 * 2080) + up(pairs * 1024))
+            + up(2 * (pairs // 8) * 2080) + up(pairs * 1024))
     assert H.workspace_bytes(small, H.HILS_WS_ATTN_PREFILL) == want
     assert H.workspace_bytes(H.make_config(1, 512, 4, 1, 64, 32, 64, 4, "f32"), H.HILS_WS_ATTN_PREFILL) == 0
     lib = H.load()
