@@ -429,18 +429,24 @@ __global__ void __launch_bounds__(THREADS, 1)
           // (measured: writing each head's 32 scores to a per-thread column of
           // shared memory and reading the chosen ones by index was slower,
           // 10.8 against 8.6 ms at 128K, than this select tree per chosen chunk)
+          constexpr int HE = KT <= 32 ? 2 : 1;  // heads per TMEM wait, as in the score loop
 #pragma unroll
-          for (int hh = 0; hh < G; ++hh) {
-            uint32_t v[HALF];
-            tmem_ld32(lane_addr + DCOL + hh * 64 + hf * HALF, v);
+          for (int h0 = 0; h0 < G; h0 += HE) {
+            uint32_t v[HE][HALF];
+#pragma unroll
+            for (int u = 0; u < HE; ++u) tmem_ld32(lane_addr + DCOL + (h0 + u) * 64 + hf * HALF, v[u]);
             tmem_wait_ld();
-            float* dst = s_sel + (((long long)b * s.Hq + g * G + hh) * s.N + i) * K;
-            uint32_t rem = sel;
-            for (int k = 0; __any_sync(0xffffffffu, k < nmine); ++k) {
-              const int j = (__ffs(rem) - 1) & 31;  // 31 once this lane has no more (unused)
-              rem &= rem - 1u;
-              const float x = __uint_as_float(pick32(v, j));
-              if (k < nmine && base + k < K) dst[base + k] = __fmaf_rn(x, scale, sm.bt[par][hh][hf * HALF + j]);
+#pragma unroll
+            for (int u = 0; u < HE; ++u) {
+              const int hh = h0 + u;
+              float* dst = s_sel + (((long long)b * s.Hq + g * G + hh) * s.N + i) * K;
+              uint32_t rem = sel;
+              for (int k = 0; __any_sync(0xffffffffu, k < nmine); ++k) {
+                const int j = (__ffs(rem) - 1) & 31;  // 31 once this lane has no more (unused)
+                rem &= rem - 1u;
+                const float x = __uint_as_float(pick32(v[u], j));
+                if (k < nmine && base + k < K) dst[base + k] = __fmaf_rn(x, scale, sm.bt[par][hh][hf * HALF + j]);
+              }
             }
           }
         }
