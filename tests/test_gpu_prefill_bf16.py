@@ -98,12 +98,44 @@ def test_attn_forced_selection_wide_window_k64(chunked):
 
 def test_attn_forced_selection_several_position_tiles():
     """B Hkv K = 1024 partial records per position: 8 GiB hold 8192 positions,
-    so this sequence runs as two position tiles (4508 + 4492)."""
+    so this sequence runs as two position tiles (4544 + 4456, multiples of a
+    chunk)."""
     w = WORKLOADS["prefill_512k_qcal"].scaled(name="tiles", B=4, N=9000, Hq=16, Hkv=4, d_model=0, qcal_rank=0,
                                               needles_per_head=2)
     assert w.B * w.Hkv * w.K == 1024
     err, _, _ = _run_forced(w, prefill_inputs(w))
     assert err <= TOL_BF16, err
+
+
+def test_attn_chunk_major_graph_capture_matches_eager():
+    """The chunk-major pass runs the next position tile's window kernel on an
+    internal stream and joins it back with events.  Captured into a CUDA graph
+    (two position tiles) and replayed, the call gives the eager output bit for
+    bit; a side-stream launch left unjoined would make the capture fail."""
+    w = WORKLOADS["prefill_512k_qcal"].scaled(name="tiles", B=4, N=9000, Hq=16, Hkv=4, d_model=0, qcal_rank=0,
+                                              needles_per_head=2)
+    x = prefill_inputs(w)
+    d = {n: x[n].to(DEV) for n in ("q", "k", "v", "q_lmk")}
+    pre = H.Prefill(H.config_of(w), DEV)
+    pre.run(d["q"], d["k"], d["v"], d["q_lmk"])
+    H.hils_sync_status()
+    ref = pre.out.clone()
+    st = torch.cuda.Stream()
+    with torch.cuda.stream(st):  # one eager call on the capture stream first
+        H.hils_attn_prefill(pre.cfg, d["q"], d["k"], d["v"], pre.idx, pre.s_sel, pre.out, pre.ws_attn, st)
+    torch.cuda.synchronize()
+    H.hils_sync_status()
+    assert torch.equal(pre.out, ref)
+    pre.out.zero_()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=st):
+        H.hils_attn_prefill(pre.cfg, d["q"], d["k"], d["v"], pre.idx, pre.s_sel, pre.out, pre.ws_attn, st)
+    g.replay()
+    torch.cuda.synchronize()
+    H.hils_sync_status()
+    assert torch.equal(pre.out, ref)
+    del g
 
 
 def test_attn_chunk_major_is_deterministic_and_matches_union_stream():
