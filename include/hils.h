@@ -162,16 +162,20 @@ hils_status_t hils_score_topk(const hils_config_t* cfg, const void* q, const hil
  * as HILS_ERR_INVALID_ARG.
  *   workspace: device scratch of at least
  *              hils_workspace_bytes(cfg, HILS_WS_ATTN_PREFILL, 0) bytes
- *              (16-byte aligned; 0 bytes for dtype F32).  With it, bf16 runs
- *              attend the selected chunks chunk by chunk (the positions that
- *              chose a chunk share one load of its K and V tiles), write one
- *              bf16 partial record per (position, selected chunk) into the
- *              workspace and fuse the records in the window pass, by tiles of
- *              positions whose records fit the workspace (about 8 GiB).
- *              workspace = NULL with ws_bytes = 0 selects the pass that needs
- *              no scratch: each block of 14 positions streams the union of its
- *              chunks (slower on long contexts; same results within the bf16
- *              tolerance).  The call owns the workspace until the stream passes it.
+ *              (16-byte aligned; 0 bytes for dtype F32; about 10 GB at
+ *              B=1, N=128K, Hkv=8, K=32).  With it, bf16 runs attend the
+ *              selected chunks chunk by chunk (the positions that chose a
+ *              chunk share one load of its K and V tiles) and write one bf16
+ *              partial record per (position, selected chunk) into the
+ *              workspace, attend each position's window on the tensor cores,
+ *              and fuse the two, by tiles of positions whose records fit about
+ *              8 GiB.  Part of this work runs on an internal stream that waits
+ *              on and is joined back into `stream` by events, so the call may
+ *              be captured into a CUDA graph.  workspace = NULL with
+ *              ws_bytes = 0 selects the pass that needs no scratch: each block
+ *              of 14 positions streams the union of its chunks (slower on long
+ *              contexts; same results within the bf16 tolerance).  The call
+ *              owns the workspace until the stream passes it.
  */
 hils_status_t hils_attn_prefill(const hils_config_t* cfg, const void* q, const void* k, const void* v,
                                 const int32_t* idx, const float* s_sel, void* out, void* workspace,
