@@ -22,7 +22,7 @@
  *        each query attends each retrieved chunk on its own and the chunk
  *        outputs are fused by the retrieval scores.
  *
- * Readings where the pages leave a step open (each is listed in the design doc):
+ * Readings where the pages leave a step open:
  *   - window of query i = keys [max(0,(cur(i)-n_w+1)*S), i], cur(i)=floor(i/S),
  *     n_w = W/S; candidates = complete chunks c <= cur(i)-n_w;
  *   - the landmark softmax uses the same 1/sqrt(d) temperature as the
