@@ -96,6 +96,19 @@ def test_attn_forced_selection_wide_window_k64(chunked):
     assert err <= TOL_BF16, err
 
 
+@PASSES
+@pytest.mark.parametrize("window", [64, 192], ids=["one_chunk", "three_chunks"])
+def test_attn_forced_selection_odd_window_chunk_counts(chunked, window):
+    """Windows of 1 and 3 chunks: the window kernel takes chunks two at a time,
+    so every item of these windows pads its last tile with a chunk whose keys
+    all lie after the position (masked), not only the first items of a
+    sequence."""
+    w = WORKLOADS["prefill_8k"].scaled(name=f"w{window}", B=2, N=3000 + 19, Hq=8, Hkv=2, W=window, K=8,
+                                       needles_per_head=2)
+    err, _, _ = _run_forced(w, prefill_inputs(w), chunked)
+    assert err <= TOL_BF16, err
+
+
 def test_attn_forced_selection_several_position_tiles():
     """B Hkv K = 1024 partial records per position: 8 GiB hold 8192 positions,
     so this sequence runs as two position tiles (4544 + 4456, multiples of a
