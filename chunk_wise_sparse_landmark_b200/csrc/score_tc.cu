@@ -21,16 +21,20 @@
 //
 // Selection is exact and deterministic.  Pass 1 streams every tile; each
 // epilogue thread keeps the multiset of the KT >= K largest group scores of
-// its half, sorted in registers, updated by branch-free insertion of the few
-// candidates above its current KT-th value, or, while a tile brings many of
-// them (a row's first tiles), by sorting the tile's 32 candidates with a
-// bitonic network and merging the two sorted lists.  After the last tile the row's
+// its half, sorted in registers.  The candidates of a tile that beat the
+// list's current KT-th value are appended to the thread's column of a
+// shared-memory buffer; once some lane of the warp holds 32 of them, the warp
+// sorts 32 buffered values per lane with a bitonic network and merges them
+// into its list (a handful of merges per row instead of one insertion per
+// candidate).  After the last tile the row's
 // threshold tau (its K-th largest score) is the minimum over j < K of
 // max(a_j, b_{K-1-j}) for the two halves' sorted lists a, b, and A = the
 // number of scores above tau.  Pass 2 recomputes the same tiles (same
 // instructions, bit-identical scores) and emits, in ascending chunk order,
 // every candidate scoring above tau plus the first K - A scoring exactly tau
-// (ties go to the smaller chunk), with each head's own s^.
+// (ties go to the smaller chunk), with each head's own s^.  For K <= 32 the
+// chosen chunks and scores are staged in shared memory and leave, after the
+// last tile, as whole rows (consecutive threads, consecutive addresses).
 #include "launch.h"
 #include "tmap.h"
 
@@ -46,20 +50,31 @@ constexpr int KMAX = 64;
 constexpr int NMMA = G;   // MMA-issuing warps, one per head
 constexpr int EPI = 256;  // epilogue threads
 constexpr int THREADS = 32 * NMMA + EPI;
-constexpr int STG = 16;   // survivors staged per thread and round
+constexpr int CAP = 64;   // buffered candidates per epilogue thread (<= 31 carried + one tile's 32)
+constexpr int RS = MQ + 1;  // row stride of the staged selection (conflict-free both ways)
 constexpr uint32_t BBOX = TCH * 128;       // one [64 chunks x 64 d] bf16 box
 constexpr uint32_t BSTAGE = G * 2 * BBOX;  // 64 KB
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACOL = 0;    // A: head h at ACOL + 64 h
 constexpr uint32_t DCOL = 256;  // D: head h at DCOL + 64 h
 
+// staging of the chosen chunks in pass 2: scores [G][KT][RS], then chunks [KT][RS]
+template <int KT>
+constexpr int kSelFloats = KT <= 32 ? (G + 1) * KT * RS : 0;
+template <int KT>
+constexpr int kAreaFloats = kSelFloats<KT> > CAP * EPI ? kSelFloats<KT> : CAP * EPI;
+
+template <int KT>
 struct __align__(1024) SmemS {
   unsigned char b[NST][G][2][BBOX];
-  float stage[STG][EPI];          // staged survivors; [32][MQ] half-merge area after pass 1
+  // pass 1: candidate buffer [CAP][EPI]; after it the [32][MQ] half-merge area;
+  // pass 2 (K <= 32): the staged selection
+  float area[kAreaFloats<KT>];
   alignas(16) float bt[2][G][TCH];  // b' of the tile, by tile parity
   uint8_t cnt[2][2][2][MQ];       // pass 2, by tile parity: [half][above / equal][row]
   float tau[MQ];
   int nab[2][MQ];
+  int nselr[MQ];
   uint64_t bfull[NST], bempty[NST], dfull, dempty, afull, done;
   uint32_t tmem;
 };
@@ -75,14 +90,6 @@ HILS_DI bool epi_all(bool v) {
       : "r"((uint32_t)v)
       : "memory");
   return out != 0;
-}
-
-// insert x into the descending list a (x = -inf leaves it unchanged)
-template <int KT>
-HILS_DI void insert_desc(float (&a)[KT], float x) {
-#pragma unroll
-  for (int j = KT - 1; j > 0; --j) a[j] = fmaxf(fminf(a[j - 1], x), a[j]);
-  a[0] = fmaxf(a[0], x);
 }
 
 // sort 32 values descending in registers (bitonic network, 240 compare-exchanges)
@@ -146,7 +153,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                          const float* __restrict__ b_sum, int32_t* __restrict__ idx, float* __restrict__ s_sel,
                          DevCtx ctx) {
   extern __shared__ unsigned char smem_raw[];
-  SmemS& sm = *reinterpret_cast<SmemS*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  SmemS<KT>& sm = *reinterpret_cast<SmemS<KT>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = blockIdx.y, b = blockIdx.z;
   const int i0 = blockIdx.x * MQ;
@@ -248,7 +255,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int i = i0 + r;
     const bool valid = i < s.N;
     const uint32_t lane_addr = tmem + ((uint32_t)(qd * 32) << 16);
-    float(*mrg)[MQ] = reinterpret_cast<float(*)[MQ]>(&sm.stage[0][0]);
+    float(*mrg)[MQ] = reinterpret_cast<float(*)[MQ]>(&sm.area[0]);
+    float* buf = &sm.area[et];  // this thread's candidate column: buf[x * EPI]
+    float* sval = &sm.area[0];  // staged scores [G][KT][RS]
+    int* sidx = reinterpret_cast<int*>(&sm.area[G * KT * RS]);  // staged chunks [KT][RS]
+    constexpr bool kStaged = KT <= 32;
     // A: this row's scoring query, heads 2 hf and 2 hf + 1 -> TMEM
     for (int hh = 2 * hf; hh < 2 * hf + 2; ++hh) {
       const uint4* src =
@@ -280,6 +291,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     float tau = -INFINITY;  // pass 2: the row's K-th largest group score
     int t_rem = 0;          // pass 2: scores equal to tau still to take
     int nsel = 0;
+    int nb = 0;             // pass 1: candidates in this thread's buffer column
     const long long row_idx = (((long long)b * s.Hkv + g) * s.N + i) * K;
     bool ok = true;
 
@@ -328,40 +340,35 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.dempty);
-        // candidates above the current KT-th value: when any lane of the warp
-        // has many (the first tiles of a row), the tile is sorted and merged
-        // into the list (~670 operations); otherwise each is staged and
-        // inserted (~63 operations each)
-        const float thr0 = top[KT - 1];
-        int nab = 0;
+        // candidates above the list's current KT-th value join the buffer; a
+        // warp merges when any lane has a tile's worth (32) buffered, and the
+        // last tile flushes everything (at most two merges, nb <= 63)
+        const float thr = top[KT - 1];
+        const int jn = ncand - c0;
 #pragma unroll
-        for (int j = 0; j < HALF; ++j) nab += (c0 + j < ncand && gv[j] > thr0) ? 1 : 0;
-        const bool bulk = __any_sync(0xffffffffu, nab >= 8);  // measured at 128K: 8 beats 2-6 and 12-20
-        if (bulk) {
-#pragma unroll
-          for (int j = 0; j < HALF; ++j) gv[j] = (c0 + j < ncand && gv[j] > thr0) ? gv[j] : -INFINITY;
-          sort32_desc(gv);
-          merge_top<KT>(top, gv);
-        }
-#pragma unroll
-        for (int rd = 0; rd < HALF / STG; ++rd) {
-          if (bulk) break;  // warp-uniform
-          const float thr = top[KT - 1];
-          int ns = 0;
-#pragma unroll
-          for (int j = 0; j < STG; ++j) {
-            const int jj = rd * STG + j;
-            if (c0 + jj < ncand && gv[jj] > thr) {
-              sm.stage[ns][et] = gv[jj];
-              ++ns;
-            }
+        for (int j = 0; j < HALF; ++j) {
+          if (j < jn && gv[j] > thr) {
+            buf[nb * EPI] = gv[j];
+            ++nb;
           }
-          for (int k = 0; __any_sync(0xffffffffu, k < ns); ++k) insert_desc(top, k < ns ? sm.stage[k][et] : -INFINITY);
+        }
+        const bool flush = t == T - 1;  // CTA-uniform
+        while (__any_sync(0xffffffffu, flush ? nb > 0 : nb >= HALF)) {
+          float bb[HALF];
+#pragma unroll
+          for (int x = 0; x < HALF; ++x) bb[x] = x < nb ? buf[x * EPI] : -INFINITY;
+          sort32_desc(bb);
+          merge_top<KT>(top, bb);
+          const int rest = max(nb - HALF, 0);
+#pragma unroll
+          for (int x = 0; x < HALF - 1; ++x)
+            if (x < rest) buf[x * EPI] = buf[(HALF + x) * EPI];
+          nb = rest;
         }
         if (t == T - 1) {
           // row threshold from the two halves' sorted lists a (half 0), b (half 1):
           // tau = min_{j<K} max(a_j, b_{K-1-j})
-          epi_barrier();  // staging reads done before the area is reused
+          epi_barrier();  // buffer reads done before the area is reused
           float tmin = INFINITY;
 #pragma unroll
           for (int rd = 0; rd < (KT + 31) / 32; ++rd) {
@@ -422,7 +429,10 @@ __global__ void __launch_bounds__(THREADS, 1)
               if (k < nmine) {
                 const int j = __ffs(rem) - 1;
                 rem &= rem - 1u;
-                if (base + k < K) idx[row_idx + base + k] = c0 + j;
+                if (base + k < K) {
+                  if constexpr (kStaged) sidx[(base + k) * RS + r] = c0 + j;
+                  else idx[row_idx + base + k] = c0 + j;
+                }
               }
             }
           }
@@ -445,7 +455,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const int j = (__ffs(rem) - 1) & 31;  // 31 once this lane has no more (unused)
                 rem &= rem - 1u;
                 const float x = __uint_as_float(pick32(v[u], j));
-                if (k < nmine && base + k < K) dst[base + k] = __fmaf_rn(x, scale, sm.bt[par][hh][hf * HALF + j]);
+                if (k < nmine && base + k < K) {
+                  const float y = __fmaf_rn(x, scale, sm.bt[par][hh][hf * HALF + j]);
+                  if constexpr (kStaged) sval[(hh * KT + base + k) * RS + r] = y;
+                  else dst[base + k] = y;
+                }
               }
             }
           }
@@ -455,8 +469,27 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (lane == 0) mbar_arrive(&sm.dempty);
       }
     }
-    if (valid && ok && hf == 0) {
-      if (nsel != min(ncand, K)) raise_status(ctx, kStatusBadIndex);
+    if (valid && ok && hf == 0 && nsel != min(ncand, K)) raise_status(ctx, kStatusBadIndex);
+    if constexpr (kStaged) {
+      // the staged rows leave whole: element f = row * K + slot of the CTA's
+      // rows, consecutive threads at consecutive addresses; slots past the
+      // row's selection get -1 / -inf
+      if (hf == 0) sm.nselr[r] = min(nsel, K);
+      epi_barrier();
+      if (ok) {
+        const int tot = (min(i0 + MQ, s.N) - i0) * K;
+        int32_t* idx0 = idx + (((long long)b * s.Hkv + g) * s.N + i0) * K;
+        for (int f = et; f < tot; f += EPI) {
+          const int rr = f / K, k = f - rr * K;
+          const bool on = k < sm.nselr[rr];
+          idx0[f] = on ? sidx[k * RS + rr] : -1;
+#pragma unroll
+          for (int hh = 0; hh < G; ++hh)
+            s_sel[(((long long)b * s.Hq + g * G + hh) * s.N + i0) * K + f] =
+                on ? sval[(hh * KT + k) * RS + rr] : -INFINITY;
+        }
+      }
+    } else if (valid && ok && hf == 0) {
       nsel = min(nsel, K);
       for (int x = nsel; x < K; ++x) {
         idx[row_idx + x] = -1;
@@ -473,15 +506,16 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-constexpr size_t kSmemBytes = sizeof(SmemS) + 1024;
+template <int KT>
+constexpr size_t kSmemBytes = sizeof(SmemS<KT>) + 1024;
 
 template <int KT>
 cudaError_t launch_kt(const Shape& s, const CUtensorMap& tmk, const void* q, const float* b_sum, int32_t* idx,
                       float* s_sel, cudaStream_t st, const DevCtx& ctx) {
-  cudaError_t e = ensure_dynamic_smem((const void*)score_topk_tc_kernel<KT>, (int)kSmemBytes);
+  cudaError_t e = ensure_dynamic_smem((const void*)score_topk_tc_kernel<KT>, (int)kSmemBytes<KT>);
   if (e != cudaSuccess) return e;
   dim3 grid((s.N + MQ - 1) / MQ, s.Hkv, s.B);
-  score_topk_tc_kernel<KT><<<grid, THREADS, kSmemBytes, st>>>(s, tmk, (const __nv_bfloat16*)q, b_sum, idx, s_sel,
+  score_topk_tc_kernel<KT><<<grid, THREADS, kSmemBytes<KT>, st>>>(s, tmk, (const __nv_bfloat16*)q, b_sum, idx, s_sel,
                                                                ctx);
   return cudaGetLastError();
 }
