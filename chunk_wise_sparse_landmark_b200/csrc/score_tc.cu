@@ -32,9 +32,12 @@
 // number of scores above tau.  Pass 2 recomputes the same tiles (same
 // instructions, bit-identical scores) and emits, in ascending chunk order,
 // every candidate scoring above tau plus the first K - A scoring exactly tau
-// (ties go to the smaller chunk), with each head's own s^.  For K <= 32 the
-// chosen chunks and scores are staged in shared memory and leave, after the
-// last tile, as whole rows (consecutive threads, consecutive addresses).
+// (ties go to the smaller chunk), with each head's own s^.  Pass 2 reads the
+// four heads' scores from TMEM once per tile and releases the accumulator
+// before selecting, so that the next tile's MMAs overlap its selection and
+// emission.  For K <= 32 the chosen chunks and scores are staged in shared
+// memory and leave, after the last tile, as whole rows (consecutive threads,
+// consecutive addresses).
 #include "launch.h"
 #include "tmap.h"
 
@@ -70,7 +73,8 @@ struct __align__(1024) SmemS {
   // pass 1: candidate buffer [CAP][EPI]; after it the [32][MQ] half-merge area;
   // pass 2 (K <= 32): the staged selection
   float area[kAreaFloats<KT>];
-  alignas(16) float bt[2][G][TCH];  // b' of the tile, by tile parity
+  alignas(16) float bt[2][G][TCH];  // b' of the tile, by tile parity, head-major
+  alignas(16) float btj[2][TCH][G];  // the same, heads innermost
   uint8_t cnt[2][2][2][MQ];       // pass 2, by tile parity: [half][above / equal][row]
   float tau[MQ];
   int nab[2][MQ];
@@ -80,6 +84,8 @@ struct __align__(1024) SmemS {
 };
 
 HILS_DI void epi_barrier() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+// barrier of the two epilogue warps that hold the same rows (lane quadrant qd)
+HILS_DI void row_pair_barrier(int qd) { asm volatile("bar.sync %0, 64;" ::"r"(2 + qd) : "memory"); }
 // barrier among the epilogue warps that also ANDs a flag, so that all of them
 // take the same branch (nobody is left waiting at a later barrier)
 HILS_DI bool epi_all(bool v) {
@@ -131,20 +137,6 @@ HILS_DI void merge_top(float (&top)[KT], const float (&b)[32]) {
         top[l] = fminf(x, y);
       }
     }
-}
-
-// v[j] for a runtime j in [0, 32), by a tree of selects (no local memory)
-HILS_DI uint32_t pick32(const uint32_t (&v)[32], int j) {
-  uint32_t a[16], c[8], d[4], e[2];
-#pragma unroll
-  for (int t = 0; t < 16; ++t) a[t] = (j & 16) ? v[t + 16] : v[t];
-#pragma unroll
-  for (int t = 0; t < 8; ++t) c[t] = (j & 8) ? a[t + 8] : a[t];
-#pragma unroll
-  for (int t = 0; t < 4; ++t) d[t] = (j & 4) ? c[t + 4] : c[t];
-#pragma unroll
-  for (int t = 0; t < 2; ++t) e[t] = (j & 2) ? d[t + 2] : d[t];
-  return (j & 1) ? e[1] : e[0];
 }
 
 template <int KT>
@@ -295,20 +287,28 @@ __global__ void __launch_bounds__(THREADS, 1)
     const long long row_idx = (((long long)b * s.Hkv + g) * s.N + i) * K;
     bool ok = true;
 
-    for (int it = 0; it < NIT; ++it) {
-      const int pass = it >= T ? 1 : 0, t = it - pass * T, par = it & 1;
-      const int c0 = t * TCH + hf * HALF;  // first chunk of this thread's half
-      // b' of the tile: thread et fetches head et / 64, chunk et % 64
+    // b' of tile t for every head: thread et fetches head et / 64, chunk
+    // et % 64, in two layouts (head-major for pass 1, heads innermost for
+    // pass 2); the barrier of the landed vote publishes them.  The buffer of
+    // this parity was last read two tiles ago, before the previous vote.
+    auto stage_bias = [&](int t, int par) {
       const int bh = et >> 6, bj = et & 63, bc = t * TCH + bj;
       const float bval = bc < s.C ? __ldg(b_sum + ((long long)b * s.Hq + g * G + bh) * s.C + bc) : 0.f;
+      sm.bt[par][bh][bj] = bval;
+      sm.btj[par][bj][bh] = bval;
+    };
+
+    // pass 1
+    for (int it = 0; it < T; ++it) {
+      const int t = it, par = it & 1;
+      const int c0 = t * TCH + hf * HALF;  // first chunk of this thread's half
+      stage_bias(t, par);
       const bool landed = mbar_wait(&sm.dfull, it & 1, ctx);
       if (!epi_all(landed)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      sm.bt[par][bh][bj] = bval;
-      epi_barrier();
       // group score of each chunk of this half: max over heads of v * scale + b'
       float gv[HALF];
       constexpr int HW = KT <= 32 ? 2 : 1;  // heads loaded per TMEM wait
@@ -318,6 +318,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int u = 0; u < HW; ++u) tmem_ld32(lane_addr + DCOL + (h0 + u) * 64 + hf * HALF, v[u]);
         tmem_wait_ld();
+        if (h0 + HW == G) {
+          // the accumulator is read: the next tile's MMAs may start
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.dempty);
+        }
 #pragma unroll
         for (int u = 0; u < HW; ++u) {
           const int hh = h0 + u;
@@ -336,137 +342,146 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
       }
-      if (pass == 0) {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.dempty);
-        // candidates above the list's current KT-th value join the buffer; a
-        // warp merges when any lane has a tile's worth (32) buffered, and the
-        // last tile flushes everything (at most two merges, nb <= 63)
-        const float thr = top[KT - 1];
-        const int jn = ncand - c0;
+      // candidates above the list's current KT-th value join the buffer; a
+      // warp merges when any lane has a tile's worth (32) buffered, and the
+      // last tile flushes everything (at most two merges, nb <= 63)
+      const float thr = top[KT - 1];
+      const int jn = ncand - c0;
 #pragma unroll
-        for (int j = 0; j < HALF; ++j) {
-          if (j < jn && gv[j] > thr) {
-            buf[nb * EPI] = gv[j];
-            ++nb;
-          }
+      for (int j = 0; j < HALF; ++j) {
+        if (j < jn && gv[j] > thr) {
+          buf[nb * EPI] = gv[j];
+          ++nb;
         }
-        const bool flush = t == T - 1;  // CTA-uniform
-        while (__any_sync(0xffffffffu, flush ? nb > 0 : nb >= HALF)) {
-          float bb[HALF];
+      }
+      const bool flush = t == T - 1;  // CTA-uniform
+      while (__any_sync(0xffffffffu, flush ? nb > 0 : nb >= HALF)) {
+        float bb[HALF];
 #pragma unroll
-          for (int x = 0; x < HALF; ++x) bb[x] = x < nb ? buf[x * EPI] : -INFINITY;
-          sort32_desc(bb);
-          merge_top<KT>(top, bb);
-          const int rest = max(nb - HALF, 0);
+        for (int x = 0; x < HALF; ++x) bb[x] = x < nb ? buf[x * EPI] : -INFINITY;
+        sort32_desc(bb);
+        merge_top<KT>(top, bb);
+        const int rest = max(nb - HALF, 0);
 #pragma unroll
-          for (int x = 0; x < HALF - 1; ++x)
-            if (x < rest) buf[x * EPI] = buf[(HALF + x) * EPI];
-          nb = rest;
-        }
-        if (t == T - 1) {
-          // row threshold from the two halves' sorted lists a (half 0), b (half 1):
-          // tau = min_{j<K} max(a_j, b_{K-1-j})
-          epi_barrier();  // buffer reads done before the area is reused
-          float tmin = INFINITY;
+        for (int x = 0; x < HALF - 1; ++x)
+          if (x < rest) buf[x * EPI] = buf[(HALF + x) * EPI];
+        nb = rest;
+      }
+      if (t == T - 1) {
+        // row threshold from the two halves' sorted lists a (half 0), b (half 1):
+        // tau = min_{j<K} max(a_j, b_{K-1-j})
+        epi_barrier();  // buffer reads done before the area is reused
+        float tmin = INFINITY;
 #pragma unroll
-          for (int rd = 0; rd < (KT + 31) / 32; ++rd) {
-            if (hf == 1) {
+        for (int rd = 0; rd < (KT + 31) / 32; ++rd) {
+          if (hf == 1) {
 #pragma unroll
-              for (int x = 0; x < 32; ++x)
-                if (32 * rd + x < KT) mrg[x][r] = top[min(32 * rd + x, KT - 1)];
-            }
-            epi_barrier();
-            if (hf == 0) {
-#pragma unroll
-              for (int j = 0; j < KT; ++j) {
-                const int jb = K - 1 - j - 32 * rd;
-                if (j < K && jb >= 0 && jb < 32) tmin = fminf(tmin, fmaxf(top[j], mrg[jb][r]));
-              }
-            }
-            epi_barrier();
+            for (int x = 0; x < 32; ++x)
+              if (32 * rd + x < KT) mrg[x][r] = top[min(32 * rd + x, KT - 1)];
           }
-          if (hf == 0) sm.tau[r] = tmin;
           epi_barrier();
-          tau = sm.tau[r];
-          int above = 0;
+          if (hf == 0) {
 #pragma unroll
-          for (int j = 0; j < KT; ++j) above += top[j] > tau ? 1 : 0;
-          sm.nab[hf][r] = above;
-          epi_barrier();
-          t_rem = max(0, K - (sm.nab[0][r] + sm.nab[1][r]));
-        }
-      } else {
-        uint32_t gt = 0u, eq = 0u;
-#pragma unroll
-        for (int j = 0; j < HALF; ++j) {
-          if (c0 + j < ncand) {
-            if (gv[j] > tau) gt |= 1u << j;
-            else if (gv[j] == tau) eq |= 1u << j;
+            for (int j = 0; j < KT; ++j) {
+              const int jb = K - 1 - j - 32 * rd;
+              if (j < K && jb >= 0 && jb < 32) tmin = fminf(tmin, fmaxf(top[j], mrg[jb][r]));
+            }
           }
+          epi_barrier();
         }
-        sm.cnt[par][hf][0][r] = (uint8_t)__popc(gt);
-        sm.cnt[par][hf][1][r] = (uint8_t)__popc(eq);
+        if (hf == 0) sm.tau[r] = tmin;
         epi_barrier();
-        const int g0 = sm.cnt[par][0][0][r], e0 = sm.cnt[par][0][1][r];
-        const int g1 = sm.cnt[par][1][0][r], e1 = sm.cnt[par][1][1][r];
-        const int take0 = min(e0, t_rem), take1 = min(e1, t_rem - take0);
-        uint32_t sel = gt, em = eq;
-        for (int x = 0; x < (hf ? take1 : take0); ++x) {
-          sel |= em & (0u - em);
-          em &= em - 1u;
+        tau = sm.tau[r];
+        int above = 0;
+#pragma unroll
+        for (int j = 0; j < KT; ++j) above += top[j] > tau ? 1 : 0;
+        sm.nab[hf][r] = above;
+        epi_barrier();
+        t_rem = max(0, K - (sm.nab[0][r] + sm.nab[1][r]));
+      }
+    }
+
+    // pass 2: the four heads' scores are read from TMEM once per tile and the
+    // accumulator is released at once, so that the next tile's MMAs overlap the
+    // selection and the emission below
+    for (int it = T; it < 2 * T && ok; ++it) {
+      const int t = it - T, par = it & 1;
+      const int c0 = t * TCH + hf * HALF;
+      stage_bias(t, par);
+      const bool landed = mbar_wait(&sm.dfull, it & 1, ctx);
+      if (!epi_all(landed)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t v[G][HALF];
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) tmem_ld32(lane_addr + DCOL + hh * 64 + hf * HALF, v[hh]);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.dempty);
+      // the same group scores as pass 1 (same operations, same order)
+      const float4* bq = reinterpret_cast<const float4*>(&sm.btj[par][hf * HALF][0]);
+      uint32_t gt = 0u, eq = 0u;
+      const int jn = ncand - c0;  // candidates of this half: j < jn
+#pragma unroll
+      for (int j = 0; j < HALF; ++j) {
+        const float4 bb = bq[j];
+        float x = __fmaf_rn(__uint_as_float(v[0][j]), scale, bb.x);
+        x = fmaxf(x, __fmaf_rn(__uint_as_float(v[1][j]), scale, bb.y));
+        x = fmaxf(x, __fmaf_rn(__uint_as_float(v[2][j]), scale, bb.z));
+        x = fmaxf(x, __fmaf_rn(__uint_as_float(v[3][j]), scale, bb.w));
+        if (j < jn) {
+          if (x > tau) gt |= 1u << j;
+          else if (x == tau) eq |= 1u << j;
         }
-        const int base = nsel + (hf ? g0 + take0 : 0);
-        nsel += g0 + take0 + g1 + take1;
-        t_rem -= take0 + take1;
-        if (__any_sync(0xffffffffu, sel != 0u)) {
-          // one pass per selected chunk of the busiest lane (usually one or two)
-          const int nmine = __popc(sel);
-          {
-            uint32_t rem = sel;
-            for (int k = 0; __any_sync(0xffffffffu, k < nmine); ++k) {
-              if (k < nmine) {
-                const int j = __ffs(rem) - 1;
-                rem &= rem - 1u;
-                if (base + k < K) {
-                  if constexpr (kStaged) sidx[(base + k) * RS + r] = c0 + j;
-                  else idx[row_idx + base + k] = c0 + j;
-                }
+      }
+      // the two threads of a row (warps qd and qd + 4) exchange their counts
+      sm.cnt[par][hf][0][r] = (uint8_t)__popc(gt);
+      sm.cnt[par][hf][1][r] = (uint8_t)__popc(eq);
+      row_pair_barrier(qd);
+      const int g0 = sm.cnt[par][0][0][r], e0 = sm.cnt[par][0][1][r];
+      const int g1 = sm.cnt[par][1][0][r], e1 = sm.cnt[par][1][1][r];
+      const int take0 = min(e0, t_rem), take1 = min(e1, t_rem - take0);
+      uint32_t sel = gt, em = eq;
+      for (int x = 0; x < (hf ? take1 : take0); ++x) {
+        sel |= em & (0u - em);
+        em &= em - 1u;
+      }
+      const int base = nsel + (hf ? g0 + take0 : 0);
+      nsel += g0 + take0 + g1 + take1;
+      t_rem -= take0 + take1;
+      if (__any_sync(0xffffffffu, sel != 0u)) {
+        // the chosen chunks of this half take slots base, base + 1, ... in
+        // ascending chunk order; one predicated step per chunk, from registers
+        // (measured at 128K: a select tree per chosen chunk and head, fed by a
+        // second TMEM read, was 2.4 ms of the kernel)
+        int slot = base;
+#pragma unroll
+        for (int j = 0; j < HALF; ++j) {
+          if (sel & (1u << j)) {
+            if (slot < K) {
+              // b' from the head-major copy: the four loads of the mask loop
+              // above are not kept alive across it
+              const float* bh = &sm.bt[par][0][hf * HALF + j];
+              const float y[G] = {__fmaf_rn(__uint_as_float(v[0][j]), scale, bh[0]),
+                                  __fmaf_rn(__uint_as_float(v[1][j]), scale, bh[TCH]),
+                                  __fmaf_rn(__uint_as_float(v[2][j]), scale, bh[2 * TCH]),
+                                  __fmaf_rn(__uint_as_float(v[3][j]), scale, bh[3 * TCH])};
+              if constexpr (kStaged) {
+                sidx[slot * RS + r] = c0 + j;
+#pragma unroll
+                for (int hh = 0; hh < G; ++hh) sval[(hh * KT + slot) * RS + r] = y[hh];
+              } else {
+                idx[row_idx + slot] = c0 + j;
+#pragma unroll
+                for (int hh = 0; hh < G; ++hh) s_sel[(((long long)b * s.Hq + g * G + hh) * s.N + i) * K + slot] = y[hh];
               }
             }
-          }
-          // (measured: writing each head's 32 scores to a per-thread column of
-          // shared memory and reading the chosen ones by index was slower,
-          // 10.8 against 8.6 ms at 128K, than this select tree per chosen chunk)
-          constexpr int HE = KT <= 32 ? 2 : 1;  // heads per TMEM wait, as in the score loop
-#pragma unroll
-          for (int h0 = 0; h0 < G; h0 += HE) {
-            uint32_t v[HE][HALF];
-#pragma unroll
-            for (int u = 0; u < HE; ++u) tmem_ld32(lane_addr + DCOL + (h0 + u) * 64 + hf * HALF, v[u]);
-            tmem_wait_ld();
-#pragma unroll
-            for (int u = 0; u < HE; ++u) {
-              const int hh = h0 + u;
-              float* dst = s_sel + (((long long)b * s.Hq + g * G + hh) * s.N + i) * K;
-              uint32_t rem = sel;
-              for (int k = 0; __any_sync(0xffffffffu, k < nmine); ++k) {
-                const int j = (__ffs(rem) - 1) & 31;  // 31 once this lane has no more (unused)
-                rem &= rem - 1u;
-                const float x = __uint_as_float(pick32(v[u], j));
-                if (k < nmine && base + k < K) {
-                  const float y = __fmaf_rn(x, scale, sm.bt[par][hh][hf * HALF + j]);
-                  if constexpr (kStaged) sval[(hh * KT + base + k) * RS + r] = y;
-                  else dst[base + k] = y;
-                }
-              }
-            }
+            ++slot;
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.dempty);
       }
     }
     if (valid && ok && hf == 0 && nsel != min(ncand, K)) raise_status(ctx, kStatusBadIndex);
