@@ -245,6 +245,35 @@ def test_end_to_end_tiny_sequences():
         _e2e(w, prefill_inputs(w))
 
 
+@pytest.mark.parametrize("K", [8, 32, 48])
+def test_score_exact_ties_take_smaller_chunks(K):
+    """k' = 0 and whole-number b' make every surrogate score exact (s^ = b')
+    and make most group scores tie.  The chosen chunks must then be the
+    oracle's bit for bit: among equal group scores the smaller chunk wins,
+    across the two 32-chunk halves of a tile and across tiles, and each s^ is
+    the chunk's own b'.  K = 8, 32 and 48 cover the three list lengths of the
+    kernel (16, 32, 64) and both ways of writing the result."""
+    w = WORKLOADS["prefill_8k"].scaled(name=f"tie{K}", B=2, N=64 * 300 + 17, Hq=8, Hkv=2, K=K, W=128,
+                                       needles_per_head=0)
+    dm = _dims(w)
+    C = w.N // w.S
+    gen = torch.Generator().manual_seed(101 + K)
+    q = torch.randn((w.B, w.Hq, w.N, w.d), generator=gen).to(torch.bfloat16)
+    b_sum = torch.randint(0, 4, (w.B, w.Hq, C), generator=gen).float()
+    k_sum = torch.zeros((w.B, w.Hq, C, w.d), dtype=torch.bfloat16)
+    idx = torch.empty((w.B, w.Hkv, w.N, K), dtype=torch.int32, device=DEV)
+    s_sel = torch.empty((w.B, w.Hq, w.N, K), dtype=torch.float32, device=DEV)
+    H.hils_score_topk(H.config_of(w), q.to(DEV), k_sum.to(DEV), b_sum.to(DEV), idx, s_sel)
+    H.hils_sync_status()
+    rows = oracle.all_rows(w.B, w.N)
+    idx_o, ssel_o = oracle.select(dm, rows, to_np(q), k_sum=np.zeros((w.B, w.Hq, C, w.d)),
+                                  b_sum=b_sum.numpy().astype(np.float64))
+    got_idx = idx.cpu().numpy().transpose(0, 2, 1, 3).reshape(-1, w.Hkv, K)
+    assert np.array_equal(got_idx, idx_o)
+    got_s = s_sel.cpu().numpy().transpose(0, 2, 1, 3).reshape(-1, w.Hq, K)
+    assert np.array_equal(got_s, ssel_o.astype(np.float32))
+
+
 @pytest.mark.parametrize("stage", ["score", "qcal", "attn"])
 def test_prefill_wait_timeout_reports_status(stage):
     """The kernels that wait on tile copies (scoring, Q-Cal, attention) report a
