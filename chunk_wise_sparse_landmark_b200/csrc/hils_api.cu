@@ -7,6 +7,8 @@
 
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "hils.h"
 #include "launch.h"
 
@@ -257,6 +259,16 @@ hils_status_t get_pipe(int dev, int nev, Pipe** pp) {
     if (_e != cudaSuccess) return cuda_fail(_e, where);     \
   } while (0)
 
+// one NVTX range per C-ABI call, named after the call (a no-op unless a
+// profiler that records NVTX is attached)
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+#define HILS_NVTX NvtxRange hils_nvtx_range_(__func__)
+
 }  // namespace
 }  // namespace hils
 
@@ -274,6 +286,7 @@ void hils_set_fault_injection(int32_t mode) { g_inject = mode == 1 ? 1 : 0; }
 
 hils_status_t hils_build_summaries(const hils_config_t* cfg, const void* k, const void* q_lmk, void* k_sum,
                                    float* b_sum, void* stream) {
+  HILS_NVTX;
   Shape s;
   HILS_TRY(make_shape(cfg, &s, kOpSummaries));
   if (!aligned16(k) || !aligned16(q_lmk) || !aligned16(k_sum) || !aligned16(b_sum))
@@ -288,6 +301,7 @@ hils_status_t hils_build_summaries(const hils_config_t* cfg, const void* k, cons
 
 hils_status_t hils_build_summaries_shared(const hils_config_t* cfg, const void* k, const void* q_shared,
                                           void* k_sum, float* b_sum, void* stream) {
+  HILS_NVTX;
   Shape s;
   HILS_TRY(make_shape(cfg, &s, kOpSummaries));
   if (!aligned16(k) || !aligned16(q_shared) || !aligned16(k_sum) || !aligned16(b_sum))
@@ -338,6 +352,7 @@ size_t hils_workspace_bytes(const hils_config_t* cfg, int32_t which, int32_t qca
 hils_status_t hils_score_topk(const hils_config_t* cfg, const void* q, const hils_qcal_t* qcal, const void* k_sum,
                               const float* b_sum, int32_t* idx, float* s_sel, void* workspace, size_t ws_bytes,
                               int32_t decode, void* stream) {
+  HILS_NVTX;
   Shape s;
   HILS_TRY(make_shape(cfg, &s, decode ? kOpScoreDecode : kOpScorePrefill));
   if (decode != 0 && decode != 1) return fail(HILS_ERR_INVALID_ARG, "decode must be 0 or 1");
@@ -382,6 +397,7 @@ hils_status_t hils_score_topk(const hils_config_t* cfg, const void* q, const hil
 hils_status_t hils_attn_prefill(const hils_config_t* cfg, const void* q, const void* k, const void* v,
                                 const int32_t* idx, const float* s_sel, void* out, void* workspace,
                                 size_t ws_bytes, void* stream) {
+  HILS_NVTX;
   Shape s;
   HILS_TRY(make_shape(cfg, &s, kOpAttnPrefill));
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(s_sel) || !aligned16(out))
@@ -412,6 +428,7 @@ hils_status_t hils_prefill_bwd(const hils_config_t* cfg, const void* q, const vo
                                const void* q_lmk, const int32_t* idx, const float* s_sel, const void* k_sum,
                                const void* dout, float* dq, float* dk, float* dv, float* dq_lmk, float* ds_sel,
                                void* workspace, size_t ws_bytes, void* stream) {
+  HILS_NVTX;
   Shape s;
   HILS_TRY(make_shape(cfg, &s, kOpPrefillBwd));
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_lmk) || !aligned16(idx) || !aligned16(s_sel) ||
@@ -432,6 +449,7 @@ hils_status_t hils_prefill_bwd(const hils_config_t* cfg, const void* q, const vo
 hils_status_t hils_prefill_host(const hils_config_t* cfg, const void* h_q, const void* h_k, const void* h_v,
                                 const void* h_q_lmk, const hils_qcal_t* qcal, void* h_out, void* workspace,
                                 size_t ws_bytes, void* stream) {
+  HILS_NVTX;
   Shape s;
   HILS_TRY(make_shape(cfg, &s, kOpPrefillHost));
   if (!h_q || !h_k || !h_v || !h_q_lmk || !h_out) return fail(HILS_ERR_INVALID_ARG, "hils_prefill_host: NULL host pointer");
@@ -555,6 +573,7 @@ hils_status_t hils_prefill_host(const hils_config_t* cfg, const void* h_q, const
 hils_status_t hils_attn_decode(const hils_config_t* cfg, const void* q, const void* k_cache, const void* v_cache,
                                const int32_t* idx, const float* s_sel, void* out, void* workspace, size_t ws_bytes,
                                void* stream) {
+  HILS_NVTX;
   Shape s;
   HILS_TRY(make_shape(cfg, &s, kOpAttnDecode));
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(idx) || !aligned16(s_sel) ||
@@ -576,6 +595,7 @@ hils_status_t hils_attn_decode(const hils_config_t* cfg, const void* q, const vo
 hils_status_t hils_attn_decode_noalloc(const hils_config_t* cfg, const void* q, const void* k_cache,
                                        const void* v_cache, const int32_t* idx, const float* s_sel, void* out,
                                        void* stream) {
+  HILS_NVTX;
   Shape s;
   HILS_TRY(make_shape(cfg, &s, kOpAttnDecode));
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(idx) || !aligned16(s_sel) ||
@@ -614,6 +634,7 @@ static hils_status_t paged_view(const Shape& s, const hils_paged_t* pg, DecView*
 hils_status_t hils_decode_append(const hils_config_t* cfg, const hils_paged_t* paged, const void* k_new,
                                  const void* v_new, const void* q_lmk_new, void* k_pool, void* v_pool, void* k_sum,
                                  float* b_sum, void* stream) {
+  HILS_NVTX;
   Shape s;
   HILS_TRY(make_shape(cfg, &s, kOpSummaries));
   DecView dv;
@@ -631,6 +652,7 @@ hils_status_t hils_decode_append(const hils_config_t* cfg, const hils_paged_t* p
 
 hils_status_t hils_build_summaries_paged(const hils_config_t* cfg, const hils_paged_t* paged, const void* k_pool,
                                          const void* q_lmk, void* k_sum, float* b_sum, void* stream) {
+  HILS_NVTX;
   Shape s;
   HILS_TRY(make_shape(cfg, &s, kOpSummaries));
   DecView dv;
@@ -647,6 +669,7 @@ hils_status_t hils_build_summaries_paged(const hils_config_t* cfg, const hils_pa
 hils_status_t hils_score_topk_paged(const hils_config_t* cfg, const void* q, const hils_paged_t* paged,
                                     const void* k_sum, const float* b_sum, int32_t* idx, float* s_sel,
                                     void* workspace, size_t ws_bytes, void* stream) {
+  HILS_NVTX;
   Shape s;
   HILS_TRY(make_shape(cfg, &s, kOpScoreDecode));
   DecView dv;
@@ -666,6 +689,7 @@ hils_status_t hils_score_topk_paged(const hils_config_t* cfg, const void* q, con
 hils_status_t hils_attn_decode_paged(const hils_config_t* cfg, const void* q, const void* k_pool, const void* v_pool,
                                      const hils_paged_t* paged, const int32_t* idx, const float* s_sel, void* out,
                                      void* workspace, size_t ws_bytes, void* stream) {
+  HILS_NVTX;
   Shape s;
   HILS_TRY(make_shape(cfg, &s, kOpAttnDecode));
   DecView dv;
@@ -686,6 +710,7 @@ hils_status_t hils_attn_decode_paged(const hils_config_t* cfg, const void* q, co
 }
 
 hils_status_t hils_host_device_pointer(const void* host, void** device_ptr) {
+  HILS_NVTX;
   if (!host || !device_ptr) return fail(HILS_ERR_INVALID_ARG, "hils_host_device_pointer: NULL argument");
   void* p = nullptr;
   const cudaError_t e = cudaHostGetDevicePointer(&p, const_cast<void*>(host), 0);
@@ -699,6 +724,7 @@ hils_status_t hils_host_device_pointer(const void* host, void** device_ptr) {
 }
 
 hils_status_t hils_sync_status(void* stream) {
+  HILS_NVTX;
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
   DevCtx ctx;
