@@ -291,18 +291,24 @@ __global__ void __launch_bounds__(THREADS, 1)
     // et % 64, in two layouts (head-major for pass 1, heads innermost for
     // pass 2); the barrier of the landed vote publishes them.  The buffer of
     // this parity was last read two tiles ago, before the previous vote.
-    auto stage_bias = [&](int t, int par) {
+    auto load_bias = [&](int t) -> float {
       const int bh = et >> 6, bj = et & 63, bc = t * TCH + bj;
-      const float bval = bc < s.C ? __ldg(b_sum + ((long long)b * s.Hq + g * G + bh) * s.C + bc) : 0.f;
+      return bc < s.C ? __ldg(b_sum + ((long long)b * s.Hq + g * G + bh) * s.C + bc) : 0.f;
+    };
+    auto stage_bias = [&](float bval, int par) {
+      const int bh = et >> 6, bj = et & 63;
       sm.bt[par][bh][bj] = bval;
       sm.btj[par][bj][bh] = bval;
     };
+    float bnext = T > 0 ? load_bias(0) : 0.f;  // b' of the next tile, fetched a tile ahead
 
     // pass 1
     for (int it = 0; it < T; ++it) {
       const int t = it, par = it & 1;
       const int c0 = t * TCH + hf * HALF;  // first chunk of this thread's half
-      stage_bias(t, par);
+      const float bval = bnext;
+      bnext = load_bias(t + 1 < T ? t + 1 : 0);  // pass 2 starts again at tile 0
+      stage_bias(bval, par);
       const bool landed = mbar_wait(&sm.dfull, it & 1, ctx);
       if (!epi_all(landed)) {
         ok = false;
@@ -407,7 +413,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int it = T; it < 2 * T && ok; ++it) {
       const int t = it - T, par = it & 1;
       const int c0 = t * TCH + hf * HALF;
-      stage_bias(t, par);
+      const float bval = bnext;
+      if (t + 1 < T) bnext = load_bias(t + 1);
+      stage_bias(bval, par);
       const bool landed = mbar_wait(&sm.dfull, it & 1, ctx);
       if (!epi_all(landed)) {
         ok = false;
