@@ -48,7 +48,8 @@ constexpr int D = 128, G = 4;
 constexpr int MQ = 128;   // positions per CTA (MMA M, TMEM lanes)
 constexpr int TCH = 64;   // chunks per tile (MMA N)
 constexpr int HALF = TCH / 2;
-constexpr int NST = 2;    // k' ring stages (measured: 3 stages were 0.5 ms slower at 128K)
+constexpr int NST = 2;    // k' ring stages (3 measured 0.5 ms slower with an earlier epilogue; beside
+                          // the staging area of K <= 32 they no longer fit in shared memory)
 constexpr int KMAX = 64;
 constexpr int NMMA = G;   // MMA-issuing warps, one per head
 constexpr int EPI = 256;  // epilogue threads
@@ -531,6 +532,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 template <int KT>
 constexpr size_t kSmemBytes = sizeof(SmemS<KT>) + 1024;
+static_assert(kSmemBytes<16> <= 232448 && kSmemBytes<32> <= 232448 && kSmemBytes<64> <= 232448,
+              "score kernel shared memory above the 227 KB a CTA may use");
 
 template <int KT>
 cudaError_t launch_kt(const Shape& s, const CUtensorMap& tmk, const void* q, const float* b_sum, int32_t* idx,
